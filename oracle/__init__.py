@@ -1,0 +1,164 @@
+"""CPU oracle for the KroQuant online activation quantizer (ctypes binding).
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, the package smoke
+check (``__graft_entry__.smoke``) and the benchmark's CPU-baseline leg may
+import this package.  The product path never routes through it.
+
+Every function takes and returns numpy arrays; the arithmetic lives in
+``kq_oracle.c`` (plain scalar C, double precision), whose header lists the
+sources and the readings it follows.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        p = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        ci = ctypes.c_int
+        L.oracle_abi_version.restype = ci
+        L.oracle_num_threads.restype = ci
+        L.oracle_set_threads.argtypes = [ci]
+        L.oracle_kron_expand.argtypes = [p, p]
+        L.oracle_inverse32.argtypes = [p, p]
+        L.oracle_inverse32.restype = ci
+        L.oracle_e8m0.argtypes = [ctypes.c_float]
+        L.oracle_e8m0.restype = ctypes.c_uint8
+        L.oracle_e2m1.argtypes = [ctypes.c_double]
+        L.oracle_e2m1.restype = ctypes.c_uint8
+        L.oracle_mx_block.argtypes = [p, p, p]
+        L.oracle_kq_transform.argtypes = [p, p, ci, i64, i64, p, p]
+        L.oracle_kq_transform.restype = ci
+        L.oracle_kq_quantize.argtypes = [p, p, ci, i64, i64, p, p]
+        L.oracle_kq_quantize.restype = ci
+        L.oracle_sq_quantize.argtypes = [p, p, i64, i64, p, p]
+        L.oracle_sq_quantize.restype = ci
+        L.oracle_mx_quantize.argtypes = [p, i64, i64, p, p]
+        L.oracle_mx_quantize.restype = ci
+        L.oracle_fold_weights.argtypes = [p, p, ci, p, p, i64, i64]
+        L.oracle_fold_weights.restype = ci
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def set_threads(n: int) -> None:
+    lib().oracle_set_threads(int(n))
+
+
+def kron_expand(F):
+    """Dense 32x32 K = G1 (x) ... (x) G5 (float64) from a [5,2,2] float32 factor set."""
+    F = _c(F, np.float32).reshape(5, 2, 2)
+    K = np.empty((32, 32), np.float64)
+    lib().oracle_kron_expand(_ptr(F), _ptr(K))
+    return K
+
+
+def inverse32(A):
+    A = _c(A, np.float64).reshape(32, 32)
+    out = np.empty((32, 32), np.float64)
+    if lib().oracle_inverse32(_ptr(A), _ptr(out)) != 0:
+        raise ValueError("singular 32x32 matrix")
+    return out
+
+
+def e8m0(amax: float) -> int:
+    return int(lib().oracle_e8m0(float(amax)))
+
+
+def e2m1(v: float) -> int:
+    return int(lib().oracle_e2m1(float(v)))
+
+
+def mx_block(y):
+    y = _c(y, np.float32).reshape(32)
+    codes = np.empty(16, np.uint8)
+    scale = np.empty(1, np.uint8)
+    lib().oracle_mx_block(_ptr(y), _ptr(codes), _ptr(scale))
+    return codes, int(scale[0])
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} failed with status {rc}")
+
+
+def _shape(x):
+    if x.ndim != 2:
+        raise ValueError("activation must be 2-D [M, d]")
+    return x.shape
+
+
+def kq_transform(x_bf16, factors, shared=False, want_absbound=False):
+    """fp32 y = T x per block (dense, double, rounded once), optionally with |K||x|."""
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    f = _c(factors, np.float32)
+    y = np.empty((M, d), np.float32)
+    ab = np.empty((M, d), np.float64) if want_absbound else None
+    _check(lib().oracle_kq_transform(_ptr(x), _ptr(f), int(bool(shared)), M, d, _ptr(y), _ptr(ab)),
+           "kq_transform")
+    return (y, ab) if want_absbound else y
+
+
+def kq_quantize(x_bf16, factors, shared=False):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    f = _c(factors, np.float32)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_kq_quantize(_ptr(x), _ptr(f), int(bool(shared)), M, d, _ptr(codes), _ptr(scales)),
+           "kq_quantize")
+    return codes, scales
+
+
+def sq_quantize(x_bf16, mult):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    m = _c(mult, np.float32)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_sq_quantize(_ptr(x), _ptr(m), M, d, _ptr(codes), _ptr(scales)), "sq_quantize")
+    return codes, scales
+
+
+def mx_quantize(x_bf16):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_mx_quantize(_ptr(x), M, d, _ptr(codes), _ptr(scales)), "mx_quantize")
+    return codes, scales
+
+
+def fold_weights(W, factors, shared=False, want_absbound=False):
+    """W' = W T^-1 (fp32 result of a double computation), optionally with |W||K^-1|."""
+    W = _c(W, np.float32)
+    N, d = _shape(W)
+    f = _c(factors, np.float32)
+    out = np.empty((N, d), np.float32)
+    ab = np.empty((N, d), np.float64) if want_absbound else None
+    _check(lib().oracle_fold_weights(_ptr(W), _ptr(f), int(bool(shared)), _ptr(out), _ptr(ab), N, d),
+           "fold_weights")
+    return (out, ab) if want_absbound else out

@@ -1,0 +1,350 @@
+/*
+ * kq_oracle.c -- plain, slow, scalar CPU oracle for the KroQuant online
+ * activation quantizer and its two baselines.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test-suite, the package
+ * smoke check and the benchmark's CPU-baseline leg may load or call this
+ * library.  It shares no code, header, table or helper with the CUDA path.
+ *
+ * Sources (cited by tag below):
+ *   [KQ-abs]   "KroQuant: Kronecker-Structured Block Transforms for Efficient
+ *              Post-Training Quantization of Diffusion Transformers"
+ *              (arXiv 2607.21446), abstract: a learned invertible transform is
+ *              applied to every 32-element block of each activation row, the
+ *              result is quantized to MXFP4 (W4A4, "MXFP4e2"); SmoothQuant
+ *              per-channel scaling is the cheap baseline.
+ *   [KQ-Eq4]   Pith review of arXiv 2607.21446, skeptic critique on paper
+ *              section 3.2, Eq. (4), and "key machinery": T is block diagonal,
+ *              each 32x32 block K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5 with 2x2 G_k;
+ *              the inverse is folded into the weights offline.
+ *   [OCP-MX]   OCP Microscaling Formats (MX) Specification v1.0, section 6.3
+ *              (the MXFP4 block-32 conversion): shared scale
+ *              2^(floor(log2(amax)) - emax_elem) with emax_elem = 2 for E2M1,
+ *              stored as E8M0 (biased by 127); elements FP4 E2M1 with values
+ *              {0, 0.5, 1, 1.5, 2, 3, 4, 6}, round-to-nearest-even, saturating.
+ *
+ * Readings taken where the sources are silent (each one is listed in the
+ * design notes of the repository):
+ *   R1 Kronecker index order is the textbook one:
+ *      (A (x) B)[i*m + p][l*m + q] = A[i][l] * B[p][q], so G1 acts on bit 4
+ *      (the most significant bit) of the in-block index and G5 on bit 0.
+ *   R2 y = T x is evaluated once in double and rounded once to fp32; the block
+ *      amax is taken over those fp32 values.
+ *   R3 amax == 0 gives the clamped exponent -127 (scale byte 0x00); a block
+ *      with a non-finite value gets scale byte 0xFF (out of contract).
+ *   R4 The sign of an e2m1 code follows the sign bit of the scaled value, as
+ *      IEEE rounding does, so a negative value that rounds to zero gives the
+ *      code 0x8 ("-0").
+ *   R5 Two codes per byte, the even element in the low nibble.
+ *   R6 Factor storage: factors[j][k][r][c] (float32, 20 per block column j),
+ *      k = 0..4 is G1..G5; "shared" mode uses one set for every column.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define BLK 32
+
+int oracle_abi_version(void) { return 1; }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* A bf16 value is the upper 16 bits of an IEEE binary32. */
+static double bf16_value(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* [KQ-Eq4] + R1: K[i][l] = prod_k G_k[bit_(4-k)(i)][bit_(4-k)(l)], in double. */
+void oracle_kron_expand(const float *F /* [5][2][2] */, double *K /* [32][32] */)
+{
+    for (int i = 0; i < BLK; ++i) {
+        for (int l = 0; l < BLK; ++l) {
+            double p = 1.0;
+            for (int k = 0; k < 5; ++k) {
+                int bi = (i >> (4 - k)) & 1;
+                int bl = (l >> (4 - k)) & 1;
+                p *= (double)F[k * 4 + bi * 2 + bl];
+            }
+            K[i * BLK + l] = p;
+        }
+    }
+}
+
+/* Dense inverse of a 32x32 matrix by Gauss-Jordan elimination with partial
+ * pivoting, in double.  Returns 0 on success, -1 if a pivot is exactly 0. */
+int oracle_inverse32(const double *A, double *Ainv)
+{
+    double a[BLK][2 * BLK];
+    for (int i = 0; i < BLK; ++i) {
+        for (int j = 0; j < BLK; ++j) {
+            a[i][j] = A[i * BLK + j];
+            a[i][BLK + j] = (i == j) ? 1.0 : 0.0;
+        }
+    }
+    for (int c = 0; c < BLK; ++c) {
+        int piv = c;
+        for (int r = c + 1; r < BLK; ++r)
+            if (fabs(a[r][c]) > fabs(a[piv][c])) piv = r;
+        if (a[piv][c] == 0.0) return -1;
+        if (piv != c) {
+            for (int j = 0; j < 2 * BLK; ++j) {
+                double t = a[c][j];
+                a[c][j] = a[piv][j];
+                a[piv][j] = t;
+            }
+        }
+        double inv = 1.0 / a[c][c];
+        for (int j = 0; j < 2 * BLK; ++j) a[c][j] *= inv;
+        for (int r = 0; r < BLK; ++r) {
+            if (r == c) continue;
+            double f = a[r][c];
+            if (f == 0.0) continue;
+            for (int j = 0; j < 2 * BLK; ++j) a[r][j] -= f * a[c][j];
+        }
+    }
+    for (int i = 0; i < BLK; ++i)
+        for (int j = 0; j < BLK; ++j) Ainv[i * BLK + j] = a[i][BLK + j];
+    return 0;
+}
+
+/* [OCP-MX] E8M0 shared-scale byte from the block amax (fp32), with R3.
+ * floor(log2(amax)) is read off frexp exactly (no log2 call):
+ * amax = m * 2^ex with 0.5 <= m < 1, so floor(log2(amax)) = ex - 1. */
+uint8_t oracle_e8m0(float amax)
+{
+    if (!isfinite(amax)) return 0xFF;
+    if (amax == 0.0f) return 0x00;
+    int ex = 0;
+    (void)frexp((double)amax, &ex);
+    int e = (ex - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/* [OCP-MX] FP4 E2M1 code of a scaled value: nearest grid magnitude by brute
+ * force; on an exact tie the even code (magnitude LSB 0) wins; magnitudes
+ * beyond 6 land on 6 (saturation); sign from the sign bit (R4). */
+static const double E2M1_GRID[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+uint8_t oracle_e2m1(double v)
+{
+    double a = fabs(v);
+    int best = 0;
+    double bestd = fabs(a - E2M1_GRID[0]);
+    for (int k = 1; k < 8; ++k) {
+        double dk = fabs(a - E2M1_GRID[k]);
+        if (dk < bestd || (dk == bestd && (k & 1) == 0)) {
+            best = k;
+            bestd = dk;
+        }
+    }
+    uint8_t code = (uint8_t)best;
+    if (signbit(v)) code |= 0x8;
+    return code;
+}
+
+/* [OCP-MX] one 32-element block: amax over |y|, E8M0 byte, scaled values
+ * v = y * 2^-e (exact in double), E2M1 codes packed two per byte (R5). */
+void oracle_mx_block(const float *y /* [32] */, uint8_t *codes /* [16] */, uint8_t *scale)
+{
+    float amax = 0.0f;
+    int finite = 1;
+    for (int i = 0; i < BLK; ++i) {
+        if (!isfinite(y[i])) finite = 0;
+        float a = fabsf(y[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t sb = finite ? oracle_e8m0(amax) : 0xFF;
+    *scale = sb;
+    if (sb == 0xFF) {
+        memset(codes, 0, BLK / 2);
+        return;
+    }
+    int e = (int)sb - 127;
+    uint8_t c[BLK];
+    for (int i = 0; i < BLK; ++i) c[i] = oracle_e2m1(ldexp((double)y[i], -e));
+    for (int b = 0; b < BLK / 2; ++b)
+        codes[b] = (uint8_t)(c[2 * b] | (c[2 * b + 1] << 4));
+}
+
+/* Expand every column's K^(j) once (nb x 1024 doubles). */
+static double *expand_all(const float *factors, int shared, int64_t nb)
+{
+    int64_t ncol = shared ? 1 : nb;
+    double *K = (double *)malloc((size_t)ncol * BLK * BLK * sizeof(double));
+    if (!K) return NULL;
+    for (int64_t j = 0; j < ncol; ++j) oracle_kron_expand(factors + j * 20, K + j * BLK * BLK);
+    return K;
+}
+
+/* [KQ-abs], [KQ-Eq4]: y = T x per 32-block of every row, dense matvec with the
+ * expanded K^(j) summed in double and rounded once to fp32 (R2).  If absb is
+ * not NULL it receives (|K^(j)| |x|)_i, the scale of the dot product's
+ * rounding error, used by tests to form tolerances. */
+int oracle_kq_transform(const uint16_t *x, const float *factors, int shared,
+                        int64_t M, int64_t d, float *y, double *absb)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+    double *K = expand_all(factors, shared, nb);
+    if (!K) return -5;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kj = K + (shared ? 0 : j) * BLK * BLK;
+            const uint16_t *xb = x + r * d + j * BLK;
+            double xv[BLK];
+            for (int l = 0; l < BLK; ++l) xv[l] = bf16_value(xb[l]);
+            for (int i = 0; i < BLK; ++i) {
+                double s = 0.0, sa = 0.0;
+                for (int l = 0; l < BLK; ++l) {
+                    s += Kj[i * BLK + l] * xv[l];
+                    sa += fabs(Kj[i * BLK + l]) * fabs(xv[l]);
+                }
+                y[r * d + j * BLK + i] = (float)s;
+                if (absb) absb[r * d + j * BLK + i] = sa;
+            }
+        }
+    }
+    free(K);
+    return 0;
+}
+
+/* The KroQuant quantizer: transform (above), then the MX block quantizer. */
+int oracle_kq_quantize(const uint16_t *x, const float *factors, int shared,
+                       int64_t M, int64_t d, uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+    double *K = expand_all(factors, shared, nb);
+    if (!K) return -5;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kj = K + (shared ? 0 : j) * BLK * BLK;
+            const uint16_t *xb = x + r * d + j * BLK;
+            double xv[BLK];
+            float yv[BLK];
+            for (int l = 0; l < BLK; ++l) xv[l] = bf16_value(xb[l]);
+            for (int i = 0; i < BLK; ++i) {
+                double s = 0.0;
+                for (int l = 0; l < BLK; ++l) s += Kj[i * BLK + l] * xv[l];
+                yv[i] = (float)s;
+            }
+            oracle_mx_block(yv, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+        }
+    }
+    free(K);
+    return 0;
+}
+
+/* [KQ-abs] SmoothQuant baseline: y_c = fp32(x_c * m_c) with the per-channel
+ * multiplier m_c = 1/s_c given as input, then the MX block quantizer.  The
+ * product of a bf16 and an fp32 value is exact in double, so the single
+ * rounding to fp32 is the correctly rounded fp32 product. */
+int oracle_sq_quantize(const uint16_t *x, const float *mult, int64_t M, int64_t d,
+                       uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < nb; ++j) {
+            float yv[BLK];
+            for (int i = 0; i < BLK; ++i) {
+                int64_t c = j * BLK + i;
+                yv[i] = (float)(bf16_value(x[r * d + c]) * (double)mult[c]);
+            }
+            oracle_mx_block(yv, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+        }
+    }
+    return 0;
+}
+
+/* Plain MXFP4 baseline: no transform, the MX block quantizer on x itself. */
+int oracle_mx_quantize(const uint16_t *x, int64_t M, int64_t d, uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < nb; ++j) {
+            float yv[BLK];
+            for (int i = 0; i < BLK; ++i) yv[i] = (float)bf16_value(x[r * d + j * BLK + i]);
+            oracle_mx_block(yv, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+        }
+    }
+    return 0;
+}
+
+/* [KQ-Eq4] offline fold of the inverse into the weights: W' = W T^-1, i.e.
+ * for every row n and column block j, W'[n, blk j] = W[n, blk j] K^(j)^-1,
+ * with K^(j)^-1 the Gauss-Jordan inverse of the dense expansion.  Summed in
+ * double, rounded once to fp32.  If absb is not NULL it receives
+ * (|W[n, blk j]| |K^(j)^-1|)_c for tolerances.  Returns -3 if some K^(j) is
+ * singular. */
+int oracle_fold_weights(const float *W, const float *factors, int shared,
+                        float *Wout, double *absb, int64_t N, int64_t d)
+{
+    if (d % BLK != 0 || N < 0) return -2;
+    int64_t nb = d / BLK;
+    int64_t ncol = shared ? 1 : nb;
+    double *K = expand_all(factors, shared, nb);
+    if (!K) return -5;
+    double *Ki = (double *)malloc((size_t)ncol * BLK * BLK * sizeof(double));
+    if (!Ki) {
+        free(K);
+        return -5;
+    }
+    int bad = 0;
+    for (int64_t j = 0; j < ncol; ++j)
+        if (oracle_inverse32(K + j * BLK * BLK, Ki + j * BLK * BLK) != 0) bad = 1;
+    free(K);
+    if (bad) {
+        free(Ki);
+        return -3;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kij = Ki + (shared ? 0 : j) * BLK * BLK;
+            const float *w = W + n * d + j * BLK;
+            for (int c = 0; c < BLK; ++c) {
+                double s = 0.0, sa = 0.0;
+                for (int r = 0; r < BLK; ++r) {
+                    s += (double)w[r] * Kij[r * BLK + c];
+                    sa += fabs((double)w[r]) * fabs(Kij[r * BLK + c]);
+                }
+                Wout[n * d + j * BLK + c] = (float)s;
+                if (absb) absb[n * d + j * BLK + c] = sa;
+            }
+        }
+    }
+    free(Ki);
+    return 0;
+}
