@@ -1,0 +1,675 @@
+#!/usr/bin/env python3
+"""Benchmark of the KroQuant online activation quantizer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the KroQuant
+quantizer, the SmoothQuant quantizer and the plain MXFP4 quantizer, each on
+both PixArt-Sigma layer inputs (M = 8192 tokens x d = 1152 and d = 4608, bf16,
+seeded synthetic activations).  The headline value is the KroQuant quantizer's
+algorithmic HBM throughput, 2.53125 bytes per element (2 B bf16 in, 0.5 B
+codes, 1/32 B scale) over the summed duration of its launches.
+
+Timing: inputs resident in HBM, rotated over 8 input sets (each launch reads a
+set that the previous 7 quantizer passes did not touch, > 6x the L2), launches
+captured in a CUDA graph of 200 steps and replayed; CUDA events on the
+launching stream bracket every launch of the last replay and the whole timed
+region; barrier + synchronize on both sides; max over ranks.  Multi-GPU: every
+rank quantizes its own batch (weak scaling, no collective on the data path).
+
+`--impl reference` times the CPU oracle (oracle/, plain C) on the host cores on
+a bounded sample of the same workload and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KroQuant quantizer HBM GB/s (bf16→MXFP4+E8M0) and % of B200 peak vs SQ"
+BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
+WORKLOAD = "pixart"
+N_SETS = 8
+GRAPH_STEPS = 200          # a multiple of 8 so the set rotation is seamless across replays
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.cu")]
+
+# DRAM traffic per launch of the dominant kernel (KroQuant quantizer, d = 4608
+# layer), from one ncu capture, valid only for the kernel source it was taken
+# on (sha256 prefix of the .cu sources).  Updated after each capture.
+TRAFFIC = {"source_sha": None, "bytes_per_launch": None, "capture": None}
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            v = float(json.load(fh)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier pool measurement)"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self._t:
+            self._t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [t.strip() for t in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch
+
+        torch.cuda.set_device(local)
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return rank, local, world, pg
+
+
+def allreduce_max(pg, values, device):
+    if pg is None:
+        return values
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ----------------------------------------------------------------------------- inputs
+def workload_inputs(seed_offset: int = 0):
+    from w4a4_mxfp4_post_b200 import synth
+
+    layers = []
+    for (M, d, model, shared, seed) in synth.workload_layers(WORKLOAD):
+        x = synth.activation(model, M, d, seed + seed_offset)
+        F = synth.factors(d // 32, seed + seed_offset, shared=shared)
+        m = synth.sq_multipliers(x)
+        layers.append({"M": M, "d": d, "x": x, "F": F, "m": m, "shared": shared})
+    return layers
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(layers, seconds: float, rows_per_pass=None):
+    """Run the oracle (KQ, SQ, MX on every layer) over row samples for ~`seconds`."""
+    import oracle
+
+    t_kq = 0.0
+    t_all = 0.0
+    kq_bytes = 0.0
+    passes = 0
+    start = time.perf_counter()
+    while True:
+        for L in layers:
+            M = L["M"] if rows_per_pass is None else min(L["M"], rows_per_pass)
+            x = L["x"][:M]
+            t0 = time.perf_counter()
+            oracle.kq_quantize(x, L["F"], shared=L["shared"])
+            t1 = time.perf_counter()
+            oracle.sq_quantize(x, L["m"])
+            oracle.mx_quantize(x)
+            t2 = time.perf_counter()
+            t_kq += t1 - t0
+            t_all += t2 - t0
+            kq_bytes += BYTES_PER_ELEM * M * L["d"]
+        passes += 1
+        if time.perf_counter() - start >= seconds:
+            break
+    return {"kq_gbs": kq_bytes / t_kq / 1e9, "passes": passes, "t_kq": t_kq, "t_all": t_all,
+            "threads": oracle.num_threads()}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def gpu_arm(args, rank, local, world, pg):
+    import torch
+
+    import w4a4_mxfp4_post_b200 as kq
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    layers = workload_inputs(seed_offset=rank)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+
+    # device buffers: N_SETS copies of every layer input, per-set outputs
+    sets = []
+    for s in range(N_SETS):
+        per = []
+        for L in layers:
+            M, d = L["M"], L["d"]
+            x = torch.from_numpy(L["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+            per.append({
+                "x": x,
+                "F": torch.from_numpy(L["F"]).to(dev),
+                "m": torch.from_numpy(L["m"]).to(dev),
+                "codes": torch.empty((M, d // 2), dtype=torch.uint8, device=dev),
+                "scales": torch.empty((M, d // 32), dtype=torch.uint8, device=dev),
+                "shared": L["shared"],
+            })
+        sets.append(per)
+    set_bytes = sum(L["M"] * L["d"] * 2 for L in layers)
+
+    def kq_call(b, stream):
+        fn = kq.kq_quantize_shared if b["shared"] else kq.kq_quantize
+        fn(b["x"], b["F"], b["codes"], b["scales"], stream=stream)
+
+    def sq_call(b, stream):
+        kq.sq_quantize(b["x"], b["m"], b["codes"], b["scales"], stream=stream)
+
+    def mx_call(b, stream):
+        kq.mx_quantize(b["x"], b["codes"], b["scales"], stream=stream)
+
+    quantizers = [("kq", kq_call), ("sq", sq_call), ("mx", mx_call)]
+    n_layers = len(layers)
+
+    def step(i, stream, events=None):
+        # quantizer q of step i reads set (3 i + q) mod 8
+        k = 0
+        for q, (name, fn) in enumerate(quantizers):
+            for li in range(n_layers):
+                b = sets[(3 * i + q) % N_SETS][li]
+                fn(b, stream)
+                if events is not None:
+                    events[k + 1].record(stream)
+                k += 1
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    # warm-up (eager)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+
+    # capture S steps with an event after every launch (events of the last replay are read)
+    K = args.steps
+    S = min(GRAPH_STEPS, K)
+    reps, tail = divmod(K, S)
+    n_launch = 3 * n_layers
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_launch + 1)] for _ in range(S)]
+
+    def capture(nsteps, with_events):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(nsteps):
+                if with_events:
+                    ev[i][0].record(stream)
+                step(i, stream, ev[i] if with_events else None)
+        return g
+
+    g_main = capture(S, True)
+    g_tail = capture(tail, False) if tail else None
+    g_main.replay()
+    if g_tail:
+        g_tail.replay()
+    stream.synchronize()
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    uuid = getattr(props, "uuid", None)
+    gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
+    clocks = ClockSampler(gpu_id) if rank == 0 else None
+    barrier(pg)
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t_start.record(stream)
+    for _ in range(reps):
+        g_main.replay()
+    if g_tail:
+        g_tail.replay()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(pg)
+    clk = clocks.stop() if clocks else None
+
+    total_ms = t_start.elapsed_time(t_end)
+    # per-launch durations of the last main replay
+    per = {name: [0.0] * n_layers for name, _ in quantizers}
+    for i in range(S):
+        k = 0
+        for name, _ in quantizers:
+            for li in range(n_layers):
+                per[name][li] += ev[i][k].elapsed_time(ev[i][k + 1])
+                k += 1
+    us = {name: [1e3 * v / S for v in per[name]] for name in per}     # mean us per launch
+    step_ms = total_ms / K
+
+    # kernel-only quantizer throughput from the per-launch means
+    elems = [L["M"] * L["d"] for L in layers]
+    qbytes = sum(BYTES_PER_ELEM * e for e in elems)
+    q_time_us = {name: sum(us[name]) for name in us}
+    vals = allreduce_max(pg, [total_ms] + [q_time_us[n] for n in ("kq", "sq", "mx")] + us["kq"], dev)
+    total_ms_max = vals[0]
+    qt = dict(zip(("kq", "sq", "mx"), vals[1:4]))
+    kq_us_max = vals[4:]
+    gbs = {n: world * qbytes / (qt[n] * 1e-6) / 1e9 for n in qt}
+
+    # dominant kernel: the KroQuant launch on the largest layer
+    dom = int(np.argmax(elems))
+    dom_bytes = BYTES_PER_ELEM * elems[dom]
+    peak, peak_src = measured_peak()
+    achieved = dom_bytes / (kq_us_max[dom] * 1e-6) / 1e9
+    sha = source_sha()
+    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["source_sha"] == sha else None
+
+    # end-to-end: pinned host input -> device -> kq_quantize -> host codes + scales
+    e2e = e2e_kq(args, layers, dev, stream, kq, pg, world)
+
+    out = {
+        "metric": METRIC,
+        "value": round(gbs["kq"], 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded PixArt-Sigma-shaped activations with per-channel outliers; no trained weights)",
+        "config": {
+            "workload": "PixArt-Sigma layer inputs: M=8192 tokens x d in {1152, 4608}, bf16 -> MXFP4 (E2M1 codes + "
+                        "E8M0 scales), per-block Kronecker factors",
+            "M": layers[0]["M"], "d": [L["d"] for L in layers], "quantizers_per_step": ["kq", "sq", "mx"],
+            "l2": f"rotating {N_SETS} input sets ({N_SETS * set_bytes / 2**20:.0f} MiB, L2 {l2 / 2**20:.0f} MiB); "
+                  "each launch reads a set untouched by the previous 7 quantizer passes",
+            "timing": f"CUDA graph of {S} steps replayed; events around every launch of the last replay",
+            "parallelism": f"dp{world} (independent batches, no collective)",
+        },
+        "kernels": {
+            n: {"gbs": round(gbs[n], 1), "frac_of_peak": round(gbs[n] / peak, 4),
+                "frac_of_8tbs_spec": round(gbs[n] / SPEC_HBM_GBS, 4),
+                "us_per_launch": {str(L["d"]): round(v, 3) for L, v in zip(layers, us[n])}}
+            for n in ("kq", "sq", "mx")
+        },
+        "kq_time_vs_sq": round(qt["kq"] / qt["sq"], 4),
+        "roofline": {"bound": "hbm", "kernel": f"kq_quantize d={layers[dom]['d']}", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src},
+        "e2e": e2e,
+        "gpu_launches": K * n_launch,
+        "clocks": clk,
+        "kernel_source_sha": sha,
+    }
+    return out
+
+
+def e2e_kq(args, layers, dev, stream, kq, pg, world):
+    """KroQuant through the public API with host buffers: H2D, quantize, D2H, per step."""
+    import torch
+
+    host = []
+    for L in layers:
+        M, d = L["M"], L["d"]
+        host.append({
+            "x": torch.from_numpy(L["x"].view(np.int16)).view(torch.bfloat16).pin_memory(),
+            "codes": torch.empty((M, d // 2), dtype=torch.uint8).pin_memory(),
+            "scales": torch.empty((M, d // 32), dtype=torch.uint8).pin_memory(),
+            "dx": torch.empty((M, d), dtype=torch.bfloat16, device=dev),
+            "dc": torch.empty((M, d // 2), dtype=torch.uint8, device=dev),
+            "ds": torch.empty((M, d // 32), dtype=torch.uint8, device=dev),
+            "F": torch.from_numpy(L["F"]).to(dev), "shared": L["shared"],
+        })
+
+    def one():
+        for h in host:
+            h["dx"].copy_(h["x"], non_blocking=True)
+            fn = kq.kq_quantize_shared if h["shared"] else kq.kq_quantize
+            fn(h["dx"], h["F"], h["dc"], h["ds"], stream=stream)
+            h["codes"].copy_(h["dc"], non_blocking=True)
+            h["scales"].copy_(h["ds"], non_blocking=True)
+
+    n = max(3, min(args.e2e_steps, args.steps))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+        stream.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier(pg)
+        a.record(stream)
+        for _ in range(n):
+            one()
+        b.record(stream)
+        b.synchronize()
+    ms = allreduce_max(pg, [a.elapsed_time(b)], dev)[0]
+    elems = sum(L["M"] * L["d"] for L in layers)
+    h2d = sum(L["M"] * L["d"] * 2 for L in layers)
+    d2h = sum(L["M"] * (L["d"] // 2 + L["d"] // 32) for L in layers)
+    return {"value": round(world * BYTES_PER_ELEM * elems * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "path": "pinned host bf16 -> cudaMemcpyAsync -> kq_quantize -> cudaMemcpyAsync -> pinned host"}
+
+
+def cpu_baseline_block(layers, seconds):
+    r = time_oracle(layers, seconds)
+    return {"value": round(r["kq_gbs"], 4), "unit": "GB/s", "cores": r["threads"], "kind": "oracle",
+            "sample": f"{r['passes']} full passes of the workload (KQ, SQ, MX on both layers), "
+                      f"{r['t_all']:.1f} s of oracle time; value = KQ bytes / KQ time"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference_arm(args, rank, world):
+    """The CPU oracle as the reference implementation, on the host cores."""
+    import oracle
+
+    if rank != 0:
+        return None
+    layers = workload_inputs()
+    oracle.kq_quantize(layers[0]["x"][:8], layers[0]["F"])         # load / warm
+    # rows per step so that (warmup + steps) steps take about `budget` seconds
+    t0 = time.perf_counter()
+    probe = time_oracle(layers, 0.0, rows_per_pass=64)
+    per_row = (time.perf_counter() - t0) / 64
+    budget = args.ref_seconds
+    rows = int(max(1, min(layers[0]["M"], budget / max(1, args.steps + args.warmup) / per_row)))
+    for _ in range(args.warmup):
+        time_oracle(layers, 0.0, rows_per_pass=rows)
+    t_kq = 0.0
+    kq_bytes = 0.0
+    t_all = 0.0
+    for _ in range(args.steps):
+        r = time_oracle(layers, 0.0, rows_per_pass=rows)
+        t_kq += r["t_kq"]
+        t_all += r["t_all"]
+        kq_bytes += sum(BYTES_PER_ELEM * min(L["M"], rows) * L["d"] for L in layers)
+    value = kq_bytes / t_kq / 1e9
+    del probe
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * t_all / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": "PixArt-Sigma layer inputs: M=8192 tokens x d in {1152, 4608}, bf16 -> MXFP4",
+                   "sample_rows_per_layer_per_step": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{rows} rows of each layer per step (KQ, SQ, MX), {args.steps} steps"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+class RotatingInputs:
+    """Device inputs of one [M, d] layer, split into sets that rotate past the L2.
+
+    One allocation holds `nsets` disjoint input sets (and their outputs) whose
+    total is >= 3x the L2, capped by `budget_bytes`; launch i reads set
+    i mod nsets, so no launch finds its input in the L2 from an earlier one.
+    """
+
+    def __init__(self, M, d, dev, l2, budget_bytes=None):
+        import torch
+
+        from w4a4_mxfp4_post_b200 import synth
+
+        self.M, self.d = M, d
+        x = synth.activation("pixart", M, d, 4)
+        F = synth.factors(d // 32, 4)
+        m = synth.sq_multipliers(x)
+        set_bytes = M * d * 2 + M * (d // 2) + M * (d // 32)
+        budget = budget_bytes or max(3 * l2, 2 * set_bytes)
+        self.nsets = max(2, min(1024, math.ceil(budget / set_bytes)))
+        self.xs = torch.empty((self.nsets, M, d), dtype=torch.bfloat16, device=dev)
+        self.xs[:] = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.cs = torch.empty((self.nsets, M, d // 2), dtype=torch.uint8, device=dev)
+        self.ss = torch.empty((self.nsets, M, d // 32), dtype=torch.uint8, device=dev)
+        self.F = torch.from_numpy(F).to(dev)
+        self.m = torch.from_numpy(m).to(dev)
+
+
+def time_launches(kind, inp, launches, warmup, stream, graph=True):
+    """Mean / median device time (us) of one quantizer launch over `launches` launches.
+
+    With graph=True the launches are captured in a CUDA graph with an event
+    after each one; the second replay is measured.
+    """
+    import torch
+
+    import w4a4_mxfp4_post_b200 as kq
+
+    def launch(i):
+        k = i % inp.nsets
+        if kind == "kq":
+            kq.kq_quantize(inp.xs[k], inp.F, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind == "sq":
+            kq.sq_quantize(inp.xs[k], inp.m, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind == "mx":
+            kq.mx_quantize(inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
+        elif kind.startswith("kq_v"):
+            kq.kq_quantize_variant(int(kind[4:]), inp.xs[k], inp.F, False, inp.cs[k], inp.ss[k], stream=stream)
+        else:
+            raise ValueError(f"unknown kernel {kind!r}")
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            launch(i)
+    stream.synchronize()
+    evs = [torch.cuda.Event(enable_timing=True, external=graph) for _ in range(launches + 1)]
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            evs[0].record(stream)
+            for i in range(launches):
+                launch(i)
+                evs[i + 1].record(stream)
+        g.replay()
+        stream.synchronize()
+        g.replay()
+    else:
+        with torch.cuda.stream(stream):
+            evs[0].record(stream)
+            for i in range(launches):
+                launch(i)
+                evs[i + 1].record(stream)
+    stream.synchronize()
+    times = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(launches)]
+    return {"mean_us": float(np.mean(times)), "median_us": float(np.median(times)), "nsets": inp.nsets}
+
+
+def kernel_mode(args):
+    """One quantizer at one shape (the small committed case for ncu captures)."""
+    import torch
+
+    from w4a4_mxfp4_post_b200 import build
+
+    build.build()
+    dev = torch.device("cuda:0")
+    M, d = (int(t) for t in args.shape.lower().split("x"))
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    inp = RotatingInputs(M, d, dev, l2, budget_bytes=args.budget_mb * 2 ** 20 if args.budget_mb else None)
+    r = time_launches(args.kernel, inp, args.launches, args.warmup, torch.cuda.Stream(device=dev),
+                      graph=not args.no_graph)
+    gbs = BYTES_PER_ELEM * M * d / (r["mean_us"] * 1e-6) / 1e9
+    peak, src = measured_peak()
+    print(json.dumps({"mode": "kernel", "kernel": args.kernel, "M": M, "d": d, **r, "gbs": round(gbs, 1),
+                      "frac_of_peak": round(gbs / peak, 4), "peak": peak, "peak_source": src}), flush=True)
+
+
+def sweep_mode(args):
+    """Bandwidth sweep: every quantizer at every (M, d) of the sweep workload."""
+    import torch
+
+    from w4a4_mxfp4_post_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda:0")
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    peak, src = measured_peak()
+    rows = []
+    kinds = args.kernels.split(",")
+    stream = torch.cuda.Stream(device=dev)
+    for M in synth.WORKLOADS["sweep"]["Ms"]:
+        for d in synth.WORKLOADS["sweep"]["ds"]:
+            row = {"M": M, "d": d, "bytes": BYTES_PER_ELEM * M * d}
+            inp = RotatingInputs(M, d, dev, l2)
+            row["input_sets"] = inp.nsets
+            for kind in kinds:
+                try:
+                    r = time_launches(kind, inp, args.launches, args.warmup, stream)
+                except Exception as e:  # a variant that this build does not carry
+                    row[kind] = {"error": str(e).splitlines()[0]}
+                    continue
+                gbs = BYTES_PER_ELEM * M * d / (r["mean_us"] * 1e-6) / 1e9
+                row[kind] = {"us": round(r["mean_us"], 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+            del inp
+            torch.cuda.empty_cache()
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+    if args.json_out:
+        with open(args.json_out, "w") as fh:
+            json.dump({"peak": peak, "peak_source": src, "rows": rows}, fh, indent=1)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the cpu_baseline block")
+    ap.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the reference arm")
+    ap.add_argument("--json-out", default="")
+    ap.add_argument("--mode", choices=["step", "kernel", "sweep"], default="step",
+                    help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes")
+    ap.add_argument("--kernel", default="kq", help="kernel mode: kq, sq, mx or kq_v<variant>")
+    ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
+    ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD")
+    ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")
+    ap.add_argument("--no-graph", action="store_true", help="kernel mode: eager launches")
+    ap.add_argument("--launches", type=int, default=100, help="kernel / sweep mode: timed launches")
+    args = ap.parse_args()
+    if args.mode == "kernel":
+        return kernel_mode(args)
+    if args.mode == "sweep":
+        return sweep_mode(args)
+    if args.steps < 1 or args.warmup < 3:
+        raise SystemExit("need --steps >= 1 and --warmup >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        out = reference_arm(args, rank, world)
+        if out is not None:
+            line = json.dumps(out)
+            print(line, flush=True)
+            if args.json_out:
+                with open(args.json_out, "w") as fh:
+                    fh.write(line + "\n")
+        return
+
+    from w4a4_mxfp4_post_b200 import build
+
+    build.build()
+    rank, local, world, pg = dist_setup(args.gpus)
+    try:
+        out = gpu_arm(args, rank, local, world, pg)
+        if rank == 0:
+            if world == 1:
+                out["cpu_baseline"] = cpu_baseline_block(workload_inputs(), args.cpu_seconds)
+            line = json.dumps(out)
+            print(line, flush=True)
+            if args.json_out:
+                with open(args.json_out, "w") as fh:
+                    fh.write(line + "\n")
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,130 @@
+/*
+ * kroquant.h -- C ABI of the KroQuant online activation quantizer for
+ * NVIDIA B200 (sm_100a), with the SmoothQuant and plain-MXFP4 baselines.
+ *
+ * What is computed ("KroQuant: Kronecker-Structured Block Transforms for
+ * Efficient Post-Training Quantization of Diffusion Transformers",
+ * arXiv 2607.21446, abstract and section 3.2, Eq. (4) as summarised by the
+ * Pith review of the paper): every token row of a bf16 activation X[M, d] is
+ * cut into d/32 blocks of 32 consecutive channels; block j of every row is
+ * multiplied by the 32x32 matrix K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5, a
+ * Kronecker product of five 2x2 factors; the result y is quantized to MXFP4:
+ *
+ *   amax  = max_i |y_i|                                  (fp32)
+ *   e     = clamp(floor(log2(amax)) - 2, -127, 127)      (amax = 0 -> -127)
+ *   scale = byte e + 127 (E8M0), one per block
+ *   code  = FP4 E2M1 of y_i * 2^-e, round-to-nearest-even, saturating at +-6,
+ *           sign bit = sign of y_i (a negative value that rounds to zero is 0x8)
+ *
+ * (the scale rule and element format are the OCP Microscaling Formats v1.0
+ * MXFP4 conversion, section 6.3).
+ *
+ * Layouts (all row-major, contiguous, no strides):
+ *   act      bf16 [M][d]              d a positive multiple of 32
+ *   factors  float32 [d/32][5][2][2]   factors[j][k] is G_(k+1) of column block
+ *                                      j, stored [row][col]; G1 acts on bit 4
+ *                                      (the MSB) of the in-block index, G5 on
+ *                                      bit 0 (the textbook Kronecker order).
+ *                                      Shared mode: one set [5][2][2] for every
+ *                                      column block.
+ *   codes    uint8 [M][d/2]           element 2i in the low nibble of byte i,
+ *                                      element 2i+1 in the high nibble.
+ *   scales   uint8 [M][d/32]          E8M0 byte of each block.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer is a DEVICE pointer owned by the caller.  The library never
+ *     allocates, frees or synchronises; work is enqueued on `stream` (NULL =
+ *     the legacy default stream) and runs asynchronously.
+ *   - The returned status covers argument checks and launch errors only;
+ *     asynchronous execution errors surface at the caller's next synchronising
+ *     CUDA call.  On any non-OK status kq_last_error() describes it.
+ *   - M == 0 (or N == 0) is a no-op that returns KQ_OK without touching the GPU.
+ *   - Argument checks run before any CUDA call, in this order: negative sizes
+ *     or d % 32 != 0 -> KQ_ERR_SHAPE; NULL pointer with nonzero size ->
+ *     KQ_ERR_NULL; misalignment -> KQ_ERR_ALIGN.
+ *   - Alignment: act, out_codes, out_y, W, W_out 16 bytes; factors and mult
+ *     16 bytes; out_scales 1 byte.
+ *   - Input with a non-finite value (inf/NaN) is outside the contract: such a
+ *     block's outputs are unspecified (but written in bounds).
+ *   - Calls on different streams that write the same output race; nothing else
+ *     is shared between calls.
+ */
+#ifndef KROQUANT_H
+#define KROQUANT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's stream handle (same definition as cuda_runtime_api.h). */
+typedef struct CUstream_st *cudaStream_t;
+
+typedef enum {
+    KQ_OK = 0,
+    KQ_ERR_NULL = -1,    /* a required pointer is NULL */
+    KQ_ERR_SHAPE = -2,   /* M < 0, N < 0, d <= 0, d % 32 != 0, or size overflow */
+    KQ_ERR_ALIGN = -3,   /* a pointer is not aligned as documented above */
+    KQ_ERR_CUDA = -4,    /* a CUDA runtime call failed (launch, attribute query) */
+    KQ_ERR_VARIANT = -5  /* kq_quantize_variant: unknown or unavailable variant */
+} kq_status;
+
+/* KroQuant quantizer, one factor set per column block ([d/32][5][2][2]).
+ * Reads act once, writes codes and scales once, in one fused kernel. */
+int kq_quantize(const void *act_bf16, const float *factors,
+                uint8_t *out_codes, uint8_t *out_scales,
+                int64_t M, int64_t d, cudaStream_t stream);
+
+/* KroQuant quantizer with one factor set ([5][2][2]) shared by every column
+ * block (the shared-parameter mode of the SANA-shaped layers). */
+int kq_quantize_shared(const void *act_bf16, const float *factors,
+                       uint8_t *out_codes, uint8_t *out_scales,
+                       int64_t M, int64_t d, cudaStream_t stream);
+
+/* SmoothQuant baseline ("KroQuant ...", abstract: per-channel scaling): y_c =
+ * fp32(x_c * mult[c]) with mult[c] = 1/s_c given (float32 [d]), then the MXFP4
+ * block quantizer above. */
+int sq_quantize(const void *act_bf16, const float *mult,
+                uint8_t *out_codes, uint8_t *out_scales,
+                int64_t M, int64_t d, cudaStream_t stream);
+
+/* Plain MXFP4 baseline: the block quantizer above applied to x itself. */
+int mx_quantize(const void *act_bf16,
+                uint8_t *out_codes, uint8_t *out_scales,
+                int64_t M, int64_t d, cudaStream_t stream);
+
+/* Offline fold of the inverse transform into weights (Pith review, "key
+ * machinery": the inverse is folded into the weights offline), used to check
+ * invertibility: W_out = W T^-1, i.e. for every row n and column block j,
+ * W_out[n, blk j] = W[n, blk j] (K^(j))^-1, so that
+ * X W^T == (X T^T)(W_out)^T.  W, W_out: float32 [N][d] (may not alias).
+ * shared != 0 selects one factor set for all blocks.  Every factor must be
+ * invertible (det != 0); a zero determinant yields inf/NaN outputs. */
+int kq_fold_weights(const float *W, const float *factors, int shared,
+                    float *W_out, int64_t N, int64_t d, cudaStream_t stream);
+
+/* Test export: the fp32 transform y = T x (float32 [M][d]) exactly as the
+ * quantizer computes it before the amax, for the transform-accuracy check. */
+int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
+                     float *out_y, int64_t M, int64_t d, cudaStream_t stream);
+
+/* Test export: the KroQuant quantizer through a chosen kernel variant.
+ * variant 0 = the register-butterfly kernel that kq_quantize uses.  Other
+ * values return KQ_ERR_VARIANT unless the library was built with them. */
+int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
+                        int shared, uint8_t *out_codes, uint8_t *out_scales,
+                        int64_t M, int64_t d, cudaStream_t stream);
+
+/* Message for the last non-OK status returned on the calling thread (a static
+ * thread-local buffer, valid until the thread's next call).  "" if none. */
+const char *kq_last_error(void);
+
+/* Library ABI version (this header: 1). */
+int kq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KROQUANT_H */

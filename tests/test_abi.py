@@ -1,0 +1,126 @@
+"""The C-ABI library loads, exports every declared entry point, and its host-side
+argument checks return the documented status before touching CUDA (no GPU).
+
+Every call below is built to FAIL validation (or to be an M == 0 no-op): none
+may pass its checks with the placeholder pointers used here, because a call
+that passes would launch a kernel on them.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w4a4_mxfp4_post_b200 import build
+
+    build.build()
+    import w4a4_mxfp4_post_b200 as kq
+
+    return kq.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(HEADER_DIR, fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M):
+            if m.group(1) not in ("if", "return", "sizeof"):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("kq_quantize", "kq_quantize_shared", "sq_quantize", "mx_quantize", "kq_fold_weights",
+                     "kq_transform_f32", "kq_quantize_variant", "kq_last_error", "kq_abi_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from w4a4_mxfp4_post_b200 import LIB_PATH
+
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert getattr(L, n) is not None
+
+
+def test_abi_version(L):
+    assert L.kq_abi_version() == 1
+
+
+def err(L):
+    return L.kq_last_error().decode()
+
+
+P = ctypes.c_void_p
+
+
+def test_shape_errors_before_cuda(L):
+    assert L.kq_quantize(P(16), P(16), P(16), P(16), 4, 33, None) == -2
+    assert "multiple of 32" in err(L)
+    assert L.kq_quantize(P(16), P(16), P(16), P(16), -1, 64, None) == -2
+    assert L.sq_quantize(P(16), P(16), P(16), P(16), 4, 0, None) == -2
+    assert L.mx_quantize(P(16), P(16), P(16), 4, -32, None) == -2
+    assert L.kq_fold_weights(P(16), P(16), 0, P(16), 4, 48, None) == -2
+    assert L.kq_transform_f32(P(16), P(16), 0, P(16), 4, 31, None) == -2
+    # overflow of M * d
+    assert L.mx_quantize(P(16), P(16), P(16), 2 ** 62, 64, None) == -2
+
+
+def test_empty_is_a_noop(L):
+    for M in (0,):
+        assert L.kq_quantize(None, None, None, None, M, 64, None) == 0
+        assert L.kq_quantize_shared(None, None, None, None, M, 64, None) == 0
+        assert L.sq_quantize(None, None, None, None, M, 64, None) == 0
+        assert L.mx_quantize(None, None, None, M, 64, None) == 0
+        assert L.kq_fold_weights(None, None, 0, None, M, 64, None) == 0
+        assert L.kq_transform_f32(None, None, 0, None, M, 64, None) == 0
+        assert err(L) == ""
+
+
+def test_null_errors(L):
+    assert L.kq_quantize(None, P(16), P(16), P(16), 4, 64, None) == -1
+    assert L.kq_quantize(P(16), None, P(16), P(16), 4, 64, None) == -1
+    assert L.kq_quantize(P(16), P(16), None, P(16), 4, 64, None) == -1
+    assert L.kq_quantize(P(16), P(16), P(16), None, 4, 64, None) == -1
+    assert L.sq_quantize(P(16), None, P(16), P(16), 4, 64, None) == -1
+    assert L.mx_quantize(P(16), P(16), None, 4, 64, None) == -1
+    assert L.kq_fold_weights(P(16), P(16), 0, None, 4, 64, None) == -1
+    assert L.kq_transform_f32(P(16), P(16), 0, None, 4, 64, None) == -1
+    assert "NULL" in err(L)
+
+
+def test_alignment_errors(L):
+    assert L.kq_quantize(P(8), P(16), P(16), P(16), 4, 64, None) == -3
+    assert L.kq_quantize(P(16), P(4), P(16), P(16), 4, 64, None) == -3
+    assert L.kq_quantize(P(16), P(16), P(24), P(16), 4, 64, None) == -3
+    assert L.sq_quantize(P(16), P(20), P(16), P(16), 4, 64, None) == -3
+    assert L.kq_fold_weights(P(16), P(16), 0, P(40), 4, 64, None) == -3
+    assert "aligned" in err(L)
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+
+    import w4a4_mxfp4_post_b200 as kq
+
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kq.mx_quantize(x)
+    with pytest.raises(TypeError):
+        kq.mx_quantize(torch.zeros(4, 64))

@@ -1,0 +1,225 @@
+"""KroQuant online activation quantizer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``include/kroquant.h`` (the shared
+library ``libkroquant.so`` built in-tree by ``w4a4_mxfp4_post_b200.build``).
+The functions below only marshal arguments: they check dtypes, devices and
+shapes of torch tensors, allocate outputs when none are given, and pass raw
+device pointers and the current CUDA stream to the library.  Every step of
+the computation runs in the library's CUDA kernels; there is no fallback, and
+every function raises if the library is missing or returns an error.
+
+    codes, scales = kq_quantize(act, factors)            # [M, d/2], [M, d/32] uint8
+    codes, scales = kq_quantize_shared(act, factors5)
+    codes, scales = sq_quantize(act, mult)
+    codes, scales = mx_quantize(act)
+    W_folded      = kq_fold_weights(W, factors, shared=False)
+    y             = kq_transform_f32(act, factors, shared=False)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "LIB_PATH", "KQ_OK", "KQ_ERR_NULL", "KQ_ERR_SHAPE", "KQ_ERR_ALIGN", "KQ_ERR_CUDA", "KQ_ERR_VARIANT",
+    "KroQuantError", "lib", "kq_quantize", "kq_quantize_shared", "kq_quantize_variant", "sq_quantize",
+    "mx_quantize", "kq_fold_weights", "kq_transform_f32", "kq_last_error", "kq_abi_version",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
+
+KQ_OK, KQ_ERR_NULL, KQ_ERR_SHAPE, KQ_ERR_ALIGN, KQ_ERR_CUDA, KQ_ERR_VARIANT = 0, -1, -2, -3, -4, -5
+
+# Entry points and their argument types (p = pointer, i = int, q = int64).
+_SIGS = {
+    "kq_quantize": "ppppqqp",
+    "kq_quantize_shared": "ppppqqp",
+    "kq_quantize_variant": "ippippqqp",
+    "sq_quantize": "ppppqqp",
+    "mx_quantize": "pppqqp",
+    "kq_fold_weights": "ppipqqp",
+    "kq_transform_f32": "ppipqqp",
+}
+
+_lib = None
+
+
+class KroQuantError(RuntimeError):
+    """A non-OK status from the library, with its status code and message."""
+
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"KroQuant CUDA library not found at {LIB_PATH}; build it with "
+                "`python -m w4a4_mxfp4_post_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        kinds = {"p": ctypes.c_void_p, "i": ctypes.c_int, "q": ctypes.c_int64}
+        for name, sig in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = [kinds[c] for c in sig]
+            fn.restype = ctypes.c_int
+        L.kq_last_error.argtypes = []
+        L.kq_last_error.restype = ctypes.c_char_p
+        L.kq_abi_version.argtypes = []
+        L.kq_abi_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def kq_last_error() -> str:
+    return lib().kq_last_error().decode()
+
+
+def kq_abi_version() -> int:
+    return lib().kq_abi_version()
+
+
+def _call(name: str, *args) -> None:
+    rc = getattr(lib(), name)(*args)
+    if rc != KQ_OK:
+        raise KroQuantError(name, rc, kq_last_error())
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() > 0 else 0)
+
+
+def _need(t, name, dtype, device=None, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _act(act):
+    torch = _torch()
+    _need(act, "act", torch.bfloat16)
+    if act.dim() != 2:
+        raise ValueError("act must be 2-D [M, d]")
+    return act.shape
+
+
+def _outs(act, out_codes, out_scales):
+    torch = _torch()
+    M, d = act.shape
+    if out_codes is None:
+        out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=act.device)
+    if out_scales is None:
+        out_scales = torch.empty((M, d // 32), dtype=torch.uint8, device=act.device)
+    _need(out_codes, "out_codes", torch.uint8, act.device, (M, d // 2))
+    _need(out_scales, "out_scales", torch.uint8, act.device, (M, d // 32))
+    return out_codes, out_scales
+
+
+def _factors(factors, d, shared, device):
+    torch = _torch()
+    _need(factors, "factors", torch.float32, device)
+    n = 1 if shared else d // 32
+    if factors.numel() != n * 20:
+        raise ValueError(f"factors must hold {n} x 5 x 2 x 2 floats, got {tuple(factors.shape)}")
+    return factors
+
+
+def kq_quantize(act, factors, out_codes=None, out_scales=None, stream=None):
+    """KroQuant quantizer with one factor set per 32-column block ([d/32, 5, 2, 2])."""
+    M, d = _act(act)
+    _factors(factors, d, False, act.device)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("kq_quantize", _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def kq_quantize_shared(act, factors, out_codes=None, out_scales=None, stream=None):
+    """KroQuant quantizer with one factor set ([5, 2, 2]) for every block."""
+    M, d = _act(act)
+    _factors(factors, d, True, act.device)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("kq_quantize_shared", _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream))
+    return out_codes, out_scales
+
+
+def kq_quantize_variant(variant, act, factors, shared=False, out_codes=None, out_scales=None, stream=None):
+    """The KroQuant quantizer through a chosen kernel variant (0 = the default)."""
+    M, d = _act(act)
+    _factors(factors, d, shared, act.device)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("kq_quantize_variant", int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes),
+          _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def sq_quantize(act, mult, out_codes=None, out_scales=None, stream=None):
+    """SmoothQuant baseline: fp32(x * mult[c]) per channel, then MXFP4."""
+    torch = _torch()
+    M, d = _act(act)
+    _need(mult, "mult", torch.float32, act.device, (d,))
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("sq_quantize", _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def mx_quantize(act, out_codes=None, out_scales=None, stream=None):
+    """Plain MXFP4 baseline (no transform)."""
+    M, d = _act(act)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("mx_quantize", _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def kq_fold_weights(W, factors, shared=False, out=None, stream=None):
+    """W T^-1 per 32-column block (fp32 [N, d])."""
+    torch = _torch()
+    _need(W, "W", torch.float32)
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [N, d]")
+    N, d = W.shape
+    _factors(factors, d, shared, W.device)
+    if out is None:
+        out = torch.empty_like(W)
+    _need(out, "out", torch.float32, W.device, (N, d))
+    _call("kq_fold_weights", _ptr(W), _ptr(factors), int(bool(shared)), _ptr(out), N, d, _stream(stream))
+    return out
+
+
+def kq_transform_f32(act, factors, shared=False, out=None, stream=None):
+    """The fp32 transform y = T x that the quantizer computes (test export)."""
+    torch = _torch()
+    M, d = _act(act)
+    _factors(factors, d, shared, act.device)
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.float32, device=act.device)
+    _need(out, "out", torch.float32, act.device, (M, d))
+    _call("kq_transform_f32", _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d, _stream(stream))
+    return out

@@ -1,0 +1,489 @@
+// kroquant.cu -- sm_100a kernels and the C ABI (include/kroquant.h) of the
+// KroQuant online activation quantizer and its two baselines.
+//
+// Operation ("KroQuant: Kronecker-Structured Block Transforms for Efficient
+// Post-Training Quantization of Diffusion Transformers", arXiv 2607.21446,
+// abstract; section 3.2, Eq. (4) as summarised by the Pith review): for every
+// 32-channel block of every bf16 token row, y = (G1 (x) ... (x) G5) x, then
+// MXFP4 (OCP MX v1.0, section 6.3): E8M0 scale 2^(floor(log2 amax) - 2),
+// E2M1 codes by round-to-nearest-even with saturation.
+//
+// Design: the path is a pure stream (2 B read, 0.53 B written per element) so
+// every kernel reads each activation byte once with 16-byte loads and writes
+// codes and scales once; the Kronecker product is never materialised -- its
+// five 2x2 factors are applied as radix-2 butterflies on values held in
+// registers.  One thread owns one 32-element block, so no shuffles are needed;
+// consecutive threads own consecutive blocks of the flattened [M*d/32] block
+// array, so a warp reads 2 KB contiguous and writes 512 B of codes and 32 B of
+// scales contiguous.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "kroquant.h"
+
+namespace {
+
+constexpr int kBlk = 32;           // MX block size == Kronecker block size
+constexpr int kThreads = 256;      // threads per CTA for the streaming kernels
+
+// ---------------------------------------------------------------------------
+// error reporting
+// ---------------------------------------------------------------------------
+thread_local char tl_err[512] = "";
+
+int fail(int status, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(tl_err, sizeof tl_err, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int ok()
+{
+    tl_err[0] = '\0';
+    return KQ_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+
+// bf16 -> fp32 is exact: a bf16 is the upper half of a binary32.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack32(const uint4 (&raw)[4], float (&v)[32])
+{
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            v[8 * q + 2 * h] = bf16_lo(w[h]);
+            v[8 * q + 2 * h + 1] = bf16_hi(w[h]);
+        }
+    }
+}
+
+// One radix-2 Kronecker stage: the 2x2 factor F acts on in-block index bit
+// BIT, i.e. on every pair (i, i | 1<<BIT) with bit BIT of i clear.
+template <int BIT>
+__device__ __forceinline__ void kron_stage(float (&v)[32], float f00, float f01, float f10, float f11)
+{
+#pragma unroll
+    for (int i = 0; i < kBlk; ++i) {
+        if (i & (1 << BIT)) continue;
+        const float lo = v[i];
+        const float hi = v[i | (1 << BIT)];
+        v[i] = fmaf(f01, hi, f00 * lo);
+        v[i | (1 << BIT)] = fmaf(f11, hi, f10 * lo);
+    }
+}
+
+// y = (G1 (x) G2 (x) G3 (x) G4 (x) G5) v.  G1 (f[0..3]) acts on bit 4, G5
+// (f[16..19]) on bit 0.  The five stages act on different index bits and
+// therefore commute; they run from bit 0 up.
+__device__ __forceinline__ void kron_apply(float (&v)[32], const float (&f)[20])
+{
+    kron_stage<0>(v, f[16], f[17], f[18], f[19]);
+    kron_stage<1>(v, f[12], f[13], f[14], f[15]);
+    kron_stage<2>(v, f[8], f[9], f[10], f[11]);
+    kron_stage<3>(v, f[4], f[5], f[6], f[7]);
+    kron_stage<4>(v, f[0], f[1], f[2], f[3]);
+}
+
+// E8M0 byte of a block from amax >= 0: e = floor(log2 amax) - 2 clamped to
+// [-127, 127] is, for a normal amax, (exponent field - 127) - 2, so the byte
+// e + 127 is (exponent field - 2); subnormal amax and 0 clamp to byte 0, the
+// largest finite amax gives 252.
+__device__ __forceinline__ uint32_t e8m0_byte(float amax)
+{
+    const uint32_t ef = __float_as_uint(amax) >> 23;
+    return ef > 2u ? ef - 2u : 0u;
+}
+
+// 2^-e for the byte above: exponent field 127 - e = 254 - byte, always normal.
+__device__ __forceinline__ float inv_scale(uint32_t sb) { return __uint_as_float((254u - sb) << 23); }
+
+// Eight fp32 values -> eight E2M1 codes in one word, element 0 in the lowest
+// nibble.  cvt...e2m1x2 puts its first source in the high nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3, float a4, float a5,
+                                               float a6, float a7)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(r)
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+    return r;
+}
+
+// The MXFP4 block quantizer on 32 fp32 values: amax, E8M0 byte, scaling by
+// the exact power of two 2^-e, E2M1 rounding, packing.
+__device__ __forceinline__ void mx_quantize_block(const float (&v)[32], uint4 &codes, uint32_t &sbyte)
+{
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kBlk; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const uint32_t sb = e8m0_byte(amax);
+    const float s = inv_scale(sb);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        w[q] = cvt_e2m1x8(v[8 * q] * s, v[8 * q + 1] * s, v[8 * q + 2] * s, v[8 * q + 3] * s,
+                          v[8 * q + 4] * s, v[8 * q + 5] * s, v[8 * q + 6] * s, v[8 * q + 7] * s);
+    codes = make_uint4(w[0], w[1], w[2], w[3]);
+    sbyte = sb;
+}
+
+__device__ __forceinline__ void load_block(const uint4 *__restrict__ act, int64_t g, uint4 (&raw)[4])
+{
+    const uint4 *p = act + g * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) raw[q] = __ldg(p + q);
+}
+
+// ---------------------------------------------------------------------------
+// kernels.  Grid: T threads (T = nb * R for the column-pinned kernels), each
+// thread walks the flattened block index g = t, t + T, t + 2T, ... < nblocks.
+// With T a multiple of nb the column j = g % nb is the same on every step, so
+// a thread loads its column's factors (or multipliers) once.
+// ---------------------------------------------------------------------------
+enum class KqOut { kCodes, kF32 };
+
+template <KqOut OUT>
+__global__ void __launch_bounds__(kThreads)
+kq_butterfly_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+                    uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
+                    int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    float f[20];
+    const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const float4 q = __ldg(fp + k);
+        f[4 * k] = q.x;
+        f[4 * k + 1] = q.y;
+        f[4 * k + 2] = q.z;
+        f[4 * k + 3] = q.w;
+    }
+    for (int64_t g = t; g < nblocks; g += T) {
+        uint4 raw[4];
+        load_block(act, g, raw);
+        float v[32];
+        unpack32(raw, v);
+        kron_apply(v, f);
+        if constexpr (OUT == KqOut::kCodes) {
+            uint4 c;
+            uint32_t sb;
+            mx_quantize_block(v, c, sb);
+            codes[g] = c;
+            scales[g] = uint8_t(sb);
+        } else {
+            float4 *yo = y_out + g * 8;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) yo[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+sq_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ mult, uint4 *__restrict__ codes,
+          uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    float m[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 a = __ldg(mult + int64_t(j) * 8 + q);
+        m[4 * q] = a.x;
+        m[4 * q + 1] = a.y;
+        m[4 * q + 2] = a.z;
+        m[4 * q + 3] = a.w;
+    }
+    for (int64_t g = t; g < nblocks; g += T) {
+        uint4 raw[4];
+        load_block(act, g, raw);
+        float v[32];
+        unpack32(raw, v);
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) v[i] *= m[i];
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_block(v, c, sb);
+        codes[g] = c;
+        scales[g] = uint8_t(sb);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+mx_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
+          int64_t nblocks, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    for (int64_t g = t; g < nblocks; g += T) {
+        uint4 raw[4];
+        load_block(act, g, raw);
+        float v[32];
+        unpack32(raw, v);
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_block(v, c, sb);
+        codes[g] = c;
+        scales[g] = uint8_t(sb);
+    }
+}
+
+// Fold: w' = w K^-1 for a row vector w, i.e. w'^T = (K^-1)^T w^T, which is
+// the Kronecker product of the 2x2 matrices (G_k^-1)^T = [[g11, -g10],
+// [-g01, g00]] / det(G_k) applied as butterflies.  fp32 in, fp32 out.
+__global__ void __launch_bounds__(kThreads)
+fold_kernel(const float4 *__restrict__ W, const float4 *__restrict__ factors, int shared,
+            float4 *__restrict__ W_out, int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    float f[20];
+    const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const float4 q = __ldg(fp + k);
+        const float det = fmaf(q.x, q.w, -q.y * q.z);
+        const float r = 1.0f / det;
+        f[4 * k] = q.w * r;
+        f[4 * k + 1] = -q.z * r;
+        f[4 * k + 2] = -q.y * r;
+        f[4 * k + 3] = q.x * r;
+    }
+    for (int64_t g = t; g < nblocks; g += T) {
+        float v[32];
+        const float4 *wp = W + g * 8;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 a = __ldg(wp + q);
+            v[4 * q] = a.x;
+            v[4 * q + 1] = a.y;
+            v[4 * q + 2] = a.z;
+            v[4 * q + 3] = a.w;
+        }
+        kron_apply(v, f);
+        float4 *wo = W_out + g * 8;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) wo[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launch geometry
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+
+int sm_count(int *out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev >= 0 && dev < kMaxDevices) {
+        int c = g_sm_count[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *out = c;
+            return KQ_OK;
+        }
+    }
+    int c = 0;
+    e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(c, std::memory_order_relaxed);
+    *out = c;
+    return KQ_OK;
+}
+
+// Threads T = nb * R with R rows per sweep chosen so that every thread runs
+// the same number of steps, ceil(M / R), and T stays near the resident-thread
+// target of the device.
+struct Geometry {
+    int64_t T;
+    unsigned grid;
+};
+
+Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
+{
+    int64_t R = target_threads / nb;
+    if (R < 1) R = 1;
+    if (R > M) R = M;
+    const int64_t steps = (M + R - 1) / R;
+    R = (M + steps - 1) / steps;
+    Geometry g;
+    g.T = nb * R;
+    g.grid = unsigned((g.T + kThreads - 1) / kThreads);
+    return g;
+}
+
+// Resident threads per SM assumed for the sizing above (register-limited
+// kernels of this file reach 4-8 CTAs of 256 threads).
+constexpr int64_t kTargetThreadsPerSm = 1024;
+
+int launch_check(const char *what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+// Common argument checks; returns KQ_OK, an error status, or 1 for "no work".
+int check_quant_args(const char *fn, const void *act, const void *params, bool need_params, const void *codes,
+                     const void *scales, int64_t M, int64_t d)
+{
+    if (M < 0 || d <= 0 || d % kBlk != 0)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32 (M=%lld, d=%lld)", fn,
+                    (long long)M, (long long)d);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d))
+        return fail(KQ_ERR_SHAPE, "%s: size too large (M=%lld, d=%lld)", fn, (long long)M, (long long)d);
+    if (M == 0) return 1;
+    if (!act || !codes || !scales || (need_params && !params))
+        return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(act, 16) || !aligned(codes, 16) || (need_params && !aligned(params, 16)))
+        return fail(KQ_ERR_ALIGN, "%s: act, out_codes and factors/mult must be 16-byte aligned", fn);
+    return KQ_OK;
+}
+
+int kq_launch(const char *fn, int variant, const void *act, const float *factors, int shared,
+              uint8_t *codes, uint8_t *scales, float *y, bool f32, int64_t M, int64_t d, cudaStream_t stream)
+{
+    int rc = f32 ? check_quant_args(fn, act, factors, true, y, y, M, d)
+                 : check_quant_args(fn, act, factors, true, codes, scales, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    if (variant != 0 && variant != 1)
+        return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    int sms = 0;
+    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
+    const int64_t nblocks = M * nb;
+    if (f32) {
+        kq_butterfly_kernel<KqOut::kF32><<<geo.grid, kThreads, 0, stream>>>(
+            static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors), shared, nullptr, nullptr,
+            reinterpret_cast<float4 *>(y), nblocks, int(nb), geo.T);
+    } else {
+        kq_butterfly_kernel<KqOut::kCodes><<<geo.grid, kThreads, 0, stream>>>(
+            static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors), shared,
+            reinterpret_cast<uint4 *>(codes), scales, nullptr, nblocks, int(nb), geo.T);
+    }
+    return launch_check(fn);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+int kq_abi_version(void) { return 1; }
+
+const char *kq_last_error(void) { return tl_err; }
+
+int kq_quantize(const void *act_bf16, const float *factors, uint8_t *out_codes, uint8_t *out_scales, int64_t M,
+                int64_t d, cudaStream_t stream)
+{
+    return kq_launch("kq_quantize", 0, act_bf16, factors, 0, out_codes, out_scales, nullptr, false, M, d, stream);
+}
+
+int kq_quantize_shared(const void *act_bf16, const float *factors, uint8_t *out_codes, uint8_t *out_scales,
+                       int64_t M, int64_t d, cudaStream_t stream)
+{
+    return kq_launch("kq_quantize_shared", 0, act_bf16, factors, 1, out_codes, out_scales, nullptr, false, M, d,
+                     stream);
+}
+
+int kq_quantize_variant(int variant, const void *act_bf16, const float *factors, int shared, uint8_t *out_codes,
+                        uint8_t *out_scales, int64_t M, int64_t d, cudaStream_t stream)
+{
+    return kq_launch("kq_quantize_variant", variant, act_bf16, factors, shared ? 1 : 0, out_codes, out_scales,
+                     nullptr, false, M, d, stream);
+}
+
+int kq_transform_f32(const void *act_bf16, const float *factors, int shared, float *out_y, int64_t M, int64_t d,
+                     cudaStream_t stream)
+{
+    return kq_launch("kq_transform_f32", 0, act_bf16, factors, shared ? 1 : 0, nullptr, nullptr, out_y, true, M, d,
+                     stream);
+}
+
+int sq_quantize(const void *act_bf16, const float *mult, uint8_t *out_codes, uint8_t *out_scales, int64_t M,
+                int64_t d, cudaStream_t stream)
+{
+    int rc = check_quant_args("sq_quantize", act_bf16, mult, true, out_codes, out_scales, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    int sms = 0;
+    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
+    sq_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                                 reinterpret_cast<const float4 *>(mult),
+                                                 reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb, int(nb),
+                                                 geo.T);
+    return launch_check("sq_quantize");
+}
+
+int mx_quantize(const void *act_bf16, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
+                cudaStream_t stream)
+{
+    int rc = check_quant_args("mx_quantize", act_bf16, nullptr, false, out_codes, out_scales, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    int sms = 0;
+    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
+    mx_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                                 reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb, geo.T);
+    return launch_check("mx_quantize");
+}
+
+int kq_fold_weights(const float *W, const float *factors, int shared, float *W_out, int64_t N, int64_t d,
+                    cudaStream_t stream)
+{
+    if (N < 0 || d <= 0 || d % kBlk != 0)
+        return fail(KQ_ERR_SHAPE, "kq_fold_weights: need N >= 0 and d a positive multiple of 32");
+    if (d / kBlk > INT32_MAX || (N > 0 && N > INT64_MAX / d))
+        return fail(KQ_ERR_SHAPE, "kq_fold_weights: size too large");
+    if (N == 0) return ok();
+    if (!W || !factors || !W_out) return fail(KQ_ERR_NULL, "kq_fold_weights: NULL pointer argument");
+    if (!aligned(W, 16) || !aligned(W_out, 16) || !aligned(factors, 16))
+        return fail(KQ_ERR_ALIGN, "kq_fold_weights: W, W_out and factors must be 16-byte aligned");
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    const Geometry geo = pinned_geometry(N, nb, int64_t(sms) * kTargetThreadsPerSm);
+    fold_kernel<<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(W),
+                                                   reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
+                                                   reinterpret_cast<float4 *>(W_out), N * nb, int(nb), geo.T);
+    return launch_check("kq_fold_weights");
+}
+
+}  // extern "C"
