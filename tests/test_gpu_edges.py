@@ -225,5 +225,10 @@ def test_extreme_magnitudes(cuda_device):
     cr, sr = oracle.kq_quantize(x, I)
     np.testing.assert_array_equal(s.cpu().numpy(), sr)
     np.testing.assert_array_equal(c.cpu().numpy(), cr)
+    # The plain MX path keeps the sign of a -0 input (bf16 underflow of tiny
+    # negatives gives -0); the transform's sum turns it into +0, so MX is
+    # compared with the oracle's MX, not with the identity-factor KQ result.
     c, s = kq.mx_quantize(dev_bf16(x, cuda_device))
-    np.testing.assert_array_equal(c.cpu().numpy(), cr)
+    cm, sm = oracle.mx_quantize(x)
+    np.testing.assert_array_equal(s.cpu().numpy(), sm)
+    np.testing.assert_array_equal(c.cpu().numpy(), cm)

@@ -204,55 +204,6 @@ kq_butterfly_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ fa
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
-sq_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ mult, uint4 *__restrict__ codes,
-          uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
-{
-    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    if (t >= T || t >= nblocks) return;
-    const int j = int(t % nb);
-    float m[32];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const float4 a = __ldg(mult + int64_t(j) * 8 + q);
-        m[4 * q] = a.x;
-        m[4 * q + 1] = a.y;
-        m[4 * q + 2] = a.z;
-        m[4 * q + 3] = a.w;
-    }
-    for (int64_t g = t; g < nblocks; g += T) {
-        uint4 raw[4];
-        load_block(act, g, raw);
-        float v[32];
-        unpack32(raw, v);
-#pragma unroll
-        for (int i = 0; i < kBlk; ++i) v[i] *= m[i];
-        uint4 c;
-        uint32_t sb;
-        mx_quantize_block(v, c, sb);
-        codes[g] = c;
-        scales[g] = uint8_t(sb);
-    }
-}
-
-__global__ void __launch_bounds__(kThreads)
-mx_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
-          int64_t nblocks, int64_t T)
-{
-    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    for (int64_t g = t; g < nblocks; g += T) {
-        uint4 raw[4];
-        load_block(act, g, raw);
-        float v[32];
-        unpack32(raw, v);
-        uint4 c;
-        uint32_t sb;
-        mx_quantize_block(v, c, sb);
-        codes[g] = c;
-        scales[g] = uint8_t(sb);
-    }
-}
-
 // Fold: w' = w K^-1 for a row vector w, i.e. w'^T = (K^-1)^T w^T, which is
 // the Kronecker product of the 2x2 matrices (G_k^-1)^T = [[g11, -g10],
 // [-g01, g00]] / det(G_k) applied as butterflies.  fp32 in, fp32 out.
@@ -290,6 +241,314 @@ fold_kernel(const float4 *__restrict__ W, const float4 *__restrict__ factors, in
         float4 *wo = W_out + g * 8;
 #pragma unroll
         for (int q = 0; q < 8; ++q) wo[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Packed-pair kernels.  A block's 32 values sit in 16 register pairs
+// p[i] = (x_i, x_{i+16}), so that every operation that treats the 32 values
+// alike, or pairs index i with i ^ 2^b for b < 4, runs as one packed f32x2
+// instruction on two values (__fmul2_rn / __ffma2_rn, sm_100).  Each thread
+// prefetches the next block of its grid-stride walk before working on the
+// current one, so two 64-byte loads per thread are in flight.
+// ---------------------------------------------------------------------------
+
+// p[i] = (x_i, x_{i+16}) from the 64 bytes of a block (raw[0..1] hold
+// elements 0..15, raw[2..3] elements 16..31).
+__device__ __forceinline__ void unpack_pairs(const uint4 (&raw)[4], float2 (&p)[16])
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t lo[4] = {raw[h].x, raw[h].y, raw[h].z, raw[h].w};
+        const uint32_t hi[4] = {raw[h + 2].x, raw[h + 2].y, raw[h + 2].z, raw[h + 2].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            p[8 * h + 2 * w] = make_float2(bf16_lo(lo[w]), bf16_lo(hi[w]));
+            p[8 * h + 2 * w + 1] = make_float2(bf16_hi(lo[w]), bf16_hi(hi[w]));
+        }
+    }
+}
+
+// max(|a|, |b|, |c|) in one instruction (three-input max, sm_100).
+__device__ __forceinline__ float max3_abs(float a, float b, float c)
+{
+    float r;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// MXFP4 block quantizer on the pair layout (same arithmetic as
+// mx_quantize_block: amax, E8M0 byte from its exponent field, exact scaling
+// by 2^-e, E2M1 round-to-nearest-even with saturation, packing).
+__device__ __forceinline__ void mx_quantize_pairs(float2 (&p)[16], uint4 &codes, uint32_t &sbyte)
+{
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = max3_abs(amax, p[i].x, p[i].y);
+    const uint32_t sb = e8m0_byte(amax);
+    const float s = inv_scale(sb);
+    const float2 ss = make_float2(s, s);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p[i] = __fmul2_rn(p[i], ss);
+    codes.x = cvt_e2m1x8(p[0].x, p[1].x, p[2].x, p[3].x, p[4].x, p[5].x, p[6].x, p[7].x);
+    codes.y = cvt_e2m1x8(p[8].x, p[9].x, p[10].x, p[11].x, p[12].x, p[13].x, p[14].x, p[15].x);
+    codes.z = cvt_e2m1x8(p[0].y, p[1].y, p[2].y, p[3].y, p[4].y, p[5].y, p[6].y, p[7].y);
+    codes.w = cvt_e2m1x8(p[8].y, p[9].y, p[10].y, p[11].y, p[12].y, p[13].y, p[14].y, p[15].y);
+    sbyte = sb;
+}
+
+// Stage on in-block index bit b < 4 (pair-index distance S = 2^b) in unit-
+// diagonal form: lo' = lo + b*hi, hi' = c*lo + hi (packed, both halves).
+template <int S>
+__device__ __forceinline__ void unit_stage2(float2 (&p)[16], float2 B, float2 C)
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        if (i & S) continue;
+        const float2 lo = p[i], hi = p[i + S];
+        p[i] = __ffma2_rn(B, hi, lo);
+        p[i + S] = __ffma2_rn(C, lo, hi);
+    }
+}
+
+// Stage on bit b < 4 in the direct form lo' = f00 lo + f01 hi, hi' = f10 lo + f11 hi.
+template <int S>
+__device__ __forceinline__ void direct_stage2(float2 (&p)[16], float2 F00, float2 F01, float2 F10, float2 F11)
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        if (i & S) continue;
+        const float2 lo = p[i], hi = p[i + S];
+        p[i] = __ffma2_rn(F01, hi, __fmul2_rn(F00, lo));
+        p[i + S] = __ffma2_rn(F11, hi, __fmul2_rn(F10, lo));
+    }
+}
+
+__device__ __forceinline__ float2 bcast(float v) { return make_float2(v, v); }
+
+// Unit-diagonal split of one factor; false if the factor is outside the range
+// where the split is used (see the kernel comment).
+__device__ __forceinline__ bool unit_split(const float4 g, float &d0, float &d1, float &b, float &c)
+{
+    d0 = g.x;
+    d1 = g.w;
+    b = __fdividef(g.y, g.x);
+    c = __fdividef(g.z, g.w);
+    const float a0 = fabsf(d0), a1 = fabsf(d1);
+    return a0 >= 0x1p-16f && a0 <= 0x1p16f && a1 >= 0x1p-16f && a1 <= 0x1p16f && fabsf(b) <= 16.0f &&
+           fabsf(c) <= 16.0f;
+}
+
+__device__ __forceinline__ void load_block_nc(const uint4 *__restrict__ act, int64_t g, uint4 (&raw)[4])
+{
+    const uint4 *p = act + g * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) raw[q] = __ldg(p + q);
+}
+
+// KroQuant quantizer, packed butterfly (variant 2).
+//
+// Each 2x2 factor is split as G = [[g00, g01], [g10, g11]]
+// = diag(g00, g11) [[1, b], [c, 1]] with b = g01/g00, c = g10/g11; by the
+// mixed-product property K = G1 (x) ... (x) G5 = D U, with D the diagonal
+// (x)_k diag(g00_k, g11_k) and U = (x)_k [[1, b_k], [c_k, 1]].  A unit-diagonal
+// stage costs one FFMA per element and D one multiply, so the transform and
+// scaling take 7 FP32 lane operations per element against 11 for the direct
+// form.  The rounding differs from the direct form by a few fp32 ulps of
+// (|K||x|)_i, the same order as the direct form's own rounding.
+// A thread whose column has a factor with |g00| or |g11| outside
+// [2^-16, 2^16] or |b| or |c| above 16 (where U's intermediate values could
+// grow by more than 17^5) runs the direct form instead.
+template <KqOut OUT>
+__global__ void __launch_bounds__(kThreads, 2)
+kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+                 uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
+                 int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+    float4 g[5];
+#pragma unroll
+    for (int k = 0; k < 5; ++k) g[k] = __ldg(fp + k);
+
+    float d0[5], d1[5], bb[5], cc[5];
+    bool fast = true;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) fast &= unit_split(g[k], d0[k], d1[k], bb[k], cc[k]);
+
+    int64_t gi = t;
+    uint4 raw[4];
+    load_block_nc(act, gi, raw);
+
+    if (fast) {
+        // D_i = prod_k (bit (4-k) of i ? g11_k : g00_k); factor k = 0 (G1) acts on bit 4.
+        float dd[32];
+        dd[0] = 1.0f;
+#pragma unroll
+        for (int bit = 0; bit < 5; ++bit) {
+            const int k = 4 - bit;
+#pragma unroll
+            for (int i = 0; i < (1 << bit); ++i) {
+                dd[i + (1 << bit)] = dd[i] * d1[k];
+                dd[i] = dd[i] * d0[k];
+            }
+        }
+        float2 DP[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) DP[i] = make_float2(dd[i], dd[i + 16]);
+        const float2 B0 = bcast(bb[4]), C0 = bcast(cc[4]);   // G5, bit 0
+        const float2 B1 = bcast(bb[3]), C1 = bcast(cc[3]);   // G4, bit 1
+        const float2 B2 = bcast(bb[2]), C2 = bcast(cc[2]);   // G3, bit 2
+        const float2 B3 = bcast(bb[1]), C3 = bcast(cc[1]);   // G2, bit 3
+        const float b4 = bb[0], c4 = cc[0];                  // G1, bit 4
+        for (;;) {
+            const int64_t gn = gi + T;
+            uint4 nxt[4];
+            if (gn < nblocks) load_block_nc(act, gn, nxt);
+            float2 p[16];
+            unpack_pairs(raw, p);
+            unit_stage2<1>(p, B0, C0);
+            unit_stage2<2>(p, B1, C1);
+            unit_stage2<4>(p, B2, C2);
+            unit_stage2<8>(p, B3, C3);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float lo = p[i].x, hi = p[i].y;
+                p[i] = __fmul2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), DP[i]);
+            }
+            if constexpr (OUT == KqOut::kCodes) {
+                uint4 c;
+                uint32_t sb;
+                mx_quantize_pairs(p, c, sb);
+                codes[gi] = c;
+                scales[gi] = uint8_t(sb);
+            } else {
+                float4 *yo = y_out + gi * 8;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    yo[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
+                    yo[q + 4] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
+                }
+            }
+            if (gn >= nblocks) break;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
+            gi = gn;
+        }
+    } else {
+        const float2 A00 = bcast(g[4].x), A01 = bcast(g[4].y), A10 = bcast(g[4].z), A11 = bcast(g[4].w);
+        const float2 E00 = bcast(g[3].x), E01 = bcast(g[3].y), E10 = bcast(g[3].z), E11 = bcast(g[3].w);
+        const float2 H00 = bcast(g[2].x), H01 = bcast(g[2].y), H10 = bcast(g[2].z), H11 = bcast(g[2].w);
+        const float2 J00 = bcast(g[1].x), J01 = bcast(g[1].y), J10 = bcast(g[1].z), J11 = bcast(g[1].w);
+        const float4 G1 = g[0];
+        for (;;) {
+            const int64_t gn = gi + T;
+            uint4 nxt[4];
+            if (gn < nblocks) load_block_nc(act, gn, nxt);
+            float2 p[16];
+            unpack_pairs(raw, p);
+            direct_stage2<1>(p, A00, A01, A10, A11);
+            direct_stage2<2>(p, E00, E01, E10, E11);
+            direct_stage2<4>(p, H00, H01, H10, H11);
+            direct_stage2<8>(p, J00, J01, J10, J11);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float lo = p[i].x, hi = p[i].y;
+                p[i] = make_float2(fmaf(G1.y, hi, G1.x * lo), fmaf(G1.w, hi, G1.z * lo));
+            }
+            if constexpr (OUT == KqOut::kCodes) {
+                uint4 c;
+                uint32_t sb;
+                mx_quantize_pairs(p, c, sb);
+                codes[gi] = c;
+                scales[gi] = uint8_t(sb);
+            } else {
+                float4 *yo = y_out + gi * 8;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    yo[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
+                    yo[q + 4] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
+                }
+            }
+            if (gn >= nblocks) break;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
+            gi = gn;
+        }
+    }
+}
+
+// SmoothQuant quantizer on the pair layout: y = fp32(x * m) per channel (one
+// correctly rounded packed multiply), then the MXFP4 block quantizer.
+__global__ void __launch_bounds__(kThreads)
+sq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ mult, uint4 *__restrict__ codes,
+                 uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    float m[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 a = __ldg(mult + int64_t(j) * 8 + q);
+        m[4 * q] = a.x;
+        m[4 * q + 1] = a.y;
+        m[4 * q + 2] = a.z;
+        m[4 * q + 3] = a.w;
+    }
+    float2 MP[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) MP[i] = make_float2(m[i], m[i + 16]);
+    int64_t gi = t;
+    uint4 raw[4];
+    load_block_nc(act, gi, raw);
+    for (;;) {
+        const int64_t gn = gi + T;
+        uint4 nxt[4];
+        if (gn < nblocks) load_block_nc(act, gn, nxt);
+        float2 p[16];
+        unpack_pairs(raw, p);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = __fmul2_rn(p[i], MP[i]);
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[gi] = c;
+        scales[gi] = uint8_t(sb);
+        if (gn >= nblocks) break;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
+        gi = gn;
+    }
+}
+
+// Plain MXFP4 quantizer on the pair layout.
+__global__ void __launch_bounds__(kThreads)
+mx_packed_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
+                 int64_t nblocks, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= nblocks) return;
+    int64_t gi = t;
+    uint4 raw[4];
+    load_block_nc(act, gi, raw);
+    for (;;) {
+        const int64_t gn = gi + T;
+        uint4 nxt[4];
+        if (gn < nblocks) load_block_nc(act, gn, nxt);
+        float2 p[16];
+        unpack_pairs(raw, p);
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[gi] = c;
+        scales[gi] = uint8_t(sb);
+        if (gn >= nblocks) break;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
+        gi = gn;
     }
 }
 
@@ -340,9 +599,29 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
     return g;
 }
 
-// Resident threads per SM assumed for the sizing above (register-limited
-// kernels of this file reach 4-8 CTAs of 256 threads).
-constexpr int64_t kTargetThreadsPerSm = 1024;
+// Resident threads of a kernel on the current device: SMs x resident CTAs
+// per SM (occupancy query, cached per device and kernel).
+enum KernelId { kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold, kNumKernels };
+std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
+
+int resident_threads(KernelId id, const void *fn, int64_t *out)
+{
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    int c = (dev >= 0 && dev < kMaxDevices) ? g_ctas_per_sm[id][dev].load(std::memory_order_relaxed) : 0;
+    if (c <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, fn, kThreads, 0);
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+        if (c < 1) c = 1;
+        if (dev >= 0 && dev < kMaxDevices) g_ctas_per_sm[id][dev].store(c, std::memory_order_relaxed);
+    }
+    *out = int64_t(sms) * c * kThreads;
+    return KQ_OK;
+}
 
 int launch_check(const char *what)
 {
@@ -368,6 +647,21 @@ int check_quant_args(const char *fn, const void *act, const void *params, bool n
     return KQ_OK;
 }
 
+template <typename Kernel>
+int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t nb, Geometry *geo)
+{
+    int64_t target = 0;
+    int rc = resident_threads(id, reinterpret_cast<const void *>(kernel), &target);
+    if (rc != KQ_OK) return rc;
+    *geo = pinned_geometry(M, nb, target);
+    (void)fn;
+    return KQ_OK;
+}
+
+// Kernel variants of the KroQuant quantizer: 1 = one block per thread, direct
+// 2x2 stages; 2 = packed pairs with the unit-diagonal split.  0 = the default.
+constexpr int kDefaultVariant = 2;
+
 int kq_launch(const char *fn, int variant, const void *act, const float *factors, int shared,
               uint8_t *codes, uint8_t *scales, float *y, bool f32, int64_t M, int64_t d, cudaStream_t stream)
 {
@@ -375,21 +669,38 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
                  : check_quant_args(fn, act, factors, true, codes, scales, M, d);
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
-    if (variant != 0 && variant != 1)
+    if (variant == 0) variant = kDefaultVariant;
+    if (variant != 1 && variant != 2)
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
-    int sms = 0;
-    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
     const int64_t nb = d / kBlk;
-    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
     const int64_t nblocks = M * nb;
-    if (f32) {
-        kq_butterfly_kernel<KqOut::kF32><<<geo.grid, kThreads, 0, stream>>>(
-            static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors), shared, nullptr, nullptr,
-            reinterpret_cast<float4 *>(y), nblocks, int(nb), geo.T);
+    const uint4 *a = static_cast<const uint4 *>(act);
+    const float4 *f = reinterpret_cast<const float4 *>(factors);
+    Geometry geo;
+    if (variant == 1) {
+        if (f32) {
+            auto k = kq_butterfly_kernel<KqOut::kF32>;
+            if ((rc = launch_pinned(fn, kKqDirectF32, k, M, nb, &geo)) != KQ_OK) return rc;
+            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
+                                                 nblocks, int(nb), geo.T);
+        } else {
+            auto k = kq_butterfly_kernel<KqOut::kCodes>;
+            if ((rc = launch_pinned(fn, kKqDirect, k, M, nb, &geo)) != KQ_OK) return rc;
+            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
+                                                 nblocks, int(nb), geo.T);
+        }
     } else {
-        kq_butterfly_kernel<KqOut::kCodes><<<geo.grid, kThreads, 0, stream>>>(
-            static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors), shared,
-            reinterpret_cast<uint4 *>(codes), scales, nullptr, nblocks, int(nb), geo.T);
+        if (f32) {
+            auto k = kq_packed_kernel<KqOut::kF32>;
+            if ((rc = launch_pinned(fn, kKqPackedF32, k, M, nb, &geo)) != KQ_OK) return rc;
+            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
+                                                 nblocks, int(nb), geo.T);
+        } else {
+            auto k = kq_packed_kernel<KqOut::kCodes>;
+            if ((rc = launch_pinned(fn, kKqPacked, k, M, nb, &geo)) != KQ_OK) return rc;
+            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
+                                                 nblocks, int(nb), geo.T);
+        }
     }
     return launch_check(fn);
 }
@@ -438,14 +749,13 @@ int sq_quantize(const void *act_bf16, const float *mult, uint8_t *out_codes, uin
     int rc = check_quant_args("sq_quantize", act_bf16, mult, true, out_codes, out_scales, M, d);
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
-    int sms = 0;
-    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
     const int64_t nb = d / kBlk;
-    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
-    sq_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
-                                                 reinterpret_cast<const float4 *>(mult),
-                                                 reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb, int(nb),
-                                                 geo.T);
+    Geometry geo;
+    if ((rc = launch_pinned("sq_quantize", kSqPacked, sq_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
+    sq_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                                        reinterpret_cast<const float4 *>(mult),
+                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb,
+                                                        int(nb), geo.T);
     return launch_check("sq_quantize");
 }
 
@@ -455,12 +765,12 @@ int mx_quantize(const void *act_bf16, uint8_t *out_codes, uint8_t *out_scales, i
     int rc = check_quant_args("mx_quantize", act_bf16, nullptr, false, out_codes, out_scales, M, d);
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
-    int sms = 0;
-    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
     const int64_t nb = d / kBlk;
-    const Geometry geo = pinned_geometry(M, nb, int64_t(sms) * kTargetThreadsPerSm);
-    mx_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
-                                                 reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb, geo.T);
+    Geometry geo;
+    if ((rc = launch_pinned("mx_quantize", kMxPacked, mx_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
+    mx_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb,
+                                                        geo.T);
     return launch_check("mx_quantize");
 }
 
@@ -475,11 +785,10 @@ int kq_fold_weights(const float *W, const float *factors, int shared, float *W_o
     if (!W || !factors || !W_out) return fail(KQ_ERR_NULL, "kq_fold_weights: NULL pointer argument");
     if (!aligned(W, 16) || !aligned(W_out, 16) || !aligned(factors, 16))
         return fail(KQ_ERR_ALIGN, "kq_fold_weights: W, W_out and factors must be 16-byte aligned");
-    int sms = 0;
-    int rc = sm_count(&sms);
-    if (rc != KQ_OK) return rc;
     const int64_t nb = d / kBlk;
-    const Geometry geo = pinned_geometry(N, nb, int64_t(sms) * kTargetThreadsPerSm);
+    Geometry geo;
+    int rc = launch_pinned("kq_fold_weights", kFold, fold_kernel, N, nb, &geo);
+    if (rc != KQ_OK) return rc;
     fold_kernel<<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(W),
                                                    reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
                                                    reinterpret_cast<float4 *>(W_out), N * nb, int(nb), geo.T);
