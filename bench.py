@@ -10,11 +10,11 @@ seeded synthetic activations).  The headline value is the KroQuant quantizer's
 algorithmic HBM throughput, 2.53125 bytes per element (2 B bf16 in, 0.5 B
 codes, 1/32 B scale) over the summed duration of its launches.
 
-Timing: inputs resident in HBM, rotated over 8 input sets (each launch reads a
-set that the previous 7 quantizer passes did not touch, > 6x the L2), launches
-captured in a CUDA graph of 200 steps and replayed; CUDA events on the
-launching stream bracket every launch of the last replay and the whole timed
-region; barrier + synchronize on both sides; max over ranks.  Multi-GPU: every
+Timing: inputs resident in HBM and rotated over per-layer input sets so that
+a set is read again only after >= 3x the L2 of other input; per (quantizer,
+layer) a CUDA graph of 200 back-to-back launches; a round replays the six
+graphs in step order; CUDA events on the launching stream sit between graph
+replays; barrier + synchronize on both sides; max over ranks.  Multi-GPU: every
 rank quantizes its own batch (weak scaling, no collective on the data path).
 
 `--impl reference` times the CPU oracle (oracle/, plain C) on the host cores on
@@ -42,8 +42,7 @@ if ROOT not in sys.path:
 METRIC = "KroQuant quantizer HBM GB/s (bf16→MXFP4+E8M0) and % of B200 peak vs SQ"
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
 WORKLOAD = "pixart"
-N_SETS = 8
-GRAPH_STEPS = 200          # a multiple of 8 so the set rotation is seamless across replays
+GRAPH_STEPS = 200          # launches per captured graph
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.cu")]
@@ -163,18 +162,31 @@ def allreduce_max(pg, values, device):
     return t.tolist()
 
 
+def allreduce_sum(pg, values, device):
+    if pg is None:
+        return values
+    import torch
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
+    return t.tolist()
+
+
 def barrier(pg):
     if pg is not None:
         pg.barrier()
 
 
 # ----------------------------------------------------------------------------- inputs
-def workload_inputs(seed_offset: int = 0):
-    from w4a4_mxfp4_post_b200 import synth
+def workload_inputs(seed_offset: int = 0, world: int = 1, rank: int = 0):
+    """Layer inputs of the workload: the whole batch (world == 1), or rank's rows of it."""
+    from w4a4_mxfp4_post_b200 import shard, synth
 
     layers = []
     for (M, d, model, shared, seed) in synth.workload_layers(WORKLOAD):
-        x = synth.activation(model, M, d, seed + seed_offset)
+        rows = shard.row_range(M, world, rank) if world > 1 else None
+        x = synth.activation(model, M, d, seed + seed_offset, rows=rows)
+        M = x.shape[0]
         F = synth.factors(d // 32, seed + seed_offset, shared=shared)
         m = synth.sq_multipliers(x)
         layers.append({"M": M, "d": d, "x": x, "F": F, "m": m, "shared": shared})
@@ -219,85 +231,78 @@ def gpu_arm(args, rank, local, world, pg):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    layers = workload_inputs(seed_offset=rank)
+    # weak: every rank quantizes its own batch; strong: the ranks split one batch by rows
+    if args.scaling == "weak":
+        layers = workload_inputs(seed_offset=rank)
+    else:
+        layers = workload_inputs(world=world, rank=rank)
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
 
-    # device buffers: N_SETS copies of every layer input, per-set outputs
-    sets = []
-    for s in range(N_SETS):
-        per = []
-        for L in layers:
-            M, d = L["M"], L["d"]
-            x = torch.from_numpy(L["x"].view(np.int16)).to(dev).view(torch.bfloat16)
-            per.append({
-                "x": x,
-                "F": torch.from_numpy(L["F"]).to(dev),
-                "m": torch.from_numpy(L["m"]).to(dev),
-                "codes": torch.empty((M, d // 2), dtype=torch.uint8, device=dev),
-                "scales": torch.empty((M, d // 32), dtype=torch.uint8, device=dev),
-                "shared": L["shared"],
-            })
-        sets.append(per)
-    set_bytes = sum(L["M"] * L["d"] * 2 for L in layers)
+    # device buffers: per layer, enough input sets that a set is reused only
+    # after >= 3x the L2 of other input has streamed by (and at least 4)
+    layer_sets = []
+    for L in layers:
+        M, d = L["M"], L["d"]
+        set_bytes = M * d * 2
+        nsets = max(4, math.ceil(3 * l2 / set_bytes) + 1)
+        x0 = torch.from_numpy(L["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+        xs = torch.empty((nsets, M, d), dtype=torch.bfloat16, device=dev)
+        xs[:] = x0
+        layer_sets.append({
+            "n": nsets, "x": xs,
+            "codes": torch.empty((nsets, M, d // 2), dtype=torch.uint8, device=dev),
+            "scales": torch.empty((nsets, M, d // 32), dtype=torch.uint8, device=dev),
+            "F": torch.from_numpy(L["F"]).to(dev), "m": torch.from_numpy(L["m"]).to(dev),
+            "shared": L["shared"],
+        })
+    resident = sum(ls["n"] * L["M"] * L["d"] * 2 for ls, L in zip(layer_sets, layers))
 
-    def kq_call(b, stream):
-        fn = kq.kq_quantize_shared if b["shared"] else kq.kq_quantize
-        fn(b["x"], b["F"], b["codes"], b["scales"], stream=stream)
+    def launch(q, li, i, stream):
+        ls = layer_sets[li]
+        k = i % ls["n"]
+        x, c, sc = ls["x"][k], ls["codes"][k], ls["scales"][k]
+        if q == "kq":
+            (kq.kq_quantize_shared if ls["shared"] else kq.kq_quantize)(x, ls["F"], c, sc, stream=stream)
+        elif q == "sq":
+            kq.sq_quantize(x, ls["m"], c, sc, stream=stream)
+        else:
+            kq.mx_quantize(x, c, sc, stream=stream)
 
-    def sq_call(b, stream):
-        kq.sq_quantize(b["x"], b["m"], b["codes"], b["scales"], stream=stream)
-
-    def mx_call(b, stream):
-        kq.mx_quantize(b["x"], b["codes"], b["scales"], stream=stream)
-
-    quantizers = [("kq", kq_call), ("sq", sq_call), ("mx", mx_call)]
+    quantizers = ("kq", "sq", "mx")
     n_layers = len(layers)
-
-    def step(i, stream, events=None):
-        # quantizer q of step i reads set (3 i + q) mod 8
-        k = 0
-        for q, (name, fn) in enumerate(quantizers):
-            for li in range(n_layers):
-                b = sets[(3 * i + q) % N_SETS][li]
-                fn(b, stream)
-                if events is not None:
-                    events[k + 1].record(stream)
-                k += 1
-
+    pairs = [(q, li) for q in quantizers for li in range(n_layers)]
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
-    # warm-up (eager)
+    # warm-up steps (eager)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            step(i, stream)
+            for q, li in pairs:
+                launch(q, li, i, stream)
     stream.synchronize()
 
-    # capture S steps with an event after every launch (events of the last replay are read)
+    # One CUDA graph per (quantizer, layer) holding S back-to-back launches;
+    # a round replays the six graphs in step order, so K steps = K/S rounds
+    # (the last round shorter).  Events sit only between graph replays.
     K = args.steps
     S = min(GRAPH_STEPS, K)
-    reps, tail = divmod(K, S)
-    n_launch = 3 * n_layers
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_launch + 1)] for _ in range(S)]
+    full, tail = divmod(K, S)
 
-    def capture(nsteps, with_events):
+    def capture(q, li, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for i in range(nsteps):
-                if with_events:
-                    ev[i][0].record(stream)
-                step(i, stream, ev[i] if with_events else None)
+            for i in range(n):
+                launch(q, li, i, stream)
         return g
 
-    g_main = capture(S, True)
-    g_tail = capture(tail, False) if tail else None
-    g_main.replay()
-    if g_tail:
-        g_tail.replay()
+    graphs = {pl: capture(*pl, S) for pl in pairs}
+    tails = {pl: capture(*pl, tail) for pl in pairs} if tail else {}
+    for g in list(graphs.values()) + list(tails.values()):
+        g.replay()
     stream.synchronize()
 
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    rounds = [graphs] * full + ([tails] if tail else [])
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(pairs) + 1)] for _ in rounds]
     uuid = getattr(props, "uuid", None)
     gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
     clocks = ClockSampler(gpu_id) if rank == 0 else None
@@ -306,27 +311,22 @@ def gpu_arm(args, rank, local, world, pg):
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    t_start.record(stream)
-    for _ in range(reps):
-        g_main.replay()
-    if g_tail:
-        g_tail.replay()
-    t_end.record(stream)
+    with torch.cuda.stream(stream):
+        for r, gs in enumerate(rounds):
+            evs[r][0].record(stream)
+            for k, pl in enumerate(pairs):
+                gs[pl].replay()
+                evs[r][k + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier(pg)
     clk = clocks.stop() if clocks else None
 
-    total_ms = t_start.elapsed_time(t_end)
-    # per-launch durations of the last main replay
-    per = {name: [0.0] * n_layers for name, _ in quantizers}
-    for i in range(S):
-        k = 0
-        for name, _ in quantizers:
-            for li in range(n_layers):
-                per[name][li] += ev[i][k].elapsed_time(ev[i][k + 1])
-                k += 1
-    us = {name: [1e3 * v / S for v in per[name]] for name in per}     # mean us per launch
-    step_ms = total_ms / K
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per = {q: [0.0] * n_layers for q in quantizers}
+    for r in range(len(rounds)):
+        for k, (q, li) in enumerate(pairs):
+            per[q][li] += evs[r][k].elapsed_time(evs[r][k + 1])
+    us = {q: [1e3 * v / K for v in per[q]] for q in per}      # mean us per launch, gaps in the graph included
 
     # kernel-only quantizer throughput from the per-launch means
     elems = [L["M"] * L["d"] for L in layers]
@@ -336,7 +336,8 @@ def gpu_arm(args, rank, local, world, pg):
     total_ms_max = vals[0]
     qt = dict(zip(("kq", "sq", "mx"), vals[1:4]))
     kq_us_max = vals[4:]
-    gbs = {n: world * qbytes / (qt[n] * 1e-6) / 1e9 for n in qt}
+    all_bytes = allreduce_sum(pg, [qbytes], dev)[0]          # units all ranks processed per step
+    gbs = {n: all_bytes / (qt[n] * 1e-6) / 1e9 for n in qt}
 
     # dominant kernel: the KroQuant launch on the largest layer
     dom = int(np.argmax(elems))
@@ -358,7 +359,7 @@ def gpu_arm(args, rank, local, world, pg):
         "warmup": args.warmup,
         "ms_per_step": round(total_ms_max / K, 6),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded PixArt-Sigma-shaped activations with per-channel outliers; no trained weights)",
@@ -366,10 +367,13 @@ def gpu_arm(args, rank, local, world, pg):
             "workload": "PixArt-Sigma layer inputs: M=8192 tokens x d in {1152, 4608}, bf16 -> MXFP4 (E2M1 codes + "
                         "E8M0 scales), per-block Kronecker factors",
             "M": layers[0]["M"], "d": [L["d"] for L in layers], "quantizers_per_step": ["kq", "sq", "mx"],
-            "l2": f"rotating {N_SETS} input sets ({N_SETS * set_bytes / 2**20:.0f} MiB, L2 {l2 / 2**20:.0f} MiB); "
-                  "each launch reads a set untouched by the previous 7 quantizer passes",
-            "timing": f"CUDA graph of {S} steps replayed; events around every launch of the last replay",
-            "parallelism": f"dp{world} (independent batches, no collective)",
+            "l2": f"inputs larger than L2: per layer {[ls['n'] for ls in layer_sets]} rotating input sets "
+                  f"({resident / 2**20:.0f} MiB resident, L2 {l2 / 2**20:.0f} MiB); a set is reused only after "
+                  ">= 3x L2 of other input",
+            "timing": f"per (quantizer, layer) a CUDA graph of {S} back-to-back launches; a step's six graphs "
+                      "replayed in order; CUDA events between replays on the launching stream",
+            "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'row shards of one batch'}"
+                           ", no collective on the data path)",
         },
         "kernels": {
             n: {"gbs": round(gbs[n], 1), "frac_of_peak": round(gbs[n] / peak, 4),
@@ -382,7 +386,7 @@ def gpu_arm(args, rank, local, world, pg):
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src},
         "e2e": e2e,
-        "gpu_launches": K * n_launch,
+        "gpu_launches": K * len(pairs),
         "clocks": clk,
         "kernel_source_sha": sha,
     }
@@ -512,10 +516,10 @@ class RotatingInputs:
 
 
 def time_launches(kind, inp, launches, warmup, stream, graph=True):
-    """Mean / median device time (us) of one quantizer launch over `launches` launches.
+    """Mean device time (us) per launch over `launches` back-to-back launches.
 
-    With graph=True the launches are captured in a CUDA graph with an event
-    after each one; the second replay is measured.
+    With graph=True the launches are captured in one CUDA graph and its second
+    replay is timed by two events around it (inter-launch gaps included).
     """
     import torch
 
@@ -538,26 +542,27 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
         for i in range(warmup):
             launch(i)
     stream.synchronize()
-    evs = [torch.cuda.Event(enable_timing=True, external=graph) for _ in range(launches + 1)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     if graph:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            evs[0].record(stream)
             for i in range(launches):
                 launch(i)
-                evs[i + 1].record(stream)
         g.replay()
         stream.synchronize()
-        g.replay()
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            g.replay()
+            t1.record(stream)
     else:
         with torch.cuda.stream(stream):
-            evs[0].record(stream)
+            t0.record(stream)
             for i in range(launches):
                 launch(i)
-                evs[i + 1].record(stream)
+            t1.record(stream)
     stream.synchronize()
-    times = [evs[i].elapsed_time(evs[i + 1]) * 1e3 for i in range(launches)]
-    return {"mean_us": float(np.mean(times)), "median_us": float(np.median(times)), "nsets": inp.nsets}
+    return {"mean_us": 1e3 * t0.elapsed_time(t1) / launches, "nsets": inp.nsets, "graph": graph}
 
 
 def kernel_mode(args):
@@ -621,6 +626,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="weak: a batch per rank; strong: the ranks split one batch by rows")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the cpu_baseline block")
     ap.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the reference arm")
     ap.add_argument("--json-out", default="")

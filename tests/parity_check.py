@@ -14,7 +14,8 @@ and ab = |K||x| (the scale of a dot product's rounding error):
              lies within w = 1e-5 * ab * 2^-e of a rounding boundary of E2M1
              (+-0.25, +-0.75, ..., +-5, or 0 for the sign of a zero); such
              "exempt" mismatches are counted and must stay <= 1e-6 of all codes;
-             any other mismatch fails.
+             any other mismatch fails.  (The 1e-6 rate is rounded up to a
+             whole code, so a case of fewer than 1e6 codes may show one.)
 
 SmoothQuant and plain MXFP4: codes and scales bit-exact, no exemptions (the
 fp32 product x * m is correctly rounded on both sides).
@@ -36,6 +37,15 @@ def nibbles(codes: np.ndarray) -> np.ndarray:
     out[..., 0::2] = c & 0xF
     out[..., 1::2] = c >> 4
     return out
+
+
+def allowed(n: int) -> int:
+    """Exempt mismatches allowed among n results: 1e-6 of them, rounded up to a whole one.
+
+    The rate bound is statistical; below a million codes a floor would allow
+    none, although one near-boundary flip is then expected now and then.
+    """
+    return math.ceil(EXEMPT_FRACTION * n)
 
 
 def scale_band_flags(y_ref: np.ndarray, ab: np.ndarray) -> np.ndarray:
@@ -94,8 +104,8 @@ def check_kq(codes_gpu, scales_gpu, codes_ref, scales_ref, y_ref, ab):
         "code_mismatch_nonexempt": n_mis - exempt,
     }
     res["ok"] = (scale_bad == 0 and res["code_mismatch_nonexempt"] == 0
-                 and exempt <= math.floor(EXEMPT_FRACTION * total_codes)
-                 and scale_flagged_mis <= max(1, math.floor(EXEMPT_FRACTION * nblk)))
+                 and exempt <= allowed(total_codes)
+                 and scale_flagged_mis <= allowed(nblk))
     return res
 
 

@@ -54,6 +54,20 @@ def test_hand_worked_blocks_on_gpu(cuda_device, case):
         assert int(s2.cpu()[0, 0]) == case["scale"]
 
 
+def test_exact_zeros_come_out_positive(cuda_device):
+    """An exactly cancelling sum is +0 (as in the oracle), whichever form the kernel uses."""
+    H = np.array([[1, 1], [1, -1]], np.float32)           # unit-diagonal split with D = diag(1, -1)
+    S = np.array([[0, 1], [1, 0]], np.float32)            # no split: the direct form
+    for F in (np.stack([H] * 5), np.stack([H, H, S, H, H])):
+        xb = bf16(np.ones((1, 32), np.float32))
+        y = kq.kq_transform_f32(dev_bf16(xb, cuda_device), dev_f32(F[None], cuda_device)).cpu().numpy()[0]
+        yr = oracle.kq_transform(xb, F[None])[0]
+        np.testing.assert_array_equal(y, yr)
+        zeros = yr == 0
+        assert zeros.sum() >= 30
+        assert not np.signbit(y[zeros]).any() and not np.signbit(yr[zeros]).any()
+
+
 RAGGED = [(1, 32), (3, 32), (37, 64), (5, 1152), (129, 5600), (7, 2240), (1000, 96), (2049, 160)]
 
 

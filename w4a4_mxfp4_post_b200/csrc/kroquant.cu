@@ -326,6 +326,8 @@ __device__ __forceinline__ void direct_stage2(float2 (&p)[16], float2 F00, float
 
 __device__ __forceinline__ float2 bcast(float v) { return make_float2(v, v); }
 
+__device__ __forceinline__ float2 plus_zero2() { return make_float2(0.0f, 0.0f); }
+
 // Unit-diagonal split of one factor; false if the factor is outside the range
 // where the split is used (see the kernel comment).
 __device__ __forceinline__ bool unit_split(const float4 g, float &d0, float &d1, float &b, float &c)
@@ -413,10 +415,13 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ facto
             unit_stage2<2>(p, B1, C1);
             unit_stage2<4>(p, B2, C2);
             unit_stage2<8>(p, B3, C3);
+            // D applied as D*z + (+0): the same value as D*z, except that an exact
+            // zero comes out as +0 whatever the signs of D and z (as a sum of
+            // products that cancels exactly does in round-to-nearest).
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float lo = p[i].x, hi = p[i].y;
-                p[i] = __fmul2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), DP[i]);
+                p[i] = __ffma2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), DP[i], plus_zero2());
             }
             if constexpr (OUT == KqOut::kCodes) {
                 uint4 c;
@@ -453,10 +458,11 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ facto
             direct_stage2<2>(p, E00, E01, E10, E11);
             direct_stage2<4>(p, H00, H01, H10, H11);
             direct_stage2<8>(p, J00, J01, J10, J11);
+            // last stage, with the same +0 canonicalisation of exact zeros
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const float lo = p[i].x, hi = p[i].y;
-                p[i] = make_float2(fmaf(G1.y, hi, G1.x * lo), fmaf(G1.w, hi, G1.z * lo));
+                p[i] = __fadd2_rn(make_float2(fmaf(G1.y, hi, G1.x * lo), fmaf(G1.w, hi, G1.z * lo)), plus_zero2());
             }
             if constexpr (OUT == KqOut::kCodes) {
                 uint4 c;
