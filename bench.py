@@ -300,6 +300,13 @@ def gpu_arm(args, rank, local, world, pg):
     for g in list(graphs.values()) + list(tails.values()):
         g.replay()
     stream.synchronize()
+    # more untimed rounds until the SM and HBM clocks have left their idle states
+    t_end = time.perf_counter() + SPINUP_S
+    with torch.cuda.stream(stream):
+        while time.perf_counter() < t_end:
+            for pl in pairs:
+                graphs[pl].replay()
+            stream.synchronize()
 
     rounds = [graphs] * full + ([tails] if tail else [])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(pairs) + 1)] for _ in rounds]
@@ -487,6 +494,22 @@ def reference_arm(args, rank, world):
     }
 
 
+SPINUP_S = 0.5
+
+
+def _replay_seconds(g, stream):
+    import torch
+
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) * 1e-3
+
+
 class RotatingInputs:
     """Device inputs of one [M, d] layer, split into sets that rotate past the L2.
 
@@ -535,6 +558,10 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
             kq.mx_quantize(inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
         elif kind.startswith("kq_v"):
             kq.kq_quantize_variant(int(kind[4:]), inp.xs[k], inp.F, False, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind.startswith("sq_v"):
+            kq.sq_quantize_variant(int(kind[4:]), inp.xs[k], inp.m, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind.startswith("mx_v"):
+            kq.mx_quantize_variant(int(kind[4:]), inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
         else:
             raise ValueError(f"unknown kernel {kind!r}")
 
@@ -549,12 +576,19 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
         with torch.cuda.graph(g, stream=stream):
             for i in range(launches):
                 launch(i)
-        g.replay()
-        stream.synchronize()
+        # spin the clocks up (SM and HBM leave their idle states only under
+        # sustained load): replay for >= SPINUP_S before the timed replays
+        t_end = time.perf_counter() + SPINUP_S
+        while time.perf_counter() < t_end:
+            g.replay()
+            stream.synchronize()
+        reps = max(1, int(0.2 / max(1e-6, _replay_seconds(g, stream))))
         with torch.cuda.stream(stream):
             t0.record(stream)
-            g.replay()
+            for _ in range(reps):
+                g.replay()
             t1.record(stream)
+        launches *= reps
     else:
         with torch.cuda.stream(stream):
             t0.record(stream)

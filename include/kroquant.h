@@ -109,12 +109,37 @@ int kq_fold_weights(const float *W, const float *factors, int shared,
 int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
                      float *out_y, int64_t M, int64_t d, cudaStream_t stream);
 
-/* Test export: the KroQuant quantizer through a chosen kernel variant.
- * variant 0 = the register-butterfly kernel that kq_quantize uses.  Other
- * values return KQ_ERR_VARIANT unless the library was built with them. */
+/* Test export: the KroQuant quantizer through a chosen kernel variant:
+ *   0  the default (what kq_quantize runs: 2),
+ *   1  one block per thread, direct 2x2 stages, 16-byte loads,
+ *   2  packed f32x2 pairs with the unit-diagonal split of each factor,
+ *      register prefetch,
+ *   3  the arithmetic of 2 on input staged through shared memory by TMA.
+ * Other values return KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
                         int shared, uint8_t *out_codes, uint8_t *out_scales,
                         int64_t M, int64_t d, cudaStream_t stream);
+
+/* Test exports: the baselines through a chosen kernel variant: 1 =
+ * register-prefetch kernel, 2 = TMA-staged kernel, 0 = the default (SQ: 2,
+ * MX: 1, the faster of the two on the benchmark shapes). */
+int sq_quantize_variant(int variant, const void *act_bf16, const float *mult,
+                        uint8_t *out_codes, uint8_t *out_scales,
+                        int64_t M, int64_t d, cudaStream_t stream);
+int mx_quantize_variant(int variant, const void *act_bf16,
+                        uint8_t *out_codes, uint8_t *out_scales,
+                        int64_t M, int64_t d, cudaStream_t stream);
+
+/* Diagnostics of the bounded waits (no counterpart on the pages).  The
+ * TMA-staged kernels wait on shared-memory barriers; every wait gives up after
+ * about a second of clock cycles, adds 1 to a device counter per giving-up
+ * thread, drains its copies in flight and returns, so the context stays
+ * usable.  kq_wait_timeouts copies the counter to *count (synchronising the
+ * device) and zeroes it if reset != 0.  kq_selftest_bounded_wait launches one
+ * staged CTA whose producer issues no copies, so its waits run out after about
+ * a millisecond; it reads and writes no memory other than the counter. */
+int kq_wait_timeouts(int *count, int reset);
+int kq_selftest_bounded_wait(cudaStream_t stream);
 
 /* Message for the last non-OK status returned on the calling thread (a static
  * thread-local buffer, valid until the thread's next call).  "" if none. */

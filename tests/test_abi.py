@@ -114,6 +114,14 @@ def test_alignment_errors(L):
     assert "aligned" in err(L)
 
 
+def test_variant_errors_before_cuda(L):
+    assert L.kq_quantize_variant(9, P(16), P(16), 0, P(16), P(16), 4, 64, None) == -5
+    assert L.sq_quantize_variant(5, P(16), P(16), P(16), P(16), 4, 64, None) == -5
+    assert L.mx_quantize_variant(-1, P(16), P(16), P(16), 4, 64, None) == -5
+    assert "variant" in err(L)
+    assert L.kq_wait_timeouts(None, 0) == -1
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
 

@@ -183,6 +183,55 @@ def test_variants_agree_with_oracle(cuda_device):
     assert tried >= 1
 
 
+VARIANT_SHAPES = [(1, 32), (37, 64), (129, 5600), (257, 2240), (1000, 1152), (300, 12288)]
+
+
+@pytest.mark.parametrize("M,d", VARIANT_SHAPES, ids=[f"{M}x{d}" for M, d in VARIANT_SHAPES])
+def test_baseline_variants_bit_exact(cuda_device, M, d):
+    """Register-prefetch and TMA-staged SQ/MX kernels agree bit for bit with the oracle
+    (ragged final stage, odd block counts, a single block)."""
+    x = synth.activation("pixart", M, d, seed=M * 7 + d)
+    m = synth.sq_multipliers(x)
+    xd, md = dev_bf16(x, cuda_device), dev_f32(m, cuda_device)
+    rs, rm = oracle.sq_quantize(x, m), oracle.mx_quantize(x)
+    for v in (1, 2):
+        c, s = kq.sq_quantize_variant(v, xd, md)
+        assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *rs)["ok"], ("sq", v)
+        c, s = kq.mx_quantize_variant(v, xd)
+        assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *rm)["ok"], ("mx", v)
+
+
+@pytest.mark.parametrize("M,d", VARIANT_SHAPES, ids=[f"{M}x{d}" for M, d in VARIANT_SHAPES])
+def test_kq_variants_2_and_3_identical(cuda_device, M, d):
+    """Variants 2 and 3 share the arithmetic, so their outputs are identical."""
+    x = synth.activation("pixart", M, d, seed=M * 3 + d)
+    F = synth.factors(d // 32, seed=d + 1)
+    xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
+    c2, s2 = kq.kq_quantize_variant(2, xd, Fd)
+    c3, s3 = kq.kq_quantize_variant(3, xd, Fd)
+    assert bool((c2 == c3).all()) and bool((s2 == s3).all())
+    F1 = synth.factors(1, seed=d, shared=True)
+    c2, s2 = kq.kq_quantize_variant(2, xd, dev_f32(F1, cuda_device), shared=True)
+    c3, s3 = kq.kq_quantize_variant(3, xd, dev_f32(F1, cuda_device), shared=True)
+    assert bool((c2 == c3).all()) and bool((s2 == s3).all())
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable(cuda_device):
+    """A staged CTA whose producer issues no copies: its waits run out, the
+    device counter records it, and the next launches still work."""
+    import torch
+
+    kq.kq_wait_timeouts(reset=True)
+    kq.kq_selftest_bounded_wait()
+    torch.cuda.synchronize()
+    assert kq.kq_wait_timeouts(reset=True) > 0
+    M, d = 64, 128
+    x = synth.activation("tiny", M, d, 0)
+    c, s = kq.mx_quantize(dev_bf16(x, cuda_device))
+    assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *oracle.mx_quantize(x))["ok"]
+    assert kq.kq_wait_timeouts() == 0
+
+
 def test_zero_rows_and_nondefault_stream(cuda_device):
     import torch
 

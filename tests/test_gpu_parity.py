@@ -85,6 +85,7 @@ def test_kq_sq_mx_full(cuda_device, M, d, model, shared, seed):
     r = pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *oracle.mx_quantize(x))
     report(f"mx-{model}-{M}x{d}", r)
     assert r["ok"], r
+    assert kq.kq_wait_timeouts() == 0       # no bounded wait gave up on the normal path
 
 
 SWEEP = [(M, d) for M in synth.WORKLOADS["sweep"]["Ms"] for d in synth.WORKLOADS["sweep"]["ds"]]

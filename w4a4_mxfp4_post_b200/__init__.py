@@ -24,6 +24,7 @@ __all__ = [
     "LIB_PATH", "KQ_OK", "KQ_ERR_NULL", "KQ_ERR_SHAPE", "KQ_ERR_ALIGN", "KQ_ERR_CUDA", "KQ_ERR_VARIANT",
     "KroQuantError", "lib", "kq_quantize", "kq_quantize_shared", "kq_quantize_variant", "sq_quantize",
     "mx_quantize", "kq_fold_weights", "kq_transform_f32", "kq_last_error", "kq_abi_version",
+    "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -35,6 +36,9 @@ _SIGS = {
     "kq_quantize": "ppppqqp",
     "kq_quantize_shared": "ppppqqp",
     "kq_quantize_variant": "ippippqqp",
+    "sq_quantize_variant": "ippppqqp",
+    "mx_quantize_variant": "ipppqqp",
+    "kq_selftest_bounded_wait": "p",
     "sq_quantize": "ppppqqp",
     "mx_quantize": "pppqqp",
     "kq_fold_weights": "ppipqqp",
@@ -70,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.kq_last_error.restype = ctypes.c_char_p
         L.kq_abi_version.argtypes = []
         L.kq_abi_version.restype = ctypes.c_int
+        L.kq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+        L.kq_wait_timeouts.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -196,6 +202,40 @@ def mx_quantize(act, out_codes=None, out_scales=None, stream=None):
     out_codes, out_scales = _outs(act, out_codes, out_scales)
     _call("mx_quantize", _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
     return out_codes, out_scales
+
+
+def sq_quantize_variant(variant, act, mult, out_codes=None, out_scales=None, stream=None):
+    """The SmoothQuant quantizer through a chosen kernel variant (0 = the default)."""
+    torch = _torch()
+    M, d = _act(act)
+    _need(mult, "mult", torch.float32, act.device, (d,))
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("sq_quantize_variant", int(variant), _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream))
+    return out_codes, out_scales
+
+
+def mx_quantize_variant(variant, act, out_codes=None, out_scales=None, stream=None):
+    """The plain MXFP4 quantizer through a chosen kernel variant (0 = the default)."""
+    M, d = _act(act)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("mx_quantize_variant", int(variant), _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream))
+    return out_codes, out_scales
+
+
+def kq_wait_timeouts(reset: bool = False) -> int:
+    """Number of bounded waits that gave up in the staged kernels (synchronises the device)."""
+    v = ctypes.c_int(0)
+    rc = lib().kq_wait_timeouts(ctypes.byref(v), int(bool(reset)))
+    if rc != KQ_OK:
+        raise KroQuantError("kq_wait_timeouts", rc, kq_last_error())
+    return v.value
+
+
+def kq_selftest_bounded_wait(stream=None) -> None:
+    """Launch one staged CTA whose waits run out (no copies issued); see the C header."""
+    _call("kq_selftest_bounded_wait", _stream(stream))
 
 
 def kq_fold_weights(W, factors, shared=False, out=None, stream=None):

@@ -16,6 +16,7 @@
 // consecutive threads own consecutive blocks of the flattened [M*d/32] block
 // array, so a warp reads 2 KB contiguous and writes 512 B of codes and 32 B of
 // scales contiguous.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -348,6 +349,103 @@ __device__ __forceinline__ void load_block_nc(const uint4 *__restrict__ act, int
     for (int q = 0; q < 4; ++q) raw[q] = __ldg(p + q);
 }
 
+// Column state of the KroQuant transform in unit-diagonal form (see the
+// variant-2 kernel below for the derivation).
+struct KqFast {
+    float2 DP[16];            // (D_i, D_{i+16})
+    float2 B[4], C[4];        // stages on bits 0..3 (G5, G4, G3, G2), broadcast
+    float b4, c4;             // stage on bit 4 (G1)
+};
+
+__device__ __forceinline__ bool kq_fast_setup(const float4 (&g)[5], KqFast &st)
+{
+    float d0[5], d1[5], bb[5], cc[5];
+    bool fast = true;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) fast &= unit_split(g[k], d0[k], d1[k], bb[k], cc[k]);
+    // D_i = prod_k (bit (4-k) of i ? g11_k : g00_k); factor k = 0 (G1) acts on bit 4.
+    float dd[32];
+    dd[0] = 1.0f;
+#pragma unroll
+    for (int bit = 0; bit < 5; ++bit) {
+        const int k = 4 - bit;
+#pragma unroll
+        for (int i = 0; i < (1 << bit); ++i) {
+            dd[i + (1 << bit)] = dd[i] * d1[k];
+            dd[i] = dd[i] * d0[k];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st.DP[i] = make_float2(dd[i], dd[i + 16]);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        st.B[b] = bcast(bb[4 - b]);
+        st.C[b] = bcast(cc[4 - b]);
+    }
+    st.b4 = bb[0];
+    st.c4 = cc[0];
+    return fast;
+}
+
+__device__ __forceinline__ void kq_fast_apply(float2 (&p)[16], const KqFast &st)
+{
+    unit_stage2<1>(p, st.B[0], st.C[0]);
+    unit_stage2<2>(p, st.B[1], st.C[1]);
+    unit_stage2<4>(p, st.B[2], st.C[2]);
+    unit_stage2<8>(p, st.B[3], st.C[3]);
+    // D applied as D*z + (+0): the same value as D*z, except that an exact
+    // zero comes out as +0 whatever the signs of D and z (as a sum of
+    // products that cancels exactly does in round-to-nearest).
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float lo = p[i].x, hi = p[i].y;
+        p[i] = __ffma2_rn(make_float2(fmaf(st.b4, hi, lo), fmaf(st.c4, lo, hi)), st.DP[i], plus_zero2());
+    }
+}
+
+// The direct form, y_lo = g00 lo + g01 hi, y_hi = g10 lo + g11 hi per stage.
+__device__ __forceinline__ void kq_direct_apply(float2 (&p)[16], const float4 (&g)[5])
+{
+    direct_stage2<1>(p, bcast(g[4].x), bcast(g[4].y), bcast(g[4].z), bcast(g[4].w));
+    direct_stage2<2>(p, bcast(g[3].x), bcast(g[3].y), bcast(g[3].z), bcast(g[3].w));
+    direct_stage2<4>(p, bcast(g[2].x), bcast(g[2].y), bcast(g[2].z), bcast(g[2].w));
+    direct_stage2<8>(p, bcast(g[1].x), bcast(g[1].y), bcast(g[1].z), bcast(g[1].w));
+    // last stage, with the same +0 canonicalisation of exact zeros
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float lo = p[i].x, hi = p[i].y;
+        p[i] = __fadd2_rn(make_float2(fmaf(g[0].y, hi, g[0].x * lo), fmaf(g[0].w, hi, g[0].z * lo)),
+                          plus_zero2());
+    }
+}
+
+template <KqOut OUT>
+__device__ __forceinline__ void kq_emit(float2 (&p)[16], int64_t gi, uint4 *__restrict__ codes,
+                                        uint8_t *__restrict__ scales, float4 *__restrict__ y_out)
+{
+    if constexpr (OUT == KqOut::kCodes) {
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[gi] = c;
+        scales[gi] = uint8_t(sb);
+    } else {
+        float4 *yo = y_out + gi * 8;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            yo[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
+            yo[q + 4] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
+        }
+    }
+}
+
+__device__ __forceinline__ void load_factors(const float4 *__restrict__ factors, int shared, int j, float4 (&g)[5])
+{
+    const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) g[k] = __ldg(fp + k);
+}
+
 // KroQuant quantizer, packed butterfly (variant 2).
 //
 // Each 2x2 factor is split as G = [[g00, g01], [g10, g11]]
@@ -369,115 +467,37 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ facto
 {
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
-    const int j = int(t % nb);
-    const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
     float4 g[5];
-#pragma unroll
-    for (int k = 0; k < 5; ++k) g[k] = __ldg(fp + k);
-
-    float d0[5], d1[5], bb[5], cc[5];
-    bool fast = true;
-#pragma unroll
-    for (int k = 0; k < 5; ++k) fast &= unit_split(g[k], d0[k], d1[k], bb[k], cc[k]);
+    load_factors(factors, shared, int(t % nb), g);
+    KqFast st;
+    const bool fast = kq_fast_setup(g, st);
 
     int64_t gi = t;
     uint4 raw[4];
     load_block_nc(act, gi, raw);
-
     if (fast) {
-        // D_i = prod_k (bit (4-k) of i ? g11_k : g00_k); factor k = 0 (G1) acts on bit 4.
-        float dd[32];
-        dd[0] = 1.0f;
-#pragma unroll
-        for (int bit = 0; bit < 5; ++bit) {
-            const int k = 4 - bit;
-#pragma unroll
-            for (int i = 0; i < (1 << bit); ++i) {
-                dd[i + (1 << bit)] = dd[i] * d1[k];
-                dd[i] = dd[i] * d0[k];
-            }
-        }
-        float2 DP[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) DP[i] = make_float2(dd[i], dd[i + 16]);
-        const float2 B0 = bcast(bb[4]), C0 = bcast(cc[4]);   // G5, bit 0
-        const float2 B1 = bcast(bb[3]), C1 = bcast(cc[3]);   // G4, bit 1
-        const float2 B2 = bcast(bb[2]), C2 = bcast(cc[2]);   // G3, bit 2
-        const float2 B3 = bcast(bb[1]), C3 = bcast(cc[1]);   // G2, bit 3
-        const float b4 = bb[0], c4 = cc[0];                  // G1, bit 4
         for (;;) {
             const int64_t gn = gi + T;
             uint4 nxt[4];
             if (gn < nblocks) load_block_nc(act, gn, nxt);
             float2 p[16];
             unpack_pairs(raw, p);
-            unit_stage2<1>(p, B0, C0);
-            unit_stage2<2>(p, B1, C1);
-            unit_stage2<4>(p, B2, C2);
-            unit_stage2<8>(p, B3, C3);
-            // D applied as D*z + (+0): the same value as D*z, except that an exact
-            // zero comes out as +0 whatever the signs of D and z (as a sum of
-            // products that cancels exactly does in round-to-nearest).
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float lo = p[i].x, hi = p[i].y;
-                p[i] = __ffma2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), DP[i], plus_zero2());
-            }
-            if constexpr (OUT == KqOut::kCodes) {
-                uint4 c;
-                uint32_t sb;
-                mx_quantize_pairs(p, c, sb);
-                codes[gi] = c;
-                scales[gi] = uint8_t(sb);
-            } else {
-                float4 *yo = y_out + gi * 8;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    yo[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
-                    yo[q + 4] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
-                }
-            }
+            kq_fast_apply(p, st);
+            kq_emit<OUT>(p, gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
             gi = gn;
         }
     } else {
-        const float2 A00 = bcast(g[4].x), A01 = bcast(g[4].y), A10 = bcast(g[4].z), A11 = bcast(g[4].w);
-        const float2 E00 = bcast(g[3].x), E01 = bcast(g[3].y), E10 = bcast(g[3].z), E11 = bcast(g[3].w);
-        const float2 H00 = bcast(g[2].x), H01 = bcast(g[2].y), H10 = bcast(g[2].z), H11 = bcast(g[2].w);
-        const float2 J00 = bcast(g[1].x), J01 = bcast(g[1].y), J10 = bcast(g[1].z), J11 = bcast(g[1].w);
-        const float4 G1 = g[0];
         for (;;) {
             const int64_t gn = gi + T;
             uint4 nxt[4];
             if (gn < nblocks) load_block_nc(act, gn, nxt);
             float2 p[16];
             unpack_pairs(raw, p);
-            direct_stage2<1>(p, A00, A01, A10, A11);
-            direct_stage2<2>(p, E00, E01, E10, E11);
-            direct_stage2<4>(p, H00, H01, H10, H11);
-            direct_stage2<8>(p, J00, J01, J10, J11);
-            // last stage, with the same +0 canonicalisation of exact zeros
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float lo = p[i].x, hi = p[i].y;
-                p[i] = __fadd2_rn(make_float2(fmaf(G1.y, hi, G1.x * lo), fmaf(G1.w, hi, G1.z * lo)), plus_zero2());
-            }
-            if constexpr (OUT == KqOut::kCodes) {
-                uint4 c;
-                uint32_t sb;
-                mx_quantize_pairs(p, c, sb);
-                codes[gi] = c;
-                scales[gi] = uint8_t(sb);
-            } else {
-                float4 *yo = y_out + gi * 8;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    yo[q] = make_float4(p[4 * q].x, p[4 * q + 1].x, p[4 * q + 2].x, p[4 * q + 3].x);
-                    yo[q + 4] = make_float4(p[4 * q].y, p[4 * q + 1].y, p[4 * q + 2].y, p[4 * q + 3].y);
-                }
-            }
+            kq_direct_apply(p, g);
+            kq_emit<OUT>(p, gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
@@ -559,6 +579,264 @@ mx_packed_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8
 }
 
 // ---------------------------------------------------------------------------
+// TMA-staged kernels.  The activation, viewed as a [nblocks][32] bf16 matrix
+// (one 64-byte row per block), streams through a ring of kStages
+// shared-memory stages of kStageRows rows each: one producer thread issues a
+// 2-D tensor copy (cp.async.bulk.tensor) per stage and mbarriers hand stages
+// between it and the consumer warps.  So the bytes in flight per SM no longer
+// depend on registers (2 CTAs x 4 stages x 16 KB), unlike a register
+// prefetch.  The copies use the 64-byte swizzle: the 16-byte chunk q of row r
+// lands at chunk q ^ ((r >> 1) & 3), which makes the consumers' 16-byte
+// shared loads (8 lanes per phase reading 8 consecutive rows) conflict-free.
+// Every wait is bounded by a clock budget; a wait that gives up records it
+// in g_wait_timeouts, and the kernel drains its copies in flight (again
+// bounded) before it returns, so a fault elsewhere cannot hang the GPU here.
+// ---------------------------------------------------------------------------
+constexpr int kStageRows = 256;                        // blocks per stage: one per consumer thread
+constexpr int kStageBytes = kStageRows * 64;           // 16 KB
+constexpr int kStages = 4;
+constexpr int kConsumers = 256;
+constexpr int kStagedThreads = kConsumers + 32;        // + one producer warp
+constexpr size_t kStagedSmem = size_t(kStages) * kStageBytes + 1024 + 2 * kStages * sizeof(uint64_t);
+
+__device__ int g_wait_timeouts;
+__device__ __align__(256) uint8_t g_selftest_dummy[256];
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done)
+                 : "r"(smem_addr(bar)), "r"(parity)
+                 : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete; false if `budget`
+// clock cycles pass first (the caller then records the timeout and unwinds).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long budget)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > budget) return false;
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_rows(void *dst, const CUtensorMap *map, int32_t row, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(smem_addr(bar))
+        : "memory");
+}
+
+struct StagedRing {
+    uint8_t *stage;
+    uint64_t *full;
+    uint64_t *empty;
+};
+
+// Carve the ring out of dynamic shared memory (stages aligned to 1 KB for the
+// swizzle) and initialise the barriers; every thread of the CTA calls this.
+__device__ __forceinline__ StagedRing staged_setup()
+{
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    StagedRing r;
+    r.stage = base;
+    r.full = reinterpret_cast<uint64_t *>(base + size_t(kStages) * kStageBytes);
+    r.empty = r.full + kStages;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&r.full[s], 1);
+            mbar_init(&r.empty[s], kConsumers / 32);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    return r;
+}
+
+// Producer (one thread): fill stage k % kStages with chunk c = blockIdx.x +
+// k * gridDim.x, after the consumers have released the stage's previous use.
+// issue_copies == 0 issues nothing (used only to test the bounded waits).
+__device__ void staged_produce(const StagedRing &r, const CUtensorMap *map, int64_t nchunks, long long budget,
+                               int issue_copies)
+{
+    int k = 0;
+    int filled = 0;                          // number of fills issued
+    for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+        const int s = k % kStages;
+        if (k >= kStages && !mbar_wait(&r.empty[s], ((k / kStages) - 1) & 1, budget)) {
+            atomicAdd(&g_wait_timeouts, 1);
+            break;
+        }
+        if (!issue_copies) continue;
+        mbar_expect_tx(&r.full[s], kStageBytes);
+        tma_load_rows(r.stage + size_t(s) * kStageBytes, map, int32_t(c * kStageRows), &r.full[s]);
+        filled = k + 1;
+    }
+    // Drain: every issued copy has landed before this thread (and so the CTA)
+    // can exit.  On the normal path the consumers have waited on all of them.
+    for (int kk = (filled > kStages ? filled - kStages : 0); kk < filled; ++kk) {
+        if (!mbar_wait(&r.full[kk % kStages], (kk / kStages) & 1, budget)) {
+            atomicAdd(&g_wait_timeouts, 1);
+            break;
+        }
+    }
+}
+
+// Consumer loop: thread tid owns row tid of every stage, i.e. block
+// g = c * kStageRows + tid.  f(raw, g) runs for the rows below nblocks.
+// Returns false after a timeout (recorded).
+template <class F>
+__device__ __forceinline__ bool staged_consume(const StagedRing &r, int64_t nchunks, int64_t nblocks, long long budget,
+                                               F &&f)
+{
+    const int tid = threadIdx.x;
+    const int sw = (tid >> 1) & 3;
+    int k = 0;
+    for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x, ++k) {
+        const int s = k % kStages;
+        if (!mbar_wait(&r.full[s], (k / kStages) & 1, budget)) {
+            atomicAdd(&g_wait_timeouts, 1);
+            return false;
+        }
+        const uint8_t *row = r.stage + size_t(s) * kStageBytes + size_t(tid) * 64;
+        uint4 raw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) raw[q] = *reinterpret_cast<const uint4 *>(row + 16 * (q ^ sw));
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(&r.empty[s]);
+        const int64_t g = c * kStageRows + tid;
+        if (g < nblocks) f(raw, g);
+    }
+    return true;
+}
+
+// KroQuant quantizer, TMA-staged (variant 3): the arithmetic of variant 2
+// (kq_fast_apply / kq_direct_apply) on blocks read from the staged ring.
+// The grid is a multiple of nb / gcd(nb, kStageRows), so gridDim.x *
+// kStageRows is a multiple of nb and a thread's column j never changes.
+__global__ void __launch_bounds__(kStagedThreads, 2)
+kq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const float4 *__restrict__ factors, int shared,
+                 uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb,
+                 long long budget, int issue_copies)
+{
+    const StagedRing r = staged_setup();
+    const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
+    if (threadIdx.x >= kConsumers) {
+        if (threadIdx.x == kConsumers) staged_produce(r, &act_map, nchunks, budget, issue_copies);
+        return;
+    }
+    const int j = int((int64_t(blockIdx.x) * kStageRows + threadIdx.x) % nb);
+    float4 g[5];
+    load_factors(factors, shared, j, g);
+    KqFast st;
+    if (kq_fast_setup(g, st)) {
+        staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
+            float2 p[16];
+            unpack_pairs(raw, p);
+            kq_fast_apply(p, st);
+            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+        });
+    } else {
+        staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
+            float2 p[16];
+            unpack_pairs(raw, p);
+            kq_direct_apply(p, g);
+            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+        });
+    }
+}
+
+// SmoothQuant quantizer, TMA-staged.
+__global__ void __launch_bounds__(kStagedThreads, 2)
+sq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const float4 *__restrict__ mult,
+                 uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, long long budget,
+                 int issue_copies)
+{
+    const StagedRing r = staged_setup();
+    const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
+    if (threadIdx.x >= kConsumers) {
+        if (threadIdx.x == kConsumers) staged_produce(r, &act_map, nchunks, budget, issue_copies);
+        return;
+    }
+    const int j = int((int64_t(blockIdx.x) * kStageRows + threadIdx.x) % nb);
+    float m[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 a = __ldg(mult + int64_t(j) * 8 + q);
+        m[4 * q] = a.x;
+        m[4 * q + 1] = a.y;
+        m[4 * q + 2] = a.z;
+        m[4 * q + 3] = a.w;
+    }
+    float2 MP[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) MP[i] = make_float2(m[i], m[i + 16]);
+    staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
+        float2 p[16];
+        unpack_pairs(raw, p);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = __fmul2_rn(p[i], MP[i]);
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[gi] = c;
+        scales[gi] = uint8_t(sb);
+    });
+}
+
+// Plain MXFP4 quantizer, TMA-staged.
+__global__ void __launch_bounds__(kStagedThreads, 2)
+mx_staged_kernel(const __grid_constant__ CUtensorMap act_map, uint4 *__restrict__ codes,
+                 uint8_t *__restrict__ scales, int64_t nblocks, long long budget, int issue_copies)
+{
+    const StagedRing r = staged_setup();
+    const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
+    if (threadIdx.x >= kConsumers) {
+        if (threadIdx.x == kConsumers) staged_produce(r, &act_map, nchunks, budget, issue_copies);
+        return;
+    }
+    staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
+        float2 p[16];
+        unpack_pairs(raw, p);
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[gi] = c;
+        scales[gi] = uint8_t(sb);
+    });
+}
+
+// ---------------------------------------------------------------------------
 // launch geometry
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;
@@ -607,7 +885,10 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 
 // Resident threads of a kernel on the current device: SMs x resident CTAs
 // per SM (occupancy query, cached per device and kernel).
-enum KernelId { kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold, kNumKernels };
+enum KernelId {
+    kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
+    kKqStaged, kSqStaged, kMxStaged, kNumKernels
+};
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
 int resident_threads(KernelId id, const void *fn, int64_t *out)
@@ -653,6 +934,106 @@ int check_quant_args(const char *fn, const void *act, const void *params, bool n
     return KQ_OK;
 }
 
+// --- TMA-staged launches -----------------------------------------------------
+// cuTensorMapEncodeTiled is looked up through the runtime, so the library
+// needs no link-time dependency on the driver library.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::atomic<EncodeTiledFn> g_encode{nullptr};
+
+int encode_fn(EncodeTiledFn *out)
+{
+    EncodeTiledFn f = g_encode.load(std::memory_order_acquire);
+    if (!f) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled not available: %s", cudaGetErrorString(e));
+        f = reinterpret_cast<EncodeTiledFn>(p);
+        g_encode.store(f, std::memory_order_release);
+    }
+    *out = f;
+    return KQ_OK;
+}
+
+// The activation as a [nblocks][32] bf16 matrix, boxes of kStageRows rows,
+// 64-byte swizzle (the row is exactly one 64-byte swizzle span).
+int encode_act_map(const void *act, int64_t nblocks, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const cuuint64_t dims[2] = {32, cuuint64_t(nblocks)};
+    const cuuint64_t strides[1] = {64};
+    const cuuint32_t box[2] = {32, cuuint32_t(kStageRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(act), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
+std::atomic<int> g_smem_set[kNumKernels][kMaxDevices];
+
+// Dynamic shared memory above 48 KB needs an opt-in per kernel and device.
+int staged_prepare(KernelId id, const void *fn, int64_t *ctas_total)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices || !g_smem_set[id][dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kStagedSmem));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_smem_set[id][dev].store(1, std::memory_order_release);
+    }
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    int c = (dev >= 0 && dev < kMaxDevices) ? g_ctas_per_sm[id][dev].load(std::memory_order_relaxed) : 0;
+    if (c <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, fn, kStagedThreads, kStagedSmem);
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+        if (c < 1) c = 1;
+        if (dev >= 0 && dev < kMaxDevices) g_ctas_per_sm[id][dev].store(c, std::memory_order_relaxed);
+    }
+    *ctas_total = int64_t(sms) * c;
+    return KQ_OK;
+}
+
+int64_t gcd64(int64_t a, int64_t b)
+{
+    while (b) {
+        const int64_t t = a % b;
+        a = b;
+        b = t;
+    }
+    return a;
+}
+
+// Grid of the staged kernels: a multiple of q = nb / gcd(nb, kStageRows), so
+// that gridDim.x * kStageRows is a multiple of nb (fixed column per thread),
+// as close to the resident-CTA count as that allows and no larger than the
+// work needs.
+unsigned staged_grid(int64_t nblocks, int64_t nb, int64_t resident)
+{
+    const int64_t q = nb / gcd64(nb, kStageRows);
+    const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
+    int64_t grid = (resident / q) * q;
+    if (grid < q) grid = q;
+    const int64_t need = ((nchunks + q - 1) / q) * q;
+    if (grid > need) grid = need;
+    return unsigned(grid);
+}
+
+// Default clock budget of a bounded wait: 2^31 cycles, about a second.
+constexpr long long kWaitBudget = 1LL << 31;
+
+// Largest block count the staged path takes (row coordinates are int32).
+constexpr int64_t kStagedMaxBlocks = (int64_t(1) << 31) - kStageRows;
+
 template <typename Kernel>
 int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t nb, Geometry *geo)
 {
@@ -665,7 +1046,10 @@ int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t
 }
 
 // Kernel variants of the KroQuant quantizer: 1 = one block per thread, direct
-// 2x2 stages; 2 = packed pairs with the unit-diagonal split.  0 = the default.
+// 2x2 stages; 2 = packed pairs with the unit-diagonal split, register
+// prefetch; 3 = the arithmetic of 2 on TMA-staged input.  0 = the default,
+// the fastest on the benchmark shapes (2: the staged input does not help a
+// kernel whose limit is its instruction stream; see the profiles).
 constexpr int kDefaultVariant = 2;
 
 int kq_launch(const char *fn, int variant, const void *act, const float *factors, int shared,
@@ -676,14 +1060,24 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
     if (variant == 0) variant = kDefaultVariant;
-    if (variant != 1 && variant != 2)
+    if (variant < 1 || variant > 3)
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    // the fp32 export and very large inputs use the variant-2 kernel (same arithmetic as 3)
+    if (variant == 3 && (f32 || M * (d / kBlk) > kStagedMaxBlocks)) variant = 2;
     const int64_t nb = d / kBlk;
     const int64_t nblocks = M * nb;
     const uint4 *a = static_cast<const uint4 *>(act);
     const float4 *f = reinterpret_cast<const float4 *>(factors);
     Geometry geo;
-    if (variant == 1) {
+    if (variant == 3) {
+        CUtensorMap map;
+        if ((rc = encode_act_map(act, nblocks, &map)) != KQ_OK) return rc;
+        int64_t resident = 0;
+        if ((rc = staged_prepare(kKqStaged, reinterpret_cast<const void *>(kq_staged_kernel), &resident)) != KQ_OK)
+            return rc;
+        kq_staged_kernel<<<staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream>>>(
+            map, f, shared, reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb), kWaitBudget, 1);
+    } else if (variant == 1) {
         if (f32) {
             auto k = kq_butterfly_kernel<KqOut::kF32>;
             if ((rc = launch_pinned(fn, kKqDirectF32, k, M, nb, &geo)) != KQ_OK) return rc;
@@ -752,32 +1146,112 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared, flo
 int sq_quantize(const void *act_bf16, const float *mult, uint8_t *out_codes, uint8_t *out_scales, int64_t M,
                 int64_t d, cudaStream_t stream)
 {
-    int rc = check_quant_args("sq_quantize", act_bf16, mult, true, out_codes, out_scales, M, d);
-    if (rc == 1) return ok();
-    if (rc != KQ_OK) return rc;
-    const int64_t nb = d / kBlk;
-    Geometry geo;
-    if ((rc = launch_pinned("sq_quantize", kSqPacked, sq_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
-    sq_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
-                                                        reinterpret_cast<const float4 *>(mult),
-                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb,
-                                                        int(nb), geo.T);
-    return launch_check("sq_quantize");
+    return sq_quantize_variant(0, act_bf16, mult, out_codes, out_scales, M, d, stream);
 }
 
 int mx_quantize(const void *act_bf16, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
                 cudaStream_t stream)
 {
-    int rc = check_quant_args("mx_quantize", act_bf16, nullptr, false, out_codes, out_scales, M, d);
+    return mx_quantize_variant(0, act_bf16, out_codes, out_scales, M, d, stream);
+}
+
+int sq_quantize_variant(int variant, const void *act_bf16, const float *mult, uint8_t *out_codes,
+                        uint8_t *out_scales, int64_t M, int64_t d, cudaStream_t stream)
+{
+    const char *fn = "sq_quantize";
+    int rc = check_quant_args(fn, act_bf16, mult, true, out_codes, out_scales, M, d);
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
+    if (variant == 0) variant = 2;
+    if (variant != 1 && variant != 2)
+        return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
     const int64_t nb = d / kBlk;
+    const int64_t nblocks = M * nb;
+    if (variant == 2 && nblocks <= kStagedMaxBlocks) {
+        CUtensorMap map;
+        if ((rc = encode_act_map(act_bf16, nblocks, &map)) != KQ_OK) return rc;
+        int64_t resident = 0;
+        if ((rc = staged_prepare(kSqStaged, reinterpret_cast<const void *>(sq_staged_kernel), &resident)) != KQ_OK)
+            return rc;
+        sq_staged_kernel<<<staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream>>>(
+            map, reinterpret_cast<const float4 *>(mult), reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
+            int(nb), kWaitBudget, 1);
+        return launch_check(fn);
+    }
     Geometry geo;
-    if ((rc = launch_pinned("mx_quantize", kMxPacked, mx_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
+    if ((rc = launch_pinned(fn, kSqPacked, sq_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
+    sq_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                                        reinterpret_cast<const float4 *>(mult),
+                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
+                                                        int(nb), geo.T);
+    return launch_check(fn);
+}
+
+int mx_quantize_variant(int variant, const void *act_bf16, uint8_t *out_codes, uint8_t *out_scales, int64_t M,
+                        int64_t d, cudaStream_t stream)
+{
+    const char *fn = "mx_quantize";
+    int rc = check_quant_args(fn, act_bf16, nullptr, false, out_codes, out_scales, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    if (variant == 0) variant = 1;   // register prefetch: 4 CTAs/SM hide the latency already
+    if (variant != 1 && variant != 2)
+        return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    const int64_t nb = d / kBlk;
+    const int64_t nblocks = M * nb;
+    if (variant == 2 && nblocks <= kStagedMaxBlocks) {
+        CUtensorMap map;
+        if ((rc = encode_act_map(act_bf16, nblocks, &map)) != KQ_OK) return rc;
+        int64_t resident = 0;
+        if ((rc = staged_prepare(kMxStaged, reinterpret_cast<const void *>(mx_staged_kernel), &resident)) != KQ_OK)
+            return rc;
+        // any grid works for MX (no per-column state); keep the same sizing
+        mx_staged_kernel<<<staged_grid(nblocks, 1, resident), kStagedThreads, kStagedSmem, stream>>>(
+            map, reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks, kWaitBudget, 1);
+        return launch_check(fn);
+    }
+    Geometry geo;
+    if ((rc = launch_pinned(fn, kMxPacked, mx_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
     mx_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
-                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, M * nb,
+                                                        reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
                                                         geo.T);
-    return launch_check("mx_quantize");
+    return launch_check(fn);
+}
+
+int kq_wait_timeouts(int *count, int reset)
+{
+    if (!count) return fail(KQ_ERR_NULL, "kq_wait_timeouts: NULL pointer argument");
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_wait_timeouts, sizeof v);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "kq_wait_timeouts: %s", cudaGetErrorString(e));
+    if (reset) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof zero);
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "kq_wait_timeouts: %s", cudaGetErrorString(e));
+    }
+    *count = v;
+    return ok();
+}
+
+int kq_selftest_bounded_wait(cudaStream_t stream)
+{
+    // One CTA whose producer issues no copies: every consumer wait and the
+    // producer's own wait run out after ~2^21 cycles (about a millisecond).
+    // No memory is read or written besides the counter; the dummy address
+    // only has to satisfy the tensor map's alignment rule.
+    void *dummy = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&dummy, g_selftest_dummy);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "kq_selftest_bounded_wait: %s", cudaGetErrorString(e));
+    const int64_t nblocks = int64_t(kStageRows) * (kStages + 1);
+    CUtensorMap map;
+    int rc = encode_act_map(dummy, nblocks, &map);
+    if (rc != KQ_OK) return rc;
+    int64_t resident = 0;
+    if ((rc = staged_prepare(kMxStaged, reinterpret_cast<const void *>(mx_staged_kernel), &resident)) != KQ_OK)
+        return rc;
+    mx_staged_kernel<<<1, kStagedThreads, kStagedSmem, stream>>>(map, static_cast<uint4 *>(dummy),
+                                                                 static_cast<uint8_t *>(dummy), nblocks, 1LL << 21, 0);
+    return launch_check("kq_selftest_bounded_wait");
 }
 
 int kq_fold_weights(const float *W, const float *factors, int shared, float *W_out, int64_t N, int64_t d,
