@@ -536,6 +536,7 @@ class RotatingInputs:
         self.ss = torch.empty((self.nsets, M, d // 32), dtype=torch.uint8, device=dev)
         self.F = torch.from_numpy(F).to(dev)
         self.m = torch.from_numpy(m).to(dev)
+        self.P = torch.from_numpy(synth.lu_params(d // 32, 4)).to(dev)
 
 
 def time_launches(kind, inp, launches, warmup, stream, graph=True):
@@ -556,6 +557,10 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
             kq.sq_quantize(inp.xs[k], inp.m, inp.cs[k], inp.ss[k], stream=stream)
         elif kind == "mx":
             kq.mx_quantize(inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
+        elif kind == "kq_lu":
+            kq.kq_quantize_lu(inp.xs[k], inp.P, False, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind.startswith("fwht"):
+            kq.fwht_quantize(inp.xs[k], int(kind[4:]), inp.cs[k], inp.ss[k], stream=stream)
         elif kind.startswith("kq_v"):
             kq.kq_quantize_variant(int(kind[4:]), inp.xs[k], inp.F, False, inp.cs[k], inp.ss[k], stream=stream)
         elif kind.startswith("sq_v"):
@@ -667,7 +672,8 @@ def main():
     ap.add_argument("--json-out", default="")
     ap.add_argument("--mode", choices=["step", "kernel", "sweep"], default="step",
                     help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes")
-    ap.add_argument("--kernel", default="kq", help="kernel mode: kq, sq, mx or kq_v<variant>")
+    ap.add_argument("--kernel", default="kq",
+                    help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu or fwht<H>")
     ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
     ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD")
     ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")

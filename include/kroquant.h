@@ -94,6 +94,28 @@ int mx_quantize(const void *act_bf16,
                 uint8_t *out_codes, uint8_t *out_scales,
                 int64_t M, int64_t d, cudaStream_t stream);
 
+/* KroQuant quantizer from the LU parametrisation of each factor (KroQuant
+ * section 3.2, Eq. (6) as summarised by the Pith review): G_k = L_k U_k with
+ * U_k = [[a_k, b_k], [0, -1/a_k]] and L_k = [[1, 0], [c_k, 1]] (L unit lower
+ * triangular: a reading, the pages print only U), i.e.
+ * G_k = [[a_k, b_k], [c_k a_k, c_k b_k - 1/a_k]], det G_k = -1.
+ * lu_params: float32 [d/32][5][3] = (a, b, c) of G1..G5 per column block, 15
+ * scalars per block; shared != 0: one set [5][3] for every block.  Every
+ * a_k must be nonzero.  The factors are expanded in-kernel (the paper's
+ * on-the-fly "K2" kernel), then as kq_quantize.  lu_params: 4-byte aligned. */
+int kq_quantize_lu(const void *act_bf16, const float *lu_params, int shared,
+                   uint8_t *out_codes, uint8_t *out_scales,
+                   int64_t M, int64_t d, cudaStream_t stream);
+
+/* Fixed-Hadamard baseline (the pages' comparison point for the on-the-fly
+ * kernel, a fast Walsh-Hadamard transform): y = H_H x / sqrt(H) on every H
+ * consecutive channels of a row, H_H the Sylvester Hadamard matrix, H a
+ * power of two in [32, 1024] dividing d; then the MXFP4 block quantizer above
+ * on each 32-block.  H outside that set or d % H != 0 -> KQ_ERR_SHAPE. */
+int fwht_quantize(const void *act_bf16, int64_t H,
+                  uint8_t *out_codes, uint8_t *out_scales,
+                  int64_t M, int64_t d, cudaStream_t stream);
+
 /* Offline fold of the inverse transform into weights (Pith review, "key
  * machinery": the inverse is folded into the weights offline), used to check
  * invertibility: W_out = W T^-1, i.e. for every row n and column block j,
@@ -114,11 +136,18 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
  *   1  one block per thread, direct 2x2 stages, 16-byte loads,
  *   2  packed f32x2 pairs with the unit-diagonal split of each factor,
  *      register prefetch,
- *   3  the arithmetic of 2 on input staged through shared memory by TMA.
+ *   3  the arithmetic of 2 on input staged through shared memory by TMA,
+ *   4  the block transform on the tcgen05 tensor cores: Y_j = X_j K_j^T with
+ *      K_j expanded in fp32 and split into three bf16 parts (each product
+ *      exact in the fp32 accumulator), TMA-fed, accumulators in tensor memory.
  * Other values return KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
                         int shared, uint8_t *out_codes, uint8_t *out_scales,
                         int64_t M, int64_t d, cudaStream_t stream);
+
+/* Test export: kq_transform_f32 through a chosen kernel variant (as above). */
+int kq_transform_f32_variant(int variant, const void *act_bf16, const float *factors, int shared,
+                             float *out_y, int64_t M, int64_t d, cudaStream_t stream);
 
 /* Test exports: the baselines through a chosen kernel variant: 1 =
  * register-prefetch kernel, 2 = TMA-staged kernel, 0 = the default (SQ: 2,

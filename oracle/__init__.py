@@ -47,6 +47,14 @@ def lib():
         L.oracle_mx_quantize.restype = ci
         L.oracle_fold_weights.argtypes = [p, p, ci, p, p, i64, i64]
         L.oracle_fold_weights.restype = ci
+        L.oracle_lu_factor.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_double, p]
+        L.oracle_kron_expand_lu.argtypes = [p, p]
+        L.oracle_kq_transform_lu.argtypes = [p, p, ci, i64, i64, p, p]
+        L.oracle_kq_transform_lu.restype = ci
+        L.oracle_kq_quantize_lu.argtypes = [p, p, ci, i64, i64, p, p]
+        L.oracle_kq_quantize_lu.restype = ci
+        L.oracle_fwht_transform.argtypes = [p, i64, i64, i64, p, p, p, p]
+        L.oracle_fwht_transform.restype = ci
         _lib = L
     return _lib
 
@@ -162,3 +170,60 @@ def fold_weights(W, factors, shared=False, want_absbound=False):
     _check(lib().oracle_fold_weights(_ptr(W), _ptr(f), int(bool(shared)), _ptr(out), _ptr(ab), N, d),
            "fold_weights")
     return (out, ab) if want_absbound else out
+
+
+def lu_factor(a, b, c):
+    """G = L U of one factor (double) from its LU scalars."""
+    G = np.empty((2, 2), np.float64)
+    lib().oracle_lu_factor(float(a), float(b), float(c), _ptr(G))
+    return G
+
+
+def kron_expand_lu(params):
+    """Dense 32x32 K (float64) from [5, 3] float32 LU scalars (a, b, c) per factor."""
+    P = _c(params, np.float32).reshape(5, 3)
+    K = np.empty((32, 32), np.float64)
+    lib().oracle_kron_expand_lu(_ptr(P), _ptr(K))
+    return K
+
+
+def kq_transform_lu(x_bf16, params, shared=False, want_absbound=False):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    P = _c(params, np.float32)
+    y = np.empty((M, d), np.float32)
+    ab = np.empty((M, d), np.float64) if want_absbound else None
+    _check(lib().oracle_kq_transform_lu(_ptr(x), _ptr(P), int(bool(shared)), M, d, _ptr(y), _ptr(ab)),
+           "kq_transform_lu")
+    return (y, ab) if want_absbound else y
+
+
+def kq_quantize_lu(x_bf16, params, shared=False):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    P = _c(params, np.float32)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_kq_quantize_lu(_ptr(x), _ptr(P), int(bool(shared)), M, d, _ptr(codes), _ptr(scales)),
+           "kq_quantize_lu")
+    return codes, scales
+
+
+def fwht_transform(x_bf16, H, want_absbound=False):
+    """fp32 y = H_H x / sqrt(H) per H-block (double, rounded once), optionally with the error scale."""
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    y = np.empty((M, d), np.float32)
+    ab = np.empty((M, d), np.float64) if want_absbound else None
+    _check(lib().oracle_fwht_transform(_ptr(x), int(H), M, d, _ptr(y), _ptr(ab), None, None), "fwht_transform")
+    return (y, ab) if want_absbound else y
+
+
+def fwht_quantize(x_bf16, H):
+    x = _c(x_bf16, np.uint16)
+    M, d = _shape(x)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_fwht_transform(_ptr(x), int(H), M, d, None, None, _ptr(codes), _ptr(scales)),
+           "fwht_quantize")
+    return codes, scales

@@ -17,6 +17,13 @@
  *              section 3.2, Eq. (4), and "key machinery": T is block diagonal,
  *              each 32x32 block K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5 with 2x2 G_k;
  *              the inverse is folded into the weights offline.
+ *   [KQ-Eq6]   Pith review of arXiv 2607.21446, referee note on paper section
+ *              3.2, Eq. (6): each factor is G_k = L_k U_k with
+ *              U_k = [[a_k, b_k], [0, -1/a_k]], three scalars per factor, 15
+ *              per block; the Hadamard transform is the initialisation.
+ *   [KQ-FWHT]  KroQuant abstract and the Pith review's "forward implications":
+ *              fixed Hadamard transforms (applied by a fast Walsh-Hadamard
+ *              transform) are the comparison point of the on-the-fly kernel.
  *   [OCP-MX]   OCP Microscaling Formats (MX) Specification v1.0, section 6.3
  *              (the MXFP4 block-32 conversion): shared scale
  *              2^(floor(log2(amax)) - emax_elem) with emax_elem = 2 for E2M1,
@@ -38,6 +45,12 @@
  *   R5 Two codes per byte, the even element in the low nibble.
  *   R6 Factor storage: factors[j][k][r][c] (float32, 20 per block column j),
  *      k = 0..4 is G1..G5; "shared" mode uses one set for every column.
+ *   R7 LU storage: params[j][k][3] = (a, b, c) of G_(k+1), L unit lower
+ *      triangular.
+ *   R8 The fixed-Hadamard baseline of block size H (a power of two, 32 <= H,
+ *      H | d) is the orthonormal Sylvester transform H_H / sqrt(H) on every
+ *      H consecutive channels, followed by the same MX quantizer (blocks of
+ *      32 inside each H-block).
  */
 #include <math.h>
 #include <stdint.h>
@@ -79,7 +92,7 @@ static double bf16_value(uint16_t b)
 }
 
 /* [KQ-Eq4] + R1: K[i][l] = prod_k G_k[bit_(4-k)(i)][bit_(4-k)(l)], in double. */
-void oracle_kron_expand(const float *F /* [5][2][2] */, double *K /* [32][32] */)
+static void kron_expand_d(const double *F /* [5][2][2] */, double *K /* [32][32] */)
 {
     for (int i = 0; i < BLK; ++i) {
         for (int l = 0; l < BLK; ++l) {
@@ -87,11 +100,38 @@ void oracle_kron_expand(const float *F /* [5][2][2] */, double *K /* [32][32] */
             for (int k = 0; k < 5; ++k) {
                 int bi = (i >> (4 - k)) & 1;
                 int bl = (l >> (4 - k)) & 1;
-                p *= (double)F[k * 4 + bi * 2 + bl];
+                p *= F[k * 4 + bi * 2 + bl];
             }
             K[i * BLK + l] = p;
         }
     }
+}
+
+void oracle_kron_expand(const float *F /* [5][2][2] */, double *K /* [32][32] */)
+{
+    double Fd[20];
+    for (int e = 0; e < 20; ++e) Fd[e] = (double)F[e];
+    kron_expand_d(Fd, K);
+}
+
+/* [KQ-Eq6] LU form of one factor: G = L U with U = [[a, b], [0, -1/a]] and
+ * L = [[1, 0], [c, 1]] (reading: L is unit lower triangular), so
+ * G = [[a, b], [c a, c b - 1/a]] and det G = -1.  In double. */
+void oracle_lu_factor(double a, double b, double c, double *G /* [2][2] */)
+{
+    G[0] = a;
+    G[1] = b;
+    G[2] = c * a;
+    G[3] = c * b - 1.0 / a;
+}
+
+/* K from the 15 LU scalars of one block: params[k] = (a_k, b_k, c_k) of G_(k+1). */
+void oracle_kron_expand_lu(const float *params /* [5][3] */, double *K /* [32][32] */)
+{
+    double Fd[20];
+    for (int k = 0; k < 5; ++k)
+        oracle_lu_factor((double)params[3 * k], (double)params[3 * k + 1], (double)params[3 * k + 2], Fd + 4 * k);
+    kron_expand_d(Fd, K);
 }
 
 /* Dense inverse of a 32x32 matrix by Gauss-Jordan elimination with partial
@@ -192,14 +232,25 @@ void oracle_mx_block(const float *y /* [32] */, uint8_t *codes /* [16] */, uint8
         codes[b] = (uint8_t)(c[2 * b] | (c[2 * b + 1] << 4));
 }
 
-/* Expand every column's K^(j) once (nb x 1024 doubles). */
-static double *expand_all(const float *factors, int shared, int64_t nb)
+/* Expand every column's K^(j) once (nb x 1024 doubles), from generic factors
+ * (20 floats per column) or, with lu != 0, from LU scalars (15 per column). */
+static double *expand_all_mode(const float *params, int shared, int64_t nb, int lu)
 {
     int64_t ncol = shared ? 1 : nb;
     double *K = (double *)malloc((size_t)ncol * BLK * BLK * sizeof(double));
     if (!K) return NULL;
-    for (int64_t j = 0; j < ncol; ++j) oracle_kron_expand(factors + j * 20, K + j * BLK * BLK);
+    for (int64_t j = 0; j < ncol; ++j) {
+        if (lu)
+            oracle_kron_expand_lu(params + j * 15, K + j * BLK * BLK);
+        else
+            oracle_kron_expand(params + j * 20, K + j * BLK * BLK);
+    }
     return K;
+}
+
+static double *expand_all(const float *factors, int shared, int64_t nb)
+{
+    return expand_all_mode(factors, shared, nb, 0);
 }
 
 /* [KQ-abs], [KQ-Eq4]: y = T x per 32-block of every row, dense matvec with the
@@ -346,5 +397,103 @@ int oracle_fold_weights(const float *W, const float *factors, int shared,
         }
     }
     free(Ki);
+    return 0;
+}
+
+/* The dense per-block transform with already expanded K (double), shared by
+ * the generic-factor and LU entry points below. */
+static void transform_with(const double *K, int shared, const uint16_t *x, int64_t M, int64_t d, float *y,
+                           double *absb, uint8_t *codes, uint8_t *scales)
+{
+    int64_t nb = d / BLK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kj = K + (shared ? 0 : j) * BLK * BLK;
+            double xv[BLK];
+            float yv[BLK];
+            for (int l = 0; l < BLK; ++l) xv[l] = bf16_value(x[r * d + j * BLK + l]);
+            for (int i = 0; i < BLK; ++i) {
+                double sacc = 0.0, sa = 0.0;
+                for (int l = 0; l < BLK; ++l) {
+                    sacc += Kj[i * BLK + l] * xv[l];
+                    sa += fabs(Kj[i * BLK + l]) * fabs(xv[l]);
+                }
+                yv[i] = (float)sacc;
+                if (y) y[r * d + j * BLK + i] = yv[i];
+                if (absb) absb[r * d + j * BLK + i] = sa;
+            }
+            if (codes) oracle_mx_block(yv, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+        }
+    }
+}
+
+/* [KQ-Eq6] the KroQuant transform and quantizer from the 15 LU scalars per block. */
+int oracle_kq_transform_lu(const uint16_t *x, const float *params, int shared, int64_t M, int64_t d, float *y,
+                           double *absb)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    double *K = expand_all_mode(params, shared, d / BLK, 1);
+    if (!K) return -5;
+    transform_with(K, shared, x, M, d, y, absb, NULL, NULL);
+    free(K);
+    return 0;
+}
+
+int oracle_kq_quantize_lu(const uint16_t *x, const float *params, int shared, int64_t M, int64_t d,
+                          uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    double *K = expand_all_mode(params, shared, d / BLK, 1);
+    if (!K) return -5;
+    transform_with(K, shared, x, M, d, NULL, NULL, codes, scales);
+    free(K);
+    return 0;
+}
+
+static int popcount_u(unsigned v)
+{
+    int c = 0;
+    while (v) {
+        c += (int)(v & 1u);
+        v >>= 1;
+    }
+    return c;
+}
+
+/* [KQ-FWHT] + R8: y = H_H x / sqrt(H) on every H-block, H[i][f] = (-1)^popcount(i & f)
+ * (the Sylvester matrix), summed in double and rounded once to fp32; then the
+ * MX quantizer on each 32-block.  absb receives (|H_H| |x|)_i / sqrt(H). */
+int oracle_fwht_transform(const uint16_t *x, int64_t H, int64_t M, int64_t d, float *y, double *absb,
+                          uint8_t *codes, uint8_t *scales)
+{
+    if (H < BLK || (H & (H - 1)) != 0 || d % H != 0 || M < 0) return -2;
+    const double inv = 1.0 / sqrt((double)H);
+    int64_t nb = d / BLK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        double *xv = (double *)malloc((size_t)H * sizeof(double));
+        float *yv = (float *)malloc((size_t)H * sizeof(float));
+        for (int64_t h0 = 0; h0 < d; h0 += H) {
+            for (int64_t f = 0; f < H; ++f) xv[f] = bf16_value(x[r * d + h0 + f]);
+            for (int64_t i = 0; i < H; ++i) {
+                double sacc = 0.0, sa = 0.0;
+                for (int64_t f = 0; f < H; ++f) {
+                    double hv = (popcount_u((unsigned)(i & f)) & 1) ? -1.0 : 1.0;
+                    sacc += hv * xv[f];
+                    sa += fabs(xv[f]);
+                }
+                yv[i] = (float)(sacc * inv);
+                if (y) y[r * d + h0 + i] = yv[i];
+                if (absb) absb[r * d + h0 + i] = sa * inv;
+            }
+            if (codes)
+                for (int64_t b = 0; b < H / BLK; ++b)
+                    oracle_mx_block(yv + b * BLK, codes + r * (d / 2) + (h0 / 2) + b * (BLK / 2),
+                                    scales + r * nb + h0 / BLK + b);
+        }
+        free(xv);
+        free(yv);
+    }
     return 0;
 }

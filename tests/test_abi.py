@@ -122,6 +122,18 @@ def test_variant_errors_before_cuda(L):
     assert L.kq_wait_timeouts(None, 0) == -1
 
 
+def test_lu_and_fwht_argument_errors(L):
+    assert L.kq_quantize_lu(P(16), None, 0, P(16), P(16), 4, 64, None) == -1
+    assert L.kq_quantize_lu(P(16), P(16), 0, P(16), P(16), 4, 40, None) == -2
+    assert L.kq_quantize_lu(P(16), P(2), 0, P(16), P(16), 4, 64, None) == -3
+    assert L.fwht_quantize(P(16), 48, P(16), P(16), 4, 96, None) == -2
+    assert L.fwht_quantize(P(16), 64, P(16), P(16), 4, 96, None) == -2
+    assert L.fwht_quantize(P(16), 2048, P(16), P(16), 4, 2048, None) == -2
+    assert L.fwht_quantize(P(16), 32, None, P(16), 4, 64, None) == -1
+    assert L.kq_quantize_lu(None, None, 0, None, None, 0, 64, None) == 0
+    assert L.fwht_quantize(None, 32, None, None, 0, 64, None) == 0
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
 

@@ -295,3 +295,75 @@ def test_hand_worked_fixture_inputs_are_bf16_exact():
         if case["name"] in ("ties_and_saturation", "negative_ties"):
             continue  # these carry a deliberate non-exact +-0.1
         np.testing.assert_array_equal(f32(bf16(case["x"])), case["x"])
+
+
+# ---------------------------------------------------------------- LU form (Eq. 6) and FWHT baseline
+def lu_np(a, b, c):
+    return np.array([[1, 0], [c, 1]], np.float64) @ np.array([[a, b], [0, -1 / a]], np.float64)
+
+
+def rand_lu(n, rng):
+    P = np.empty((n, 5, 3), np.float32)
+    P[..., 0] = (0.6 + 0.8 * rng.random((n, 5))) * rng.choice([-1, 1], (n, 5))
+    P[..., 1] = 0.4 * rng.standard_normal((n, 5))
+    P[..., 2] = 0.4 * rng.standard_normal((n, 5))
+    return P
+
+
+def test_lu_expansion_matches_numpy_kron_of_lu_products():
+    rng = np.random.default_rng(21)
+    for P in rand_lu(10, rng):
+        ref = lu_np(*map(float, P[0]))
+        for k in range(1, 5):
+            ref = np.kron(ref, lu_np(*map(float, P[k])))
+        np.testing.assert_allclose(oracle.kron_expand_lu(P), ref, rtol=1e-13, atol=1e-15)
+        assert np.linalg.det(oracle.kron_expand_lu(P)) == pytest.approx(1.0, rel=1e-8)
+
+
+def test_lu_hadamard_initialisation():
+    a = np.float32(1 / np.sqrt(2.0))
+    P = np.tile(np.array([a, a, 1.0], np.float32), (5, 1))
+    K = oracle.kron_expand_lu(P)
+    np.testing.assert_allclose(K, scipy.linalg.hadamard(32) / np.sqrt(32.0), atol=3e-7)
+
+
+def test_lu_transform_agrees_with_factor_form():
+    rng = np.random.default_rng(22)
+    M, d = 9, 128
+    x = synth.activation("pixart", M, d, 22)
+    P = rand_lu(d // 32, rng)
+    F = np.array([[lu_np(*map(float, P[j, k])) for k in range(5)] for j in range(d // 32)]).astype(np.float32)
+    y_lu, ab = oracle.kq_transform_lu(x, P, want_absbound=True)
+    y_f = oracle.kq_transform(x, F)
+    # the factor form rounds G to fp32 first: a few fp32 ulps of |K||x|
+    np.testing.assert_array_less(np.abs(y_lu.astype(np.float64) - y_f), 1e-6 * ab + 1e-30)
+    c, s = oracle.kq_quantize_lu(x, P)
+    ci, si = independent_mx(y_lu.reshape(-1, 32))
+    np.testing.assert_array_equal(c.reshape(-1, 16), ci)
+    np.testing.assert_array_equal(s.reshape(-1), si)
+
+
+@pytest.mark.parametrize("H", [32, 64, 128, 256])
+def test_fwht_matches_scipy_hadamard(H):
+    M, d = 5, 512
+    x = synth.activation("pixart", M, d, H)
+    y, ab = oracle.fwht_transform(x, H, want_absbound=True)
+    xv = f32(x).astype(np.float64).reshape(M, d // H, H)
+    ref = (xv @ scipy.linalg.hadamard(H).T.astype(np.float64) / np.sqrt(H)).reshape(M, d)
+    np.testing.assert_array_less(np.abs(y - ref), np.abs(ref) * 2.0 ** -24 + 1e-12 * ab + 1e-30)
+    # orthonormal: energy is preserved block by block (Parseval)
+    np.testing.assert_allclose((ref ** 2).reshape(M, -1, H).sum(-1), (xv ** 2).sum(-1), rtol=1e-12)
+    np.testing.assert_allclose(ab, np.repeat(np.abs(xv).sum(-1), H, axis=1).reshape(M, d) / np.sqrt(H), rtol=1e-13)
+    c, s = oracle.fwht_quantize(x, H)
+    ci, si = independent_mx(y.reshape(-1, 32))
+    np.testing.assert_array_equal(c.reshape(-1, 16), ci)
+    np.testing.assert_array_equal(s.reshape(-1), si)
+
+
+def test_fwht_32_is_kroquant_with_hadamard_factors():
+    M, d = 7, 96
+    x = synth.activation("pixart", M, d, 23)
+    F = np.tile(np.array([[1, 1], [1, -1]], np.float32) / np.float32(np.sqrt(2.0)), (d // 32, 5, 1, 1))
+    y_h, ab = oracle.fwht_transform(x, 32, want_absbound=True)
+    y_k = oracle.kq_transform(x, F)
+    np.testing.assert_array_less(np.abs(y_h.astype(np.float64) - y_k), 1e-6 * ab + 1e-30)

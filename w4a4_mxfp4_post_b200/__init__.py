@@ -25,6 +25,7 @@ __all__ = [
     "KroQuantError", "lib", "kq_quantize", "kq_quantize_shared", "kq_quantize_variant", "sq_quantize",
     "mx_quantize", "kq_fold_weights", "kq_transform_f32", "kq_last_error", "kq_abi_version",
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
+    "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -43,6 +44,9 @@ _SIGS = {
     "mx_quantize": "pppqqp",
     "kq_fold_weights": "ppipqqp",
     "kq_transform_f32": "ppipqqp",
+    "kq_transform_f32_variant": "ippipqqp",
+    "kq_quantize_lu": "ppippqqp",
+    "fwht_quantize": "pqppqqp",
 }
 
 _lib = None
@@ -204,6 +208,28 @@ def mx_quantize(act, out_codes=None, out_scales=None, stream=None):
     return out_codes, out_scales
 
 
+def kq_quantize_lu(act, lu_params, shared=False, out_codes=None, out_scales=None, stream=None):
+    """KroQuant quantizer from 15 LU scalars per block ([d/32, 5, 3] or [5, 3] if shared)."""
+    torch = _torch()
+    M, d = _act(act)
+    _need(lu_params, "lu_params", torch.float32, act.device)
+    n = 1 if shared else d // 32
+    if lu_params.numel() != n * 15:
+        raise ValueError(f"lu_params must hold {n} x 5 x 3 floats, got {tuple(lu_params.shape)}")
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("kq_quantize_lu", _ptr(act), _ptr(lu_params), int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream))
+    return out_codes, out_scales
+
+
+def fwht_quantize(act, H, out_codes=None, out_scales=None, stream=None):
+    """Fixed-Hadamard (block size H) baseline quantizer."""
+    M, d = _act(act)
+    out_codes, out_scales = _outs(act, out_codes, out_scales)
+    _call("fwht_quantize", _ptr(act), int(H), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
 def sq_quantize_variant(variant, act, mult, out_codes=None, out_scales=None, stream=None):
     """The SmoothQuant quantizer through a chosen kernel variant (0 = the default)."""
     torch = _torch()
@@ -250,6 +276,19 @@ def kq_fold_weights(W, factors, shared=False, out=None, stream=None):
         out = torch.empty_like(W)
     _need(out, "out", torch.float32, W.device, (N, d))
     _call("kq_fold_weights", _ptr(W), _ptr(factors), int(bool(shared)), _ptr(out), N, d, _stream(stream))
+    return out
+
+
+def kq_transform_f32_variant(variant, act, factors, shared=False, out=None, stream=None):
+    """The fp32 transform through a chosen kernel variant (test export)."""
+    torch = _torch()
+    M, d = _act(act)
+    _factors(factors, d, shared, act.device)
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.float32, device=act.device)
+    _need(out, "out", torch.float32, act.device, (M, d))
+    _call("kq_transform_f32_variant", int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d,
+          _stream(stream))
     return out
 
 

@@ -14,7 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 INCLUDE = os.path.join(ROOT, "include")
 SOURCES = [os.path.join(HERE, "csrc", "kroquant.cu")]
-HEADERS = [os.path.join(INCLUDE, "kroquant.h")]
+HEADERS = [os.path.join(INCLUDE, "kroquant.h")] + sorted(
+    os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc")) if f.endswith((".cuh", ".h")))
 LIB = os.path.join(HERE, "libkroquant.so")
 
 NVCC_FLAGS = [

@@ -1,0 +1,450 @@
+// kq_mma.cuh -- KroQuant quantizer with the block transform on the tcgen05
+// tensor cores (variant 4).  Included by kroquant.cu; uses its helpers
+// (mbarriers, TMA, the MXFP4 epilogue pieces).
+//
+// Per 32-column block j, Y_j = X_j K_j^T is a [rows x 32] x [32 x 32] product
+// (K_j = G1 (x) ... (x) G5 expanded in fp32).  The product must keep fp32
+// accuracy (the quantizer's fp32 transform), so K_j is split into three bf16
+// parts K_hi + K_mid + K_lo (8 + 8 + 8 significand bits, the rest below fp32
+// rounding); X is bf16 already, so each of the three products is exact in the
+// fp32 accumulator and Y_j = X_j K_hi^T + X_j K_mid^T + X_j K_lo^T.
+//
+// A CTA owns one SM (1 CTA/SM, persistent) and walks a contiguous range of
+// tiles in group-major order: a tile is 128 rows x kNC block columns; the
+// tiles of one column group share the B operands, which are rebuilt only when
+// the group changes.
+//   warp 0     producer: builds the B operands of a column group (K_j split
+//              into 3 bf16 matrices, K-major, 64-byte swizzle) into one of
+//              two B buffers, and issues the TMA loads of the A tiles (two
+//              {64 cols x 128 rows} boxes, 128-byte swizzle) into a 4-stage ring
+//   warp 1     allocates the tensor memory; one thread issues the MMAs:
+//              kNC x 3 splits x 2 k-steps of M128 N32 K16 per tile into one of
+//              two 128-column fp32 accumulators
+//   warps 2-17 epilogue: tcgen05.ld of a row's 32 values of a block, amax,
+//              E8M0 byte, exact 2^-e scaling (packed FFMA with +0, so exact
+//              zeros come out +0 as in the other variants), E2M1.  Warp w reads
+//              TMEM lanes 32 (w % 4) .. +31 of block column (w - 2) / 4 and
+//              releases the accumulator at once; the codes of a tile are
+//              gathered in shared memory (double-buffered) and written by one
+//              TMA tensor store, the scales by one 4-byte store per row.
+// Every mbarrier wait is bounded (g_wait_timeouts); the tensor memory is
+// freed on every path.
+
+namespace mma {
+
+constexpr int kNC = 4;                                   // block columns per tile
+constexpr int kRows = 128;                               // tile rows (MMA M)
+constexpr int kAStages = 4;
+constexpr int kABoxBytes = kRows * 128;                  // {64 cols x 128 rows} bf16 = 16 KB
+constexpr int kAStageBytes = 2 * kABoxBytes;             // kNC = 4 block columns: 32 KB
+constexpr int kBMatBytes = 32 * 64;                      // one 32 x 32 bf16 matrix: 2 KB
+constexpr int kBSetBytes = kNC * 3 * kBMatBytes;         // 24 KB
+constexpr int kTmemCols = 2 * kNC * 32;                  // two accumulators of kNC x 32 columns
+constexpr int kEpiWarps = 16;                            // 4 lane quarters x kNC block columns
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;               // 576
+constexpr int kCodesTileBytes = kRows * kNC * 16;        // 8 KB of codes per tile
+constexpr int kScalesTileBytes = kRows * kNC;            // 512 B of scales per tile
+constexpr size_t kSmemA = size_t(kAStages) * kAStageBytes;
+constexpr size_t kSmemB = 2 * size_t(kBSetBytes);
+constexpr size_t kSmemOut = 2 * size_t(kCodesTileBytes + kScalesTileBytes);
+constexpr size_t kSmemBars = 16 * sizeof(uint64_t) + 16;
+constexpr size_t kSmem = kSmemA + kSmemB + kSmemOut + kSmemBars + 1024;
+
+// Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
+// = 1), B bf16 (bits 10-12 = 1), A and B K-major (bits 15, 16 = 0),
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(32 >> 3) << 17) |
+                            (uint32_t(kRows >> 4) << 24);
+
+// Shared-memory matrix descriptor: start address >> 4 (bits 0-13), leading
+// byte offset >> 4 (bits 16-29; unused by swizzled K-major layouts, 1),
+// stride byte offset >> 4 (bits 32-45: the distance between 8-row groups),
+// version 1 (bits 46-47), base offset 0, layout type in bits 61-63
+// (2 = 128-byte swizzle, 4 = 64-byte swizzle).
+constexpr uint64_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t sbo_bytes, uint64_t layout)
+{
+    return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+           (uint64_t(1) << 46) | (layout << 61);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+                 "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+                 : "memory");
+}
+
+// Arrive (once) on `bar` when every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int32_t x, int32_t y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);   // .x = lo (low half), .y = hi
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Build the B operands of column group g into `dst` (warp-collective; lane n
+// writes row n of every matrix): for block column jj (j = g*kNC + jj) and
+// split s, matrix (jj, s) holds part s of K_j as 32 rows n x 32 columns l
+// (K-major, B[n][l] = K_j[n][l], since Y = X K^T), in the 64-byte swizzle
+// layout: row n at n*64, its 16-byte chunk c at chunk c ^ ((n >> 1) & 3).
+__device__ void build_b_operands(uint8_t *dst, const float4 *__restrict__ factors, int shared, int g, int nb,
+                                 int lane)
+{
+    const int n = lane;
+    const int sw = (n >> 1) & 3;
+#pragma unroll 1
+    for (int jj = 0; jj < kNC; ++jj) {
+        const int j = g * kNC + jj;
+        float r[5][2];
+        if (j < nb) {
+            const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+#pragma unroll
+            for (int k = 0; k < 5; ++k) {
+                const float4 f = __ldg(fp + k);            // [g00, g01, g10, g11] of G_(k+1)
+                const int bn = (n >> (4 - k)) & 1;          // G_(k+1) acts on index bit 4-k
+                r[k][0] = bn ? f.z : f.x;
+                r[k][1] = bn ? f.w : f.y;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 5; ++k) r[k][0] = r[k][1] = 0.0f;
+        }
+        // one 16-byte chunk (8 columns l) of the row at a time
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float part[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int l = 8 * c + e;
+                const float a0 = ((l >> 4) & 1) ? r[0][1] : r[0][0];
+                const float a1 = ((l >> 3) & 1) ? r[1][1] : r[1][0];
+                const float a2 = ((l >> 2) & 1) ? r[2][1] : r[2][0];
+                const float a3 = ((l >> 1) & 1) ? r[3][1] : r[3][0];
+                const float a4 = (l & 1) ? r[4][1] : r[4][0];
+                part[e] = a0 * a1 * a2 * a3 * a4;
+            }
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp) {
+                // part sp of the split: round to bf16, carry the exact remainder on
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const __nv_bfloat16 ha = __float2bfloat16_rn(part[e]), hb = __float2bfloat16_rn(part[e + 1]);
+                    part[e] -= __bfloat162float(ha);
+                    part[e + 1] -= __bfloat162float(hb);
+                    w[e / 2] = uint32_t(__bfloat16_as_ushort(ha)) | (uint32_t(__bfloat16_as_ushort(hb)) << 16);
+                }
+                *reinterpret_cast<uint4 *>(dst + (jj * 3 + sp) * kBMatBytes + n * 64 + 16 * (c ^ sw)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int32_t x, int32_t y, const void *src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_addr(src))
+                 : "memory");
+}
+
+// Named barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
+// AND of `pred` over all epilogue threads (barrier id 2): makes a give-up
+// decision uniform across the epilogue warps, which share named barriers.
+__device__ __forceinline__ bool epi_all(bool pred)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.b32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, 2, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(uint32_t(pred)), "n"(kEpiThreads)
+                 : "memory");
+    return r != 0;
+}
+
+template <KqOut OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant__ CUtensorMap codes_map,
+              const float4 *__restrict__ factors, int shared, uint8_t *__restrict__ scales,
+              float4 *__restrict__ y_out, int64_t M, int nb, long long budget)
+{
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;
+    uint8_t *sB = base + kSmemA;
+    uint8_t *sOut = sB + kSmemB;                               // [2] x (codes tile, scales tile)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sOut + kSmemOut);
+    uint64_t *full_a = bars;          // [kAStages] A tile landed (TMA tx)
+    uint64_t *empty_a = bars + 4;     // [kAStages] MMAs reading the stage done (commit)
+    uint64_t *tfull = bars + 8;       // [2] accumulator ready (commit)
+    uint64_t *tempty = bars + 10;     // [2] accumulator read by the epilogue warps
+    uint64_t *bfull = bars + 12;      // [2] B set built
+    uint64_t *bempty = bars + 14;     // [2] MMAs reading the B set done (commit)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int64_t RT = (M + kRows - 1) / kRows;
+    const int ngroups = (nb + kNC - 1) / kNC;
+    const int64_t T = RT * ngroups;
+    const int64_t t_begin = int64_t(blockIdx.x) * T / gridDim.x;
+    const int64_t t_end = int64_t(blockIdx.x + 1) * T / gridDim.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kAStages; ++s) {
+            mbar_init(&full_a[s], 1);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&bfull[b], 1);
+            mbar_init(&bempty[b], 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- producer: B sets and A tiles
+        int last_g = -1, buse = -1, k = 0, filled = 0;
+        bool ok = true;
+        for (int64_t t = t_begin; t < t_end && ok; ++t, ++k) {
+            const int g = int(t / RT);
+            const int64_t rt = t % RT;
+            if (g != last_g) {
+                ++buse;
+                const int bb = buse & 1;
+                // every lane waits (each acquires the release of the old B set);
+                // the give-up decision is made warp-uniform
+                const bool freed = buse < 2 || mbar_wait(&bempty[bb], ((buse >> 1) - 1) & 1, budget);
+                if (!__all_sync(0xffffffffu, freed)) {
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
+                    ok = false;
+                    break;
+                }
+                build_b_operands(sB + bb * kBSetBytes, factors, shared, g, nb, lane);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bfull[bb]);
+                last_g = g;
+            }
+            if (lane == 0) {
+                const int s = k % kAStages;
+                if (k >= kAStages && !mbar_wait(&empty_a[s], ((k / kAStages) - 1) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    ok = false;
+                } else {
+                    mbar_expect_tx(&full_a[s], kAStageBytes);
+                    uint8_t *st = sA + size_t(s) * kAStageBytes;
+                    tma_load_2d(st, &act_map, g * kNC * 32, int32_t(rt * kRows), &full_a[s]);
+                    tma_load_2d(st + kABoxBytes, &act_map, g * kNC * 32 + 64, int32_t(rt * kRows), &full_a[s]);
+                    filled = k + 1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        if (lane == 0) {   // drain: the copies issued have landed before the CTA may exit
+            for (int kk = (filled > kAStages ? filled - kAStages : 0); kk < filled; ++kk)
+                if (!mbar_wait(&full_a[kk % kAStages], (kk / kAStages) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    break;
+                }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            int last_g = -1, bcount = -1, k = 0, issued = 0;
+            for (int64_t t = t_begin; t < t_end; ++t, ++k) {
+                const int g = int(t / RT);
+                if (g != last_g) {
+                    if (bcount >= 0) umma_commit(&bempty[bcount & 1]);
+                    ++bcount;
+                    if (!mbar_wait(&bfull[bcount & 1], (bcount >> 1) & 1, budget)) {
+                        atomicAdd(&g_wait_timeouts, 1);
+                        break;
+                    }
+                    last_g = g;
+                }
+                const int s = k % kAStages;
+                if (!mbar_wait(&full_a[s], (k / kAStages) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    break;
+                }
+                const int tb = k & 1;
+                if (k >= 2 && !mbar_wait(&tempty[tb], ((k >> 1) - 1) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_addr(sA + size_t(s) * kAStageBytes);
+                const uint32_t b0 = smem_addr(sB + (bcount & 1) * kBSetBytes);
+#pragma unroll
+                for (int jj = 0; jj < kNC; ++jj) {
+                    const uint32_t d = tmem_base + uint32_t(tb * kNC * 32 + jj * 32);
+#pragma unroll
+                    for (int sp = 0; sp < 3; ++sp) {
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            const uint64_t ad =
+                                smem_desc(a0 + (jj >> 1) * kABoxBytes + (jj & 1) * 64 + kk * 32, 1024, kLayoutSw128);
+                            const uint64_t bd = smem_desc(b0 + (jj * 3 + sp) * kBMatBytes + kk * 32, 512, kLayoutSw64);
+                            umma_bf16(d, ad, bd, (sp | kk) != 0);
+                        }
+                    }
+                }
+                umma_commit(&empty_a[s]);
+                umma_commit(&tfull[tb]);
+                issued = k + 1;
+            }
+            // every MMA issued has completed before the tensor memory is freed
+            if (issued > 0 && !mbar_wait(&tfull[(issued - 1) & 1], ((issued - 1) >> 1) & 1, budget))
+                atomicAdd(&g_wait_timeouts, 1);
+        }
+    } else {
+        // ---------------- epilogue warps: warp w reads TMEM lane quarter w % 4
+        // (tile rows 32q .. 32q+31) of block column (w - 2) / 4
+        const int q = warp & 3;
+        const int jj = (warp - 2) >> 2;
+        const int et = threadIdx.x - 64;                  // 0 .. kEpiThreads-1
+        const bool store_leader = (et == 0);
+        int k = 0;
+        for (int64_t t = t_begin; t < t_end; ++t, ++k) {
+            const int g = int(t / RT);
+            const int64_t rt = t % RT;
+            const int tb = k & 1;
+            const bool ready = mbar_wait(&tfull[tb], (k >> 1) & 1, budget);
+            // uniform over the epilogue: tcgen05.ld is warp-collective and the
+            // epilogue warps meet at named barriers below
+            if (!epi_all(ready)) {
+                if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
+                break;
+            }
+            tc_fence_after();
+            const int rloc = q * 32 + lane;                 // row within the tile
+            const int64_t row = rt * kRows + rloc;
+            const int j = g * kNC + jj;
+            float v[32];
+            tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(tb * kNC * 32 + jj * 32), v);
+            // the accumulator has been read: hand it back to the MMA thread
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tb]);
+
+            if constexpr (OUT == KqOut::kF32) {
+                if (row < M && j < nb) {
+                    // the fp32 transform itself (+0: exact zeros come out +0)
+                    float4 *yo = y_out + (row * nb + j) * 8;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        yo[i] = make_float4(v[4 * i] + 0.0f, v[4 * i + 1] + 0.0f, v[4 * i + 2] + 0.0f,
+                                            v[4 * i + 3] + 0.0f);
+                }
+            } else {
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) amax = max3_abs(amax, v[2 * i], v[2 * i + 1]);
+                const uint32_t sb = e8m0_byte(amax);
+                const float sc = inv_scale(sb);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 pr = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), make_float2(sc, sc), plus_zero2());
+                    v[2 * i] = pr.x;
+                    v[2 * i + 1] = pr.y;
+                }
+                uint4 cw;
+                cw.x = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+                cw.y = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+                cw.z = cvt_e2m1x8(v[16], v[17], v[18], v[19], v[20], v[21], v[22], v[23]);
+                cw.w = cvt_e2m1x8(v[24], v[25], v[26], v[27], v[28], v[29], v[30], v[31]);
+                // staging buffer k & 1: the tile store that read it two tiles ago must be done
+                uint8_t *ocodes = sOut + (k & 1) * (kCodesTileBytes + kScalesTileBytes);
+                uint8_t *oscales = ocodes + kCodesTileBytes;
+                if (store_leader) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                epi_sync();
+                // codes tile = rows x 64 bytes (the box of the codes tensor map, no swizzle)
+                *reinterpret_cast<uint4 *>(ocodes + rloc * (kNC * 16) + jj * 16) = cw;
+                oscales[rloc * kNC + jj] = uint8_t(sb);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                epi_sync();
+                if (store_leader) {
+                    // rows beyond M and columns beyond d/2 are clipped by the tensor map
+                    tma_store_2d(&codes_map, g * kNC * 16, int32_t(rt * kRows), ocodes);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+                if (jj == 0 && row < M) {
+                    // this row's kNC scale bytes, one 4-byte store where the row layout allows it
+                    const int nj = nb - g * kNC < kNC ? nb - g * kNC : kNC;
+                    uint8_t *dst = scales + row * nb + int64_t(g) * kNC;
+                    const uint32_t w4 = *reinterpret_cast<const uint32_t *>(oscales + rloc * kNC);
+                    if (nj == kNC && (reinterpret_cast<uintptr_t>(dst) & 3) == 0) {
+                        *reinterpret_cast<uint32_t *>(dst) = w4;
+                    } else {
+                        for (int e = 0; e < nj; ++e) dst[e] = uint8_t(w4 >> (8 * e));
+                    }
+                }
+            }
+        }
+        if constexpr (OUT == KqOut::kCodes) {
+            if (store_leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace mma

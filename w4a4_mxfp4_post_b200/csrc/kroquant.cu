@@ -24,6 +24,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 
 #include "kroquant.h"
@@ -446,6 +447,20 @@ __device__ __forceinline__ void load_factors(const float4 *__restrict__ factors,
     for (int k = 0; k < 5; ++k) g[k] = __ldg(fp + k);
 }
 
+// The factors from the LU form of KroQuant section 3.2, Eq. (6): G = L U with
+// U = [[a, b], [0, -1/a]] and L = [[1, 0], [c, 1]], i.e.
+// G = [[a, b], [c a, c b - 1/a]]: 15 scalars per block (a, b, c per factor)
+// expanded once per thread (the paper's on-the-fly "K2" reconstruction).
+__device__ __forceinline__ void load_lu(const float *__restrict__ lu, int shared, int j, float4 (&g)[5])
+{
+    const float *pp = lu + (shared ? 0 : int64_t(j) * 15);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const float a = __ldg(pp + 3 * k), b = __ldg(pp + 3 * k + 1), c = __ldg(pp + 3 * k + 2);
+        g[k] = make_float4(a, b, c * a, fmaf(c, b, -(1.0f / a)));
+    }
+}
+
 // KroQuant quantizer, packed butterfly (variant 2).
 //
 // Each 2x2 factor is split as G = [[g00, g01], [g10, g11]]
@@ -459,16 +474,19 @@ __device__ __forceinline__ void load_factors(const float4 *__restrict__ factors,
 // A thread whose column has a factor with |g00| or |g11| outside
 // [2^-16, 2^16] or |b| or |c| above 16 (where U's intermediate values could
 // grow by more than 17^5) runs the direct form instead.
-template <KqOut OUT>
+template <KqOut OUT, bool LU = false>
 __global__ void __launch_bounds__(kThreads, 2)
-kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params, int shared,
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
                  int64_t nblocks, int nb, int64_t T)
 {
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
     float4 g[5];
-    load_factors(factors, shared, int(t % nb), g);
+    if constexpr (LU)
+        load_lu(params, shared, int(t % nb), g);
+    else
+        load_factors(reinterpret_cast<const float4 *>(params), shared, int(t % nb), g);
     KqFast st;
     const bool fast = kq_fast_setup(g, st);
 
@@ -502,6 +520,72 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ facto
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
             gi = gn;
+        }
+    }
+}
+
+// Fixed-Hadamard baseline (the transform the pages compare the on-the-fly
+// kernel against): y = H_H x / sqrt(H) on every H consecutive channels, H =
+// 2^(5 + xstages) in [32, 1024], H | d, with H_H the Sylvester matrix
+// (H2 (x) ... (x) H2), then the MXFP4 quantizer on each 32-block.  A thread
+// holds one 32-block: the five stages on its in-block index bits are
+// in-register (lo + hi, lo - hi); an H-block spans H/32 consecutive lanes of a
+// warp, and each further stage exchanges all 32 values with the partner lane
+// lane ^ 2^s by shuffles.  Warps walk the flattened block array together (the
+// grid stride is a multiple of 32, so the lanes of an H-block stay aligned).
+template <int S>
+__device__ __forceinline__ void hadamard_stage2(float2 (&p)[16])
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        if (i & S) continue;
+        const float2 lo = p[i], hi = p[i + S];
+        p[i] = __fadd2_rn(lo, hi);
+        p[i + S] = __ffma2_rn(hi, make_float2(-1.0f, -1.0f), lo);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+fwht_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks,
+            int64_t T, int xstages, float inv_sqrt_h)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t t0 = int64_t(blockIdx.x) * kThreads + (threadIdx.x & ~31);   // the warp's first thread
+    for (int64_t g0 = t0; g0 < nblocks; g0 += T) {                            // warp-uniform walk
+        const int64_t gi = g0 + lane;
+        const bool valid = gi < nblocks;       // whole H-blocks are valid or not (H | d)
+        uint4 raw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                        make_uint4(0, 0, 0, 0)};
+        if (valid) load_block_nc(act, gi, raw);
+        float2 p[16];
+        unpack_pairs(raw, p);
+        hadamard_stage2<1>(p);
+        hadamard_stage2<2>(p);
+        hadamard_stage2<4>(p);
+        hadamard_stage2<8>(p);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = make_float2(p[i].x + p[i].y, p[i].x - p[i].y);
+#pragma unroll
+        for (int s = 0; s < 5; ++s) {
+            if (s >= xstages) break;
+            const int m = 1 << s;
+            const float sg = (lane & m) ? -1.0f : 1.0f;   // partner holds the other half of the pair
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float ox = __shfl_xor_sync(0xffffffffu, p[i].x, m);
+                const float oy = __shfl_xor_sync(0xffffffffu, p[i].y, m);
+                p[i] = make_float2(fmaf(sg, p[i].x, ox), fmaf(sg, p[i].y, oy));
+            }
+        }
+        const float2 nrm = make_float2(inv_sqrt_h, inv_sqrt_h);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) p[i] = __fmul2_rn(p[i], nrm);
+        if (valid) {
+            uint4 c;
+            uint32_t sb;
+            mx_quantize_pairs(p, c, sb);
+            codes[gi] = c;
+            scales[gi] = uint8_t(sb);
         }
     }
 }
@@ -836,6 +920,8 @@ mx_staged_kernel(const __grid_constant__ CUtensorMap act_map, uint4 *__restrict_
     });
 }
 
+#include "kq_mma.cuh"
+
 // ---------------------------------------------------------------------------
 // launch geometry
 // ---------------------------------------------------------------------------
@@ -887,7 +973,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 // per SM (occupancy query, cached per device and kernel).
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
-    kKqStaged, kSqStaged, kMxStaged, kNumKernels
+    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1028,6 +1114,55 @@ unsigned staged_grid(int64_t nblocks, int64_t nb, int64_t resident)
     return unsigned(grid);
 }
 
+// The activation as the [M][d] bf16 matrix, boxes of {64 columns x 128 rows}
+// with the 128-byte swizzle (the A operand layout of the tcgen05 variant).
+int encode_act_map_rows(const void *act, int64_t M, int64_t d, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+    const cuuint32_t box[2] = {64, cuuint32_t(mma::kRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(act), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
+// The codes as the [M][d/2] uint8 matrix, boxes of {kNC*16 bytes x 128 rows}
+// (one tile of the tcgen05 variant), no swizzle.
+int encode_codes_map(void *codes, int64_t M, int64_t d, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const cuuint64_t dims[2] = {cuuint64_t(d / 2), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(d / 2)};
+    const cuuint32_t box[2] = {cuuint32_t(mma::kNC * 16), cuuint32_t(mma::kRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
+int mma_prepare(KernelId id, const void *fn)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices || !g_smem_set[id][dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(mma::kSmem));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_smem_set[id][dev].store(1, std::memory_order_release);
+    }
+    return KQ_OK;
+}
+
 // Default clock budget of a bounded wait: 2^31 cycles, about a second.
 constexpr long long kWaitBudget = 1LL << 31;
 
@@ -1047,7 +1182,8 @@ int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t
 
 // Kernel variants of the KroQuant quantizer: 1 = one block per thread, direct
 // 2x2 stages; 2 = packed pairs with the unit-diagonal split, register
-// prefetch; 3 = the arithmetic of 2 on TMA-staged input.  0 = the default,
+// prefetch; 3 = the arithmetic of 2 on TMA-staged input; 4 = the transform
+// as tcgen05 MMAs on K split into three bf16 parts.  0 = the default,
 // the fastest on the benchmark shapes (2: the staged input does not help a
 // kernel whose limit is its instruction stream; see the profiles).
 constexpr int kDefaultVariant = 2;
@@ -1060,8 +1196,34 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
     if (variant == 0) variant = kDefaultVariant;
-    if (variant < 1 || variant > 3)
+    if (variant < 1 || variant > 4)
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    if (variant == 4 && M < (int64_t(1) << 31)) {
+        const int64_t nb4 = d / kBlk;
+        CUtensorMap map;
+        if ((rc = encode_act_map_rows(act, M, d, &map)) != KQ_OK) return rc;
+        const int64_t tiles = ((M + mma::kRows - 1) / mma::kRows) * ((nb4 + mma::kNC - 1) / mma::kNC);
+        int sms = 0;
+        if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+        const unsigned grid = unsigned(tiles < sms ? tiles : sms);
+        const float4 *f4 = reinterpret_cast<const float4 *>(factors);
+        if (f32) {
+            auto k = mma::kq_mma_kernel<KqOut::kF32>;
+            if ((rc = mma_prepare(kKqMmaF32, reinterpret_cast<const void *>(k))) != KQ_OK) return rc;
+            // the codes map is unused by the fp32 export; any valid map will do
+            k<<<grid, mma::kThreads, mma::kSmem, stream>>>(map, map, f4, shared, nullptr,
+                                                           reinterpret_cast<float4 *>(y), M, int(nb4), kWaitBudget);
+        } else {
+            CUtensorMap cmap;
+            if ((rc = encode_codes_map(codes, M, d, &cmap)) != KQ_OK) return rc;
+            auto k = mma::kq_mma_kernel<KqOut::kCodes>;
+            if ((rc = mma_prepare(kKqMma, reinterpret_cast<const void *>(k))) != KQ_OK) return rc;
+            k<<<grid, mma::kThreads, mma::kSmem, stream>>>(map, cmap, f4, shared, scales, nullptr, M, int(nb4),
+                                                           kWaitBudget);
+        }
+        return launch_check(fn);
+    }
+    if (variant == 4) variant = 2;   // row coordinates beyond int32: the butterfly
     // the fp32 export and very large inputs use the variant-2 kernel (same arithmetic as 3)
     if (variant == 3 && (f32 || M * (d / kBlk) > kStagedMaxBlocks)) variant = 2;
     const int64_t nb = d / kBlk;
@@ -1093,12 +1255,12 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
         if (f32) {
             auto k = kq_packed_kernel<KqOut::kF32>;
             if ((rc = launch_pinned(fn, kKqPackedF32, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
+            k<<<geo.grid, kThreads, 0, stream>>>(a, factors, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
                                                  nblocks, int(nb), geo.T);
         } else {
             auto k = kq_packed_kernel<KqOut::kCodes>;
             if ((rc = launch_pinned(fn, kKqPacked, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
+            k<<<geo.grid, kThreads, 0, stream>>>(a, factors, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
                                                  nblocks, int(nb), geo.T);
         }
     }
@@ -1134,6 +1296,13 @@ int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
 {
     return kq_launch("kq_quantize_variant", variant, act_bf16, factors, shared ? 1 : 0, out_codes, out_scales,
                      nullptr, false, M, d, stream);
+}
+
+int kq_transform_f32_variant(int variant, const void *act_bf16, const float *factors, int shared, float *out_y,
+                             int64_t M, int64_t d, cudaStream_t stream)
+{
+    return kq_launch("kq_transform_f32_variant", variant, act_bf16, factors, shared ? 1 : 0, nullptr, nullptr, out_y,
+                     true, M, d, stream);
 }
 
 int kq_transform_f32(const void *act_bf16, const float *factors, int shared, float *out_y, int64_t M, int64_t d,
@@ -1215,6 +1384,64 @@ int mx_quantize_variant(int variant, const void *act_bf16, uint8_t *out_codes, u
     mx_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
                                                         reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
                                                         geo.T);
+    return launch_check(fn);
+}
+
+int kq_quantize_lu(const void *act_bf16, const float *lu_params, int shared, uint8_t *out_codes,
+                   uint8_t *out_scales, int64_t M, int64_t d, cudaStream_t stream)
+{
+    const char *fn = "kq_quantize_lu";
+    if (M < 0 || d <= 0 || d % kBlk != 0)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32 (M=%lld, d=%lld)", fn,
+                    (long long)M, (long long)d);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d))
+        return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (M == 0) return ok();
+    if (!act_bf16 || !lu_params || !out_codes || !out_scales) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(act_bf16, 16) || !aligned(out_codes, 16) || !aligned(lu_params, 4))
+        return fail(KQ_ERR_ALIGN, "%s: act and out_codes must be 16-byte aligned, lu_params 4-byte", fn);
+    const int64_t nb = d / kBlk;
+    Geometry geo;
+    auto k = kq_packed_kernel<KqOut::kCodes, true>;
+    int rc = launch_pinned(fn, kKqLu, k, M, nb, &geo);
+    if (rc != KQ_OK) return rc;
+    k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16), lu_params, shared ? 1 : 0,
+                                         reinterpret_cast<uint4 *>(out_codes), out_scales, nullptr, M * nb, int(nb),
+                                         geo.T);
+    return launch_check(fn);
+}
+
+int fwht_quantize(const void *act_bf16, int64_t H, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
+                  cudaStream_t stream)
+{
+    const char *fn = "fwht_quantize";
+    int xstages = -1;
+    for (int s = 0; s <= 5; ++s)
+        if (H == (int64_t(32) << s)) xstages = s;
+    if (xstages < 0) return fail(KQ_ERR_SHAPE, "%s: H must be a power of two in [32, 1024] (H=%lld)", fn, (long long)H);
+    if (M < 0 || d <= 0 || d % H != 0)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of H (M=%lld, d=%lld, H=%lld)", fn,
+                    (long long)M, (long long)d, (long long)H);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d))
+        return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (M == 0) return ok();
+    if (!act_bf16 || !out_codes || !out_scales) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(act_bf16, 16) || !aligned(out_codes, 16))
+        return fail(KQ_ERR_ALIGN, "%s: act and out_codes must be 16-byte aligned", fn);
+    const int64_t nblocks = M * (d / kBlk);
+    int64_t target = 0;
+    int rc = resident_threads(kFwht, reinterpret_cast<const void *>(fwht_kernel), &target);
+    if (rc != KQ_OK) return rc;
+    int64_t T = (target / 32) * 32;
+    const int64_t need = ((nblocks + 31) / 32) * 32;
+    if (T > need) T = need;
+    if (T < 32) T = 32;
+    const unsigned grid = unsigned((T + kThreads - 1) / kThreads);
+    // 1/sqrt(H) rounded to fp32: H = 2^(5 + s); sqrt(2^n) = 2^(n/2) * (sqrt 2 if n odd)
+    const double inv = 1.0 / std::sqrt(double(H));
+    fwht_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+                                               reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
+                                               int64_t(grid) * kThreads, xstages, float(inv));
     return launch_check(fn);
 }
 

@@ -153,6 +153,22 @@ def factors(nb: int, seed: int, shared: bool = False) -> np.ndarray:
     return out
 
 
+def lu_params(nb: int, seed: int, shared: bool = False, noise: float = 0.1) -> np.ndarray:
+    """LU scalars [n, 5, 3] float32 = (a, b, c) per factor (n = 1 if shared else nb).
+
+    A learned transform starts at the Hadamard initialisation (a = b = 1/sqrt 2,
+    c = 1) and moves from there: each scalar gets noise * N(0,1) added; |a|
+    is kept >= 0.2.
+    """
+    g = _rng(seed + 2000, 4)
+    n = 1 if shared else nb
+    base = np.array([1 / np.sqrt(2.0), 1 / np.sqrt(2.0), 1.0])
+    out = (base[None, None, :] + noise * g.standard_normal((n, 5, 3))).astype(np.float32)
+    a = out[..., 0]
+    out[..., 0] = np.where(np.abs(a) < 0.2, np.copysign(np.float32(0.2), a), a)
+    return out
+
+
 def sq_multipliers(x_bf16: np.ndarray, alpha: float = 0.5, floor: float = 1e-5) -> np.ndarray:
     """SmoothQuant per-channel multipliers m_c = 1/s_c, s_c = max(max_r |X_rc|, floor)^alpha.
 
