@@ -658,6 +658,76 @@ def sweep_mode(args):
             json.dump({"peak": peak, "peak_source": src, "rows": rows}, fh, indent=1)
 
 
+def sqnr_mode(args):
+    """Quantisation-error proxy: SQNR of the round trip x -> codes/scales -> x^ per method.
+
+    A dataset-free stand-in for the pages' quality comparison (learned
+    block transform vs per-channel scaling vs plain MXFP4 vs fixed Hadamard):
+    seeded activations with per-channel outliers, the inverse of each method's
+    transform applied after decoding.  SQNR = 10 log10(sum x^2 / sum (x - x^)^2).
+    """
+    import torch
+
+    import w4a4_mxfp4_post_b200 as kq
+    from w4a4_mxfp4_post_b200 import build, synth
+
+    build.build()
+    torch.backends.cuda.matmul.allow_tf32 = False
+    dev = torch.device("cuda:0")
+    rows = []
+
+    def sqnr(x, xh):
+        return float(10 * torch.log10((x.double() ** 2).sum() / ((x.double() - xh.double()) ** 2).sum()))
+
+    def lu_to_factors(P):
+        a, b, c = P[..., 0].astype(np.float64), P[..., 1].astype(np.float64), P[..., 2].astype(np.float64)
+        F = np.stack([np.stack([a, b], -1), np.stack([c * a, c * b - 1 / a], -1)], -2)
+        return F.astype(np.float32)
+
+    for name in ("pixart", "sana", "flux"):
+        for (M, d, model, shared, seed) in synth.workload_layers(name):
+            xb = synth.activation(model, M, d, seed)
+            x = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+            xf = x.float()
+            nb = d // 32
+            row = {"workload": name, "M": M, "d": d}
+            c, s = kq.mx_quantize(x)
+            row["mx"] = sqnr(xf, kq.mx_dequantize(c, s))
+            m = torch.from_numpy(synth.sq_multipliers(xb)).to(dev)
+            c, s = kq.sq_quantize(x, m)
+            row["sq"] = sqnr(xf, kq.mx_dequantize(c, s) / m)
+            F = synth.factors(nb, seed)
+            Fd = torch.from_numpy(F).to(dev)
+            c, s = kq.kq_quantize(x, Fd)
+            row["kq_random_factors"] = sqnr(xf, kq.kq_inverse_f32(kq.mx_dequantize(c, s), Fd))
+            H2 = np.tile(np.array([[1, 1], [1, -1]], np.float32) / np.float32(np.sqrt(2.0)), (nb, 5, 1, 1))
+            Hd = torch.from_numpy(H2).to(dev)
+            c, s = kq.kq_quantize(x, Hd)
+            row["kq_hadamard_init"] = sqnr(xf, kq.kq_inverse_f32(kq.mx_dequantize(c, s), Hd))
+            P = synth.lu_params(nb, seed)
+            c, s = kq.kq_quantize_lu(x, torch.from_numpy(P).to(dev))
+            Fl = torch.from_numpy(lu_to_factors(P)).to(dev)
+            row["kq_lu_near_hadamard"] = sqnr(xf, kq.kq_inverse_f32(kq.mx_dequantize(c, s), Fl))
+            for H in (128, 1024):
+                if d % H:
+                    continue
+                c, s = kq.fwht_quantize(x, H)
+                Hm = torch.from_numpy(scipy_hadamard(H) / np.sqrt(H)).to(dev).float()
+                yh = kq.mx_dequantize(c, s).view(M, d // H, H)
+                row[f"fwht_{H}"] = sqnr(xf, (yh @ Hm).view(M, d))   # H_H is symmetric and orthonormal
+            rows.append(row)
+            print(json.dumps(row), flush=True)
+    if args.json_out:
+        with open(args.json_out, "w") as fh:
+            json.dump(rows, fh, indent=1)
+
+
+def scipy_hadamard(n):
+    import scipy.linalg
+
+    return scipy.linalg.hadamard(n).astype(np.float64)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -670,8 +740,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the cpu_baseline block")
     ap.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the reference arm")
     ap.add_argument("--json-out", default="")
-    ap.add_argument("--mode", choices=["step", "kernel", "sweep"], default="step",
-                    help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes")
+    ap.add_argument("--mode", choices=["step", "kernel", "sweep", "sqnr"], default="step",
+                    help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes; "
+                         "sqnr: quantisation-error proxy per method")
     ap.add_argument("--kernel", default="kq",
                     help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu or fwht<H>")
     ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
@@ -684,6 +755,8 @@ def main():
         return kernel_mode(args)
     if args.mode == "sweep":
         return sweep_mode(args)
+    if args.mode == "sqnr":
+        return sqnr_mode(args)
     if args.steps < 1 or args.warmup < 3:
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
 

@@ -107,6 +107,21 @@ int kq_quantize_lu(const void *act_bf16, const float *lu_params, int shared,
                    uint8_t *out_codes, uint8_t *out_scales,
                    int64_t M, int64_t d, cudaStream_t stream);
 
+/* The KroQuant quantizer fused with the normalisation that produces its input
+ * ("KroQuant ...", abstract: normalisation layers between blocks force the
+ * transform online).  For every token row h (bf16 [M][d]):
+ *   x_mod = LayerNorm(h) * (1 + gamma[b]) + beta[b]
+ * with LayerNorm without affine (mean and biased variance over the d
+ * channels, eps inside the square root) and AdaLN modulation by per-sample
+ * vectors gamma, beta (float32 [nsamples][d]; row r belongs to sample
+ * r / (M / nsamples)); then kq_quantize on x_mod, which stays in fp32 and is
+ * never written out.  Needs M % nsamples == 0 and d <= 16384.  h, gamma, beta,
+ * factors, out_codes: 16-byte aligned. */
+int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta,
+                     int64_t nsamples, float eps, const float *factors, int shared,
+                     uint8_t *out_codes, uint8_t *out_scales,
+                     int64_t M, int64_t d, cudaStream_t stream);
+
 /* Fixed-Hadamard baseline (the pages' comparison point for the on-the-fly
  * kernel, a fast Walsh-Hadamard transform): y = H_H x / sqrt(H) on every H
  * consecutive channels of a row, H_H the Sylvester Hadamard matrix, H a
@@ -125,6 +140,19 @@ int fwht_quantize(const void *act_bf16, int64_t H,
  * invertible (det != 0); a zero determinant yields inf/NaN outputs. */
 int kq_fold_weights(const float *W, const float *factors, int shared,
                     float *W_out, int64_t N, int64_t d, cudaStream_t stream);
+
+/* Inverse transform, x = T^-1 y per 32-block (y, x_out float32 [M][d], may not
+ * alias): the Kronecker product of the factor inverses G_k^-1 applied as
+ * butterflies.  With mx_dequantize it gives the round trip x -> codes/scales
+ * -> x^ used to measure quantisation error.  Every factor must be invertible. */
+int kq_inverse_f32(const float *y, const float *factors, int shared,
+                   float *x_out, int64_t M, int64_t d, cudaStream_t stream);
+
+/* MXFP4 decode: out[r][32j + i] = E2M1(code) * 2^(scale - 127) (float32
+ * [M][d]; exact in fp32; scale byte 0xFF gives NaN).  codes and out 16-byte
+ * aligned. */
+int mx_dequantize(const uint8_t *codes, const uint8_t *scales, float *out,
+                  int64_t M, int64_t d, cudaStream_t stream);
 
 /* Test export: the fp32 transform y = T x (float32 [M][d]) exactly as the
  * quantizer computes it before the amax, for the transform-accuracy check. */

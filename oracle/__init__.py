@@ -55,6 +55,12 @@ def lib():
         L.oracle_kq_quantize_lu.restype = ci
         L.oracle_fwht_transform.argtypes = [p, i64, i64, i64, p, p, p, p]
         L.oracle_fwht_transform.restype = ci
+        L.oracle_mx_dequantize.argtypes = [p, p, i64, i64, p]
+        L.oracle_mx_dequantize.restype = ci
+        L.oracle_kq_inverse.argtypes = [p, p, ci, i64, i64, p, p]
+        L.oracle_kq_inverse.restype = ci
+        L.oracle_norm_kq.argtypes = [p, p, p, i64, ctypes.c_double, p, ci, i64, i64, p, p, p, p]
+        L.oracle_norm_kq.restype = ci
         _lib = L
     return _lib
 
@@ -227,3 +233,52 @@ def fwht_quantize(x_bf16, H):
     _check(lib().oracle_fwht_transform(_ptr(x), int(H), M, d, None, None, _ptr(codes), _ptr(scales)),
            "fwht_quantize")
     return codes, scales
+
+
+def mx_dequantize(codes, scales):
+    """fp32 [M, d] decode of MXFP4 codes [M, d/2] and E8M0 scales [M, d/32]."""
+    c = _c(codes, np.uint8)
+    sc = _c(scales, np.uint8)
+    M, d = c.shape[0], c.shape[1] * 2
+    out = np.empty((M, d), np.float32)
+    _check(lib().oracle_mx_dequantize(_ptr(c), _ptr(sc), M, d, _ptr(out)), "mx_dequantize")
+    return out
+
+
+def kq_inverse(y, factors, shared=False, want_absbound=False):
+    """x = K^-1 y per 32-block (double Gauss-Jordan inverse, rounded once to fp32)."""
+    yv = _c(y, np.float32)
+    M, d = _shape(yv)
+    f = _c(factors, np.float32)
+    x = np.empty((M, d), np.float32)
+    ab = np.empty((M, d), np.float64) if want_absbound else None
+    _check(lib().oracle_kq_inverse(_ptr(yv), _ptr(f), int(bool(shared)), M, d, _ptr(x), _ptr(ab)), "kq_inverse")
+    return (x, ab) if want_absbound else x
+
+
+def norm_kq(h_bf16, gamma, beta, eps, factors, shared=False, want=("codes",)):
+    """LayerNorm + AdaLN modulation + KroQuant quantizer (double), see kq_oracle.c R9.
+
+    gamma, beta: [nsamples, d] float32.  `want` picks outputs among
+    "codes" (codes, scales), "y" (fp32 transform) and "absb" (|K||x_mod|).
+    """
+    h = _c(h_bf16, np.uint16)
+    M, d = _shape(h)
+    g = _c(gamma, np.float32)
+    b = _c(beta, np.float32)
+    ns = g.shape[0]
+    f = _c(factors, np.float32)
+    y = np.empty((M, d), np.float32) if "y" in want else None
+    ab = np.empty((M, d), np.float64) if "absb" in want else None
+    codes = np.empty((M, d // 2), np.uint8) if "codes" in want else None
+    scales = np.empty((M, d // 32), np.uint8) if "codes" in want else None
+    _check(lib().oracle_norm_kq(_ptr(h), _ptr(g), _ptr(b), ns, float(eps), _ptr(f), int(bool(shared)), M, d,
+                                _ptr(y), _ptr(ab), _ptr(codes), _ptr(scales)), "norm_kq")
+    out = {}
+    if codes is not None:
+        out["codes"], out["scales"] = codes, scales
+    if y is not None:
+        out["y"] = y
+    if ab is not None:
+        out["absb"] = ab
+    return out

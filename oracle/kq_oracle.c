@@ -47,6 +47,13 @@
  *      k = 0..4 is G1..G5; "shared" mode uses one set for every column.
  *   R7 LU storage: params[j][k][3] = (a, b, c) of G_(k+1), L unit lower
  *      triangular.
+ *   R9 The producer the quantizer is fused into is the DiT block's
+ *      pre-linear normalisation: LayerNorm without affine over the d channels
+ *      of a token row (mean, biased variance, eps inside the square root),
+ *      then AdaLN modulation x_mod = LN(h) (1 + gamma_b) + beta_b with
+ *      per-sample vectors gamma_b, beta_b of length d; rows are grouped by
+ *      sample, M / nsamples consecutive rows per sample.  x_mod is not rounded
+ *      to bf16 (nothing is written between the two steps).
  *   R8 The fixed-Hadamard baseline of block size H (a power of two, 32 <= H,
  *      H | d) is the orthonormal Sylvester transform H_H / sqrt(H) on every
  *      H consecutive channels, followed by the same MX quantizer (blocks of
@@ -495,5 +502,114 @@ int oracle_fwht_transform(const uint16_t *x, int64_t H, int64_t M, int64_t d, fl
         free(xv);
         free(yv);
     }
+    return 0;
+}
+
+/* [OCP-MX] MXFP4 decode: value = E2M1(code) * 2^(byte - 127); byte 0xFF is NaN. */
+int oracle_mx_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t M, int64_t d, float *out)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t j = 0; j < nb; ++j) {
+            uint8_t sb = scales[r * nb + j];
+            for (int i = 0; i < BLK; ++i) {
+                uint8_t byte = codes[r * (d / 2) + j * (BLK / 2) + i / 2];
+                uint8_t c = (i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+                double v = E2M1_GRID[c & 7];
+                if (c & 8) v = -v;
+                out[r * d + j * BLK + i] = (sb == 0xFF) ? (float)NAN : (float)ldexp(v, (int)sb - 127);
+            }
+        }
+    return 0;
+}
+
+/* x = K^(j)^-1 y on every 32-block (Gauss-Jordan inverse of the dense K, in
+ * double, rounded once); absb receives (|K^-1| |y|)_i. */
+int oracle_kq_inverse(const float *y, const float *factors, int shared, int64_t M, int64_t d, float *x, double *absb)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+    int64_t ncol = shared ? 1 : nb;
+    double *K = expand_all(factors, shared, nb);
+    if (!K) return -5;
+    double *Ki = (double *)malloc((size_t)ncol * BLK * BLK * sizeof(double));
+    if (!Ki) {
+        free(K);
+        return -5;
+    }
+    int bad = 0;
+    for (int64_t j = 0; j < ncol; ++j)
+        if (oracle_inverse32(K + j * BLK * BLK, Ki + j * BLK * BLK) != 0) bad = 1;
+    free(K);
+    if (bad) {
+        free(Ki);
+        return -3;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kij = Ki + (shared ? 0 : j) * BLK * BLK;
+            for (int i = 0; i < BLK; ++i) {
+                double sacc = 0.0, sa = 0.0;
+                for (int l = 0; l < BLK; ++l) {
+                    double yv = (double)y[r * d + j * BLK + l];
+                    sacc += Kij[i * BLK + l] * yv;
+                    sa += fabs(Kij[i * BLK + l]) * fabs(yv);
+                }
+                x[r * d + j * BLK + i] = (float)sacc;
+                if (absb) absb[r * d + j * BLK + i] = sa;
+            }
+        }
+    free(Ki);
+    return 0;
+}
+
+/* [KQ-abs] "normalization layers ... force this transform to run online": the
+ * quantizer fused with the normalisation that produces its input (R9).  In
+ * double: mu, var over the row, x_mod, then y = K x_mod per block, rounded once
+ * to fp32; absb = (|K| |x_mod|)_i; codes/scales by the MX quantizer. */
+int oracle_norm_kq(const uint16_t *h, const float *gamma, const float *beta, int64_t nsamples, double eps,
+                   const float *factors, int shared, int64_t M, int64_t d, float *y, double *absb,
+                   uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0 || nsamples <= 0 || M % nsamples != 0) return -2;
+    int64_t nb = d / BLK;
+    int64_t rows_per = M / nsamples;
+    double *K = expand_all(factors, shared, nb);
+    if (!K) return -5;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        const int64_t b = r / rows_per;
+        double *xm = (double *)malloc((size_t)d * sizeof(double));
+        double mu = 0.0, var = 0.0;
+        for (int64_t c = 0; c < d; ++c) mu += bf16_value(h[r * d + c]);
+        mu /= (double)d;
+        for (int64_t c = 0; c < d; ++c) {
+            double t = bf16_value(h[r * d + c]) - mu;
+            var += t * t;
+        }
+        var /= (double)d;
+        double inv = 1.0 / sqrt(var + eps);
+        for (int64_t c = 0; c < d; ++c)
+            xm[c] = (bf16_value(h[r * d + c]) - mu) * inv * (1.0 + (double)gamma[b * d + c]) + (double)beta[b * d + c];
+        for (int64_t j = 0; j < nb; ++j) {
+            const double *Kj = K + (shared ? 0 : j) * BLK * BLK;
+            float yv[BLK];
+            for (int i = 0; i < BLK; ++i) {
+                double sacc = 0.0, sa = 0.0;
+                for (int l = 0; l < BLK; ++l) {
+                    sacc += Kj[i * BLK + l] * xm[j * BLK + l];
+                    sa += fabs(Kj[i * BLK + l]) * fabs(xm[j * BLK + l]);
+                }
+                yv[i] = (float)sacc;
+                if (y) y[r * d + j * BLK + i] = yv[i];
+                if (absb) absb[r * d + j * BLK + i] = sa;
+            }
+            if (codes) oracle_mx_block(yv, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+        }
+        free(xm);
+    }
+    free(K);
     return 0;
 }

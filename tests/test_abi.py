@@ -134,6 +134,21 @@ def test_lu_and_fwht_argument_errors(L):
     assert L.fwht_quantize(None, 32, None, None, 0, 64, None) == 0
 
 
+def test_norm_inverse_dequant_argument_errors(L):
+    import ctypes as C
+
+    f = C.c_float
+    assert L.norm_kq_quantize(P(16), P(16), P(16), 2, f(1e-6), P(16), 0, P(16), P(16), 5, 64, None) == -2
+    assert L.norm_kq_quantize(P(16), P(16), P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 32 * 513, None) == -2
+    assert L.norm_kq_quantize(P(16), None, P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 64, None) == -1
+    assert L.norm_kq_quantize(P(16), P(8), P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 64, None) == -3
+    assert L.norm_kq_quantize(P(16), P(16), P(16), 1, f(-1.0), P(16), 0, P(16), P(16), 4, 64, None) == -2
+    assert L.kq_inverse_f32(P(16), P(16), 0, None, 4, 64, None) == -1
+    assert L.kq_inverse_f32(P(16), P(16), 0, P(16), 4, 40, None) == -2
+    assert L.mx_dequantize(P(16), P(16), P(8), 4, 64, None) == -3
+    assert L.mx_dequantize(None, None, None, 0, 64, None) == 0
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
 

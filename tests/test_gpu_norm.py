@@ -1,0 +1,52 @@
+"""The quantizer fused with LayerNorm + AdaLN modulation vs the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import parity_check as pc
+import w4a4_mxfp4_post_b200 as kq
+from w4a4_mxfp4_post_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-6
+
+
+def dev(a, device):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def dev_bf16(bits, device):
+    import torch
+
+    return dev(bits.view(np.int16), device).view(torch.bfloat16)
+
+
+CASES = [(64, 128, 1, False), (37, 96, 1, False), (8192, 1152, 2, False), (2048, 5600, 2, False),
+         (2048, 2240, 4, True), (512, 12288, 2, False), (300, 4608, 3, False)]
+
+
+@pytest.mark.parametrize("M,d,ns,shared", CASES, ids=[f"{c[0]}x{c[1]}-s{c[2]}{'-shared' if c[3] else ''}"
+                                                       for c in CASES])
+def test_norm_kq_matches_oracle(cuda_device, M, d, ns, shared):
+    h = synth.activation("pixart", M, d, seed=M + d)
+    gamma, beta = synth.adaln(ns, d, seed=d)
+    F = synth.factors(d // 32, seed=d, shared=shared)
+    c, s = kq.norm_kq_quantize(dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device),
+                               dev(F, cuda_device), eps=EPS, shared=shared)
+    ref = oracle.norm_kq(h, gamma, beta, EPS, F, shared=shared, want=("codes", "y", "absb"))
+    res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
+    assert res["ok"], res
+
+
+def test_norm_kq_shape_errors(cuda_device):
+    import torch
+
+    h = dev_bf16(synth.activation("pixart", 6, 64, 1), cuda_device)
+    g = torch.zeros((4, 64), dtype=torch.float32, device=cuda_device)
+    F = dev(synth.factors(2, 1), cuda_device)
+    with pytest.raises(kq.KroQuantError) as ei:          # 6 rows, 4 samples
+        kq.norm_kq_quantize(h, g, g.clone(), F)
+    assert ei.value.status == kq.KQ_ERR_SHAPE

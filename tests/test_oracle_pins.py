@@ -367,3 +367,72 @@ def test_fwht_32_is_kroquant_with_hadamard_factors():
     y_h, ab = oracle.fwht_transform(x, 32, want_absbound=True)
     y_k = oracle.kq_transform(x, F)
     np.testing.assert_array_less(np.abs(y_h.astype(np.float64) - y_k), 1e-6 * ab + 1e-30)
+
+
+# ---------------------------------------------------------------- decode and inverse
+def test_dequantize_matches_ml_dtypes_decode():
+    rng = np.random.default_rng(31)
+    M, d = 6, 128
+    codes = rng.integers(0, 256, (M, d // 2), dtype=np.uint8)
+    scales = rng.integers(0, 255, (M, d // 32), dtype=np.uint8)     # 0..254: finite
+    out = oracle.mx_dequantize(codes, scales)
+    nib = np.empty((M, d), np.uint8)
+    nib[:, 0::2] = codes & 0xF
+    nib[:, 1::2] = codes >> 4
+    vals = nib.astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    sc = scales.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    np.testing.assert_array_equal(out, (vals * np.repeat(sc, 32, axis=1)).astype(np.float32))
+    s255 = scales.copy()
+    s255[0, 0] = 0xFF
+    assert np.isnan(oracle.mx_dequantize(codes, s255)[0, :32]).all()
+
+
+def test_round_trip_error_is_within_half_a_step():
+    # MX round trip: |x - x^| <= half the E2M1 spacing at |x| (times 2^e), except
+    # where |x| 2^-e is beyond the largest grid point 6 (saturation).
+    x = synth.activation("pixart", 64, 256, 33)
+    c, s = oracle.mx_quantize(x)
+    xh = oracle.mx_dequantize(c, s).astype(np.float64)
+    xv = f32(x).astype(np.float64)
+    e = np.repeat(s.astype(np.int64) - 127, 32, axis=1)
+    a = np.abs(xv) * 2.0 ** -e
+    step = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+    assert np.all(a <= 8)
+    ok = np.abs(xv - xh) * 2.0 ** -e <= np.where(a > 6, a - 6, step / 2) + 1e-12
+    assert ok.all()
+
+
+def test_inverse_undoes_the_transform():
+    M, d = 8, 128
+    x = synth.activation("pixart", M, d, 34)
+    F = rand_factors(d // 32)
+    y = oracle.kq_transform(x, F)
+    xr, ab = oracle.kq_inverse(y, F, want_absbound=True)
+    np.testing.assert_array_less(np.abs(xr.astype(np.float64) - f32(x)), 1e-5 * ab + 1e-30)
+    # and equals the library inverse of each dense block
+    Kinv = [np.linalg.inv(oracle.kron_expand(F[j])) for j in range(d // 32)]
+    ref = np.concatenate([y[:, 32 * j:32 * j + 32].astype(np.float64) @ Kinv[j].T for j in range(d // 32)], axis=1)
+    np.testing.assert_array_less(np.abs(xr - ref), ab * 2.0 ** -23 + 1e-30)
+
+
+# ---------------------------------------------------------------- fused normalisation (producer) + quantizer
+def test_norm_kq_matches_torch_layer_norm_then_kron():
+    import torch
+
+    M, d, ns, eps = 12, 128, 3, 1e-6
+    h = synth.activation("pixart", M, d, 51)
+    rng = np.random.default_rng(51)
+    gamma = (0.2 * rng.standard_normal((ns, d))).astype(np.float32)
+    beta = (0.1 * rng.standard_normal((ns, d))).astype(np.float32)
+    F = rand_factors(d // 32)
+    out = oracle.norm_kq(h, gamma, beta, eps, F, want=("codes", "y", "absb"))
+    hv = torch.from_numpy(f32(h).astype(np.float64))
+    ln = torch.nn.functional.layer_norm(hv, (d,), eps=eps).numpy()          # library LayerNorm
+    g64 = np.repeat(gamma.astype(np.float64), M // ns, axis=0)
+    b64 = np.repeat(beta.astype(np.float64), M // ns, axis=0)
+    xm = ln * (1 + g64) + b64
+    ref = np.stack([tensor_apply(F[j], xm[:, 32 * j:32 * j + 32]) for j in range(d // 32)], 1).reshape(M, d)
+    np.testing.assert_array_less(np.abs(out["y"] - ref), np.abs(ref) * 2.0 ** -24 + 1e-9 * out["absb"] + 1e-30)
+    ci, si = independent_mx(out["y"].reshape(-1, 32))
+    np.testing.assert_array_equal(out["codes"].reshape(-1, 16), ci)
+    np.testing.assert_array_equal(out["scales"].reshape(-1), si)

@@ -25,7 +25,7 @@ __all__ = [
     "KroQuantError", "lib", "kq_quantize", "kq_quantize_shared", "kq_quantize_variant", "sq_quantize",
     "mx_quantize", "kq_fold_weights", "kq_transform_f32", "kq_last_error", "kq_abi_version",
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
-    "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize",
+    "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize", "kq_inverse_f32", "mx_dequantize", "norm_kq_quantize",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -47,6 +47,8 @@ _SIGS = {
     "kq_transform_f32_variant": "ippipqqp",
     "kq_quantize_lu": "ppippqqp",
     "fwht_quantize": "pqppqqp",
+    "kq_inverse_f32": "ppipqqp",
+    "mx_dequantize": "pppqqp",
 }
 
 _lib = None
@@ -80,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.kq_abi_version.restype = ctypes.c_int
         L.kq_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_int]
         L.kq_wait_timeouts.restype = ctypes.c_int
+        L.norm_kq_quantize.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64, ctypes.c_float, ctypes.c_void_p,
+                                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                                                ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
+        L.norm_kq_quantize.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -228,6 +234,52 @@ def fwht_quantize(act, H, out_codes=None, out_scales=None, stream=None):
     out_codes, out_scales = _outs(act, out_codes, out_scales)
     _call("fwht_quantize", _ptr(act), int(H), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
     return out_codes, out_scales
+
+
+def norm_kq_quantize(h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=None, out_scales=None,
+                     stream=None):
+    """LayerNorm + AdaLN modulation (gamma, beta: [nsamples, d]) fused with kq_quantize."""
+    torch = _torch()
+    M, d = _act(h)
+    _need(gamma, "gamma", torch.float32, h.device)
+    _need(beta, "beta", torch.float32, h.device, tuple(gamma.shape))
+    if gamma.dim() != 2 or gamma.shape[1] != d:
+        raise ValueError("gamma and beta must be [nsamples, d]")
+    _factors(factors, d, shared, h.device)
+    out_codes, out_scales = _outs(h, out_codes, out_scales)
+    _call("norm_kq_quantize", _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps), _ptr(factors),
+          int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def kq_inverse_f32(y, factors, shared=False, out=None, stream=None):
+    """x = T^-1 y per 32-block (fp32 [M, d])."""
+    torch = _torch()
+    _need(y, "y", torch.float32)
+    if y.dim() != 2:
+        raise ValueError("y must be 2-D [M, d]")
+    M, d = y.shape
+    _factors(factors, d, shared, y.device)
+    if out is None:
+        out = torch.empty_like(y)
+    _need(out, "out", torch.float32, y.device, (M, d))
+    _call("kq_inverse_f32", _ptr(y), _ptr(factors), int(bool(shared)), _ptr(out), M, d, _stream(stream))
+    return out
+
+
+def mx_dequantize(codes, scales, out=None, stream=None):
+    """MXFP4 decode of codes [M, d/2] and scales [M, d/32] to fp32 [M, d]."""
+    torch = _torch()
+    _need(codes, "codes", torch.uint8)
+    if codes.dim() != 2:
+        raise ValueError("codes must be 2-D [M, d/2]")
+    M, d = codes.shape[0], codes.shape[1] * 2
+    _need(scales, "scales", torch.uint8, codes.device, (M, d // 32))
+    if out is None:
+        out = torch.empty((M, d), dtype=torch.float32, device=codes.device)
+    _need(out, "out", torch.float32, codes.device, (M, d))
+    _call("mx_dequantize", _ptr(codes), _ptr(scales), _ptr(out), M, d, _stream(stream))
+    return out
 
 
 def sq_quantize_variant(variant, act, mult, out_codes=None, out_scales=None, stream=None):

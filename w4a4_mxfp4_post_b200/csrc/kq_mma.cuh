@@ -18,8 +18,9 @@
 //              two B buffers, and issues the TMA loads of the A tiles (two
 //              {64 cols x 128 rows} boxes, 128-byte swizzle) into a 4-stage ring
 //   warp 1     allocates the tensor memory; one thread issues the MMAs:
-//              kNC x 3 splits x 2 k-steps of M128 N32 K16 per tile into one of
-//              two 128-column fp32 accumulators
+//              2 k-steps x 3 splits x kNC block columns of M128 N32 K16 per
+//              tile (columns innermost) into one of two 128-column fp32
+//              accumulators
 //   warps 2-17 epilogue: tcgen05.ld of a row's 32 values of a block, amax,
 //              E8M0 byte, exact 2^-e scaling (packed FFMA with +0, so exact
 //              zeros come out +0 as in the other variants), E2M1.  Warp w reads
@@ -326,13 +327,17 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(sA + size_t(s) * kAStageBytes);
                 const uint32_t b0 = smem_addr(sB + (bcount & 1) * kBSetBytes);
+                // Consecutive MMAs go to different accumulators (block column
+                // innermost): the six MMAs that accumulate into one column are
+                // kNC issues apart, so their latencies overlap instead of
+                // serialising.
 #pragma unroll
-                for (int jj = 0; jj < kNC; ++jj) {
-                    const uint32_t d = tmem_base + uint32_t(tb * kNC * 32 + jj * 32);
+                for (int kk = 0; kk < 2; ++kk) {
 #pragma unroll
                     for (int sp = 0; sp < 3; ++sp) {
 #pragma unroll
-                        for (int kk = 0; kk < 2; ++kk) {
+                        for (int jj = 0; jj < kNC; ++jj) {
+                            const uint32_t d = tmem_base + uint32_t(tb * kNC * 32 + jj * 32);
                             const uint64_t ad =
                                 smem_desc(a0 + (jj >> 1) * kABoxBytes + (jj & 1) * 64 + kk * 32, 1024, kLayoutSw128);
                             const uint64_t bd = smem_desc(b0 + (jj * 3 + sp) * kBMatBytes + kk * 32, 512, kLayoutSw64);

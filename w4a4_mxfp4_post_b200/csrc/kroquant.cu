@@ -19,6 +19,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <atomic>
 #include <cstdarg>
@@ -208,7 +209,10 @@ kq_butterfly_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ fa
 
 // Fold: w' = w K^-1 for a row vector w, i.e. w'^T = (K^-1)^T w^T, which is
 // the Kronecker product of the 2x2 matrices (G_k^-1)^T = [[g11, -g10],
-// [-g01, g00]] / det(G_k) applied as butterflies.  fp32 in, fp32 out.
+// [-g01, g00]] / det(G_k) applied as butterflies.  With INVERSE, the
+// matrices are G_k^-1 = [[g11, -g01], [-g10, g00]] / det(G_k) instead, i.e.
+// x = K^-1 y per block (the inverse transform).  fp32 in, fp32 out.
+template <bool INVERSE>
 __global__ void __launch_bounds__(kThreads)
 fold_kernel(const float4 *__restrict__ W, const float4 *__restrict__ factors, int shared,
             float4 *__restrict__ W_out, int64_t nblocks, int nb, int64_t T)
@@ -224,8 +228,8 @@ fold_kernel(const float4 *__restrict__ W, const float4 *__restrict__ factors, in
         const float det = fmaf(q.x, q.w, -q.y * q.z);
         const float r = 1.0f / det;
         f[4 * k] = q.w * r;
-        f[4 * k + 1] = -q.z * r;
-        f[4 * k + 2] = -q.y * r;
+        f[4 * k + 1] = (INVERSE ? -q.y : -q.z) * r;
+        f[4 * k + 2] = (INVERSE ? -q.z : -q.y) * r;
         f[4 * k + 3] = q.x * r;
     }
     for (int64_t g = t; g < nblocks; g += T) {
@@ -351,10 +355,13 @@ __device__ __forceinline__ void load_block_nc(const uint4 *__restrict__ act, int
 }
 
 // Column state of the KroQuant transform in unit-diagonal form (see the
-// variant-2 kernel below for the derivation).
+// variant-2 kernel below for the derivation): the 32 values of D as 16 pairs
+// (D_i, D_{i+16}) matching the register pairs of the data, and the
+// off-diagonal coefficients of the five unit factors (scalars, used as
+// broadcast operands of the packed instructions).
 struct KqFast {
     float2 DP[16];            // (D_i, D_{i+16})
-    float2 B[4], C[4];        // stages on bits 0..3 (G5, G4, G3, G2), broadcast
+    float B[4], C[4];         // stages on bits 0..3 (G5, G4, G3, G2)
     float b4, c4;             // stage on bit 4 (G1)
 };
 
@@ -380,8 +387,8 @@ __device__ __forceinline__ bool kq_fast_setup(const float4 (&g)[5], KqFast &st)
     for (int i = 0; i < 16; ++i) st.DP[i] = make_float2(dd[i], dd[i + 16]);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-        st.B[b] = bcast(bb[4 - b]);
-        st.C[b] = bcast(cc[4 - b]);
+        st.B[b] = bb[4 - b];
+        st.C[b] = cc[4 - b];
     }
     st.b4 = bb[0];
     st.c4 = cc[0];
@@ -390,17 +397,83 @@ __device__ __forceinline__ bool kq_fast_setup(const float4 (&g)[5], KqFast &st)
 
 __device__ __forceinline__ void kq_fast_apply(float2 (&p)[16], const KqFast &st)
 {
-    unit_stage2<1>(p, st.B[0], st.C[0]);
-    unit_stage2<2>(p, st.B[1], st.C[1]);
-    unit_stage2<4>(p, st.B[2], st.C[2]);
-    unit_stage2<8>(p, st.B[3], st.C[3]);
-    // D applied as D*z + (+0): the same value as D*z, except that an exact
-    // zero comes out as +0 whatever the signs of D and z (as a sum of
-    // products that cancels exactly does in round-to-nearest).
+    unit_stage2<1>(p, bcast(st.B[0]), bcast(st.C[0]));
+    unit_stage2<2>(p, bcast(st.B[1]), bcast(st.C[1]));
+    unit_stage2<4>(p, bcast(st.B[2]), bcast(st.C[2]));
+    unit_stage2<8>(p, bcast(st.B[3]), bcast(st.C[3]));
+    // stage on bit 4, then D applied as D*z + (+0): the same value as D*z,
+    // except that an exact zero comes out as +0 whatever the signs of D and z
+    // (as a sum of products that cancels exactly does in round-to-nearest).
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float lo = p[i].x, hi = p[i].y;
         p[i] = __ffma2_rn(make_float2(fmaf(st.b4, hi, lo), fmaf(st.c4, lo, hi)), st.DP[i], plus_zero2());
+    }
+}
+
+// Compact column state (used where registers are scarce: the fused
+// normalisation kernel).  D = (x)_k diag(g00_k, g11_k) is kept factored as
+// diag_G1 (x) D_rest: the pair (g00, g11) of G1 (index
+// bit 4, the two halves of every register pair) and the 16 values of D_rest
+// (bits 0..3), which multiply both halves of pair i alike.  All coefficients
+// are then scalars used as broadcast operands of the packed instructions,
+// 28 registers in all, at the cost of one more packed multiply per pair than
+// the paired form below.
+struct KqFastC {
+    float Dr[16];             // D_rest_i, i = 0..15
+    float d40, d41;           // diagonal of G1
+    float B[4], C[4];         // stages on bits 0..3 (G5, G4, G3, G2)
+    float b4, c4;             // stage on bit 4 (G1)
+};
+
+__device__ __forceinline__ bool kq_fast_setup_c(const float4 (&g)[5], KqFastC &st)
+{
+    float d0[5], d1[5], bb[5], cc[5];
+    bool fast = true;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) fast &= unit_split(g[k], d0[k], d1[k], bb[k], cc[k]);
+    // D_rest_i = prod over bits 0..3 of (bit b of i ? g11 : g00) of G_(5-b)
+    float dd[16];
+    dd[0] = 1.0f;
+#pragma unroll
+    for (int bit = 0; bit < 4; ++bit) {
+        const int k = 4 - bit;
+#pragma unroll
+        for (int i = 0; i < (1 << bit); ++i) {
+            dd[i + (1 << bit)] = dd[i] * d1[k];
+            dd[i] = dd[i] * d0[k];
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st.Dr[i] = dd[i];
+    st.d40 = d0[0];
+    st.d41 = d1[0];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        st.B[b] = bb[4 - b];
+        st.C[b] = cc[4 - b];
+    }
+    st.b4 = bb[0];
+    st.c4 = cc[0];
+    return fast;
+}
+
+__device__ __forceinline__ void kq_fast_apply_c(float2 (&p)[16], const KqFastC &st)
+{
+    unit_stage2<1>(p, bcast(st.B[0]), bcast(st.C[0]));
+    unit_stage2<2>(p, bcast(st.B[1]), bcast(st.C[1]));
+    unit_stage2<4>(p, bcast(st.B[2]), bcast(st.C[2]));
+    unit_stage2<8>(p, bcast(st.B[3]), bcast(st.C[3]));
+    // stage on bit 4, then D = diag_G1 (x) D_rest.  The last multiply is an FMA
+    // with +0: the same value, except that an exact zero comes out +0 whatever
+    // the signs (as a sum of products that cancels exactly does in
+    // round-to-nearest).
+    const float2 d4 = make_float2(st.d40, st.d41);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float lo = p[i].x, hi = p[i].y;
+        const float2 t = __fmul2_rn(make_float2(fmaf(st.b4, hi, lo), fmaf(st.c4, lo, hi)), d4);
+        p[i] = __ffma2_rn(t, bcast(st.Dr[i]), plus_zero2());
     }
 }
 
@@ -920,6 +993,147 @@ mx_staged_kernel(const __grid_constant__ CUtensorMap act_map, uint4 *__restrict_
     });
 }
 
+// MXFP4 decode (the consumer side of the quantizers): value = E2M1(code) *
+// 2^(byte - 127), exact in fp32 (two significant bits times a power of two;
+// byte 0 gives the subnormal 2^-127, byte 0xFF is NaN).  The codes go
+// through the hardware E2M1 -> f16x2 conversion (exact: every E2M1 value is
+// an f16 value).
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte)
+{
+    uint32_t h2;
+    asm("{\n\t.reg .b8 q;\n\tcvt.u8.u32 q, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, q;\n\t}" : "=r"(h2) : "r"(byte));
+    const __half2 h = *reinterpret_cast<const __half2 *>(&h2);
+    return make_float2(__low2float(h), __high2float(h));
+}
+
+__device__ __forceinline__ float e8m0_value(uint32_t sb)
+{
+    if (sb == 0xFFu) return __uint_as_float(0x7fc00000u);
+    return sb ? __uint_as_float(sb << 23) : __uint_as_float(0x00400000u);
+}
+
+__global__ void __launch_bounds__(kThreads)
+mx_dequantize_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict__ scales, float4 *__restrict__ out,
+                     int64_t nblocks)
+{
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < nblocks; g += stride) {
+        const uint4 c = __ldg(codes + g);
+        const float s = e8m0_value(__ldg(scales + g));
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const float2 e = e2m1x2_to_f32x2((w[q] >> (8 * b)) & 0xFFu);   // low nibble = even element
+                v[8 * q + 2 * b] = e.x * s;
+                v[8 * q + 2 * b + 1] = e.y * s;
+            }
+        float4 *o = out + g * 8;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+// The quantizer fused with the normalisation that produces its input (KroQuant
+// abstract: normalisation layers force the transform online).  For every token
+// row h of a bf16 activation: LayerNorm without affine (mean, biased
+// variance, eps inside the square root), AdaLN modulation
+// x_mod = LN(h) (1 + gamma_b) + beta_b with per-sample vectors (rows grouped by
+// sample, rows_per consecutive rows each), then the KroQuant transform and
+// MXFP4 -- x_mod never leaves registers.  A CTA holds R rows x nb threads:
+// thread (row rl, column j) owns block j of its row, so its column's transform
+// coefficients are set up once; the row statistics are two deterministic tree
+// reductions over the row's nb partial sums in shared memory (two passes, so
+// the variance is the mean of squared deviations, not E[h^2] - mean^2).
+__global__ void __launch_bounds__(512)
+norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
+               int64_t rows_per, float eps, const float *__restrict__ factors, int shared, uint4 *__restrict__ codes,
+               uint8_t *__restrict__ scales, int64_t M, int nb, int R, int npow)
+{
+    extern __shared__ float red[];   // [R * nb] partial sums
+    const int tid = threadIdx.x;
+    const int rl = tid / nb, j = tid - (tid / nb) * nb;
+    const int base = rl * nb;
+    const int d = nb * kBlk;
+    KqFastC st;
+    bool fast;
+    {
+        float4 g[5];
+        load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
+        fast = kq_fast_setup_c(g, st);
+    }
+
+    for (int64_t r0 = int64_t(blockIdx.x) * R; r0 < M; r0 += int64_t(gridDim.x) * R) {   // CTA-uniform
+        const int64_t r = r0 + rl;
+        const bool valid = r < M;
+        uint4 raw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                        make_uint4(0, 0, 0, 0)};
+        if (valid) load_block_nc(h, r * nb + j, raw);
+        float2 p[16];
+        unpack_pairs(raw, p);
+        // row mean
+        float2 acc = p[0];
+#pragma unroll
+        for (int i = 1; i < 16; ++i) acc = __fadd2_rn(acc, p[i]);
+        red[tid] = acc.x + acc.y;
+        __syncthreads();
+        for (int s2 = npow >> 1; s2 > 0; s2 >>= 1) {
+            if (j < s2 && j + s2 < nb) red[base + j] += red[base + j + s2];
+            __syncthreads();
+        }
+        const float mu = red[base] / float(d);
+        __syncthreads();
+        // row variance (mean of squared deviations)
+        const float2 nmu = make_float2(-mu, -mu);
+        float2 q = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float2 t = __fadd2_rn(p[i], nmu);
+            q = __ffma2_rn(t, t, q);
+        }
+        red[tid] = q.x + q.y;
+        __syncthreads();
+        for (int s2 = npow >> 1; s2 > 0; s2 >>= 1) {
+            if (j < s2 && j + s2 < nb) red[base + j] += red[base + j + s2];
+            __syncthreads();
+        }
+        const float var = red[base] / float(d);
+        __syncthreads();
+        if (!valid) continue;
+        const float inv = 1.0f / sqrtf(var + eps);
+        // modulation with this row's sample vectors
+        const int64_t b = r / rows_per;
+        const float4 *gp = reinterpret_cast<const float4 *>(gamma + b * d + j * kBlk);
+        const float4 *bp = reinterpret_cast<const float4 *>(beta + b * d + j * kBlk);
+        const float2 iv = make_float2(inv, inv);
+        // pair i holds elements (i, i + 16): gamma/beta of 4 consecutive pairs come
+        // from float4 q4 (elements 4 q4 ..) and q4 + 4 (elements 16 + 4 q4 ..)
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 ga = __ldg(gp + q4), gb = __ldg(gp + q4 + 4);
+            const float4 ba = __ldg(bp + q4), bb = __ldg(bp + q4 + 4);
+            const float g_lo[4] = {ga.x, ga.y, ga.z, ga.w}, g_hi[4] = {gb.x, gb.y, gb.z, gb.w};
+            const float b_lo[4] = {ba.x, ba.y, ba.z, ba.w}, b_hi[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * q4 + e;
+                const float2 t = __fmul2_rn(__fadd2_rn(p[i], nmu), iv);
+                p[i] = __ffma2_rn(t, make_float2(1.0f + g_lo[e], 1.0f + g_hi[e]), make_float2(b_lo[e], b_hi[e]));
+            }
+        }
+        if (fast) {
+            kq_fast_apply_c(p, st);
+        } else {   // rare: the factors are reloaded (L1) rather than kept live
+            float4 g[5];
+            load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
+            kq_direct_apply(p, g);
+        }
+        kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+    }
+}
+
 #include "kq_mma.cuh"
 
 // ---------------------------------------------------------------------------
@@ -973,7 +1187,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 // per SM (occupancy query, cached per device and kernel).
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
-    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kNumKernels
+    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1445,6 +1659,86 @@ int fwht_quantize(const void *act_bf16, int64_t H, uint8_t *out_codes, uint8_t *
     return launch_check(fn);
 }
 
+int kq_inverse_f32(const float *y, const float *factors, int shared, float *x_out, int64_t M, int64_t d,
+                   cudaStream_t stream)
+{
+    const char *fn = "kq_inverse_f32";
+    if (M < 0 || d <= 0 || d % kBlk != 0) return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32", fn);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d)) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (M == 0) return ok();
+    if (!y || !factors || !x_out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(y, 16) || !aligned(x_out, 16) || !aligned(factors, 16))
+        return fail(KQ_ERR_ALIGN, "%s: y, x_out and factors must be 16-byte aligned", fn);
+    const int64_t nb = d / kBlk;
+    Geometry geo;
+    int rc = launch_pinned(fn, kInverse, fold_kernel<true>, M, nb, &geo);
+    if (rc != KQ_OK) return rc;
+    fold_kernel<true><<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(y),
+                                                         reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
+                                                         reinterpret_cast<float4 *>(x_out), M * nb, int(nb), geo.T);
+    return launch_check(fn);
+}
+
+int mx_dequantize(const uint8_t *codes, const uint8_t *scales, float *out, int64_t M, int64_t d, cudaStream_t stream)
+{
+    const char *fn = "mx_dequantize";
+    if (M < 0 || d <= 0 || d % kBlk != 0) return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32", fn);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d)) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (M == 0) return ok();
+    if (!codes || !scales || !out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(codes, 16) || !aligned(out, 16)) return fail(KQ_ERR_ALIGN, "%s: codes and out must be 16-byte aligned", fn);
+    const int64_t nblocks = M * (d / kBlk);
+    int64_t target = 0;
+    int rc = resident_threads(kDequant, reinterpret_cast<const void *>(mx_dequantize_kernel), &target);
+    if (rc != KQ_OK) return rc;
+    int64_t T = target < nblocks ? target : nblocks;
+    mx_dequantize_kernel<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(codes), scales, reinterpret_cast<float4 *>(out), nblocks);
+    return launch_check(fn);
+}
+
+int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, int64_t nsamples, float eps,
+                     const float *factors, int shared, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
+                     cudaStream_t stream)
+{
+    const char *fn = "norm_kq_quantize";
+    if (M < 0 || d <= 0 || d % kBlk != 0 || d / kBlk > 512)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32, at most 16384 (M=%lld, d=%lld)",
+                    fn, (long long)M, (long long)d);
+    if (nsamples <= 0 || M % nsamples != 0)
+        return fail(KQ_ERR_SHAPE, "%s: M must be a multiple of nsamples > 0 (M=%lld, nsamples=%lld)", fn,
+                    (long long)M, (long long)nsamples);
+    if (M > 0 && M > INT64_MAX / d) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (!(eps >= 0.0f)) return fail(KQ_ERR_SHAPE, "%s: eps must be >= 0", fn);
+    if (M == 0) return ok();
+    if (!h_bf16 || !gamma || !beta || !factors || !out_codes || !out_scales)
+        return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(h_bf16, 16) || !aligned(out_codes, 16) || !aligned(factors, 16) || !aligned(gamma, 16) ||
+        !aligned(beta, 16))
+        return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
+    const int nb = int(d / kBlk);
+    int R = 256 / nb;
+    if (R < 1) R = 1;
+    int npow = 1;
+    while (npow < nb) npow <<= 1;
+    const int threads = R * nb;
+    const size_t smem = size_t(threads) * sizeof(float);
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel, threads, smem);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+    if (per_sm < 1) per_sm = 1;
+    const int64_t groups = (M + R - 1) / R;
+    int64_t grid = int64_t(sms) * per_sm;
+    if (grid > groups) grid = groups;
+    norm_kq_kernel<<<unsigned(grid), threads, smem, stream>>>(
+        static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
+        reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb, R, npow);
+    return launch_check(fn);
+}
+
 int kq_wait_timeouts(int *count, int reset)
 {
     if (!count) return fail(KQ_ERR_NULL, "kq_wait_timeouts: NULL pointer argument");
@@ -1494,9 +1788,9 @@ int kq_fold_weights(const float *W, const float *factors, int shared, float *W_o
         return fail(KQ_ERR_ALIGN, "kq_fold_weights: W, W_out and factors must be 16-byte aligned");
     const int64_t nb = d / kBlk;
     Geometry geo;
-    int rc = launch_pinned("kq_fold_weights", kFold, fold_kernel, N, nb, &geo);
+    int rc = launch_pinned("kq_fold_weights", kFold, fold_kernel<false>, N, nb, &geo);
     if (rc != KQ_OK) return rc;
-    fold_kernel<<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(W),
+    fold_kernel<false><<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(W),
                                                    reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
                                                    reinterpret_cast<float4 *>(W_out), N * nb, int(nb), geo.T);
     return launch_check("kq_fold_weights");

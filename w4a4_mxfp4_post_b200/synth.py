@@ -169,6 +169,15 @@ def lu_params(nb: int, seed: int, shared: bool = False, noise: float = 0.1) -> n
     return out
 
 
+def adaln(nsamples: int, d: int, seed: int):
+    """AdaLN modulation vectors (gamma, beta), each float32 [nsamples, d]:
+    gamma ~ 0.2 N(0,1), beta ~ 0.1 N(0,1) (conditioning of a diffusion step)."""
+    g = _rng(seed + 3000, 5)
+    gamma = (0.2 * g.standard_normal((nsamples, d))).astype(np.float32)
+    beta = (0.1 * g.standard_normal((nsamples, d))).astype(np.float32)
+    return gamma, beta
+
+
 def sq_multipliers(x_bf16: np.ndarray, alpha: float = 0.5, floor: float = 1e-5) -> np.ndarray:
     """SmoothQuant per-channel multipliers m_c = 1/s_c, s_c = max(max_r |X_rc|, floor)^alpha.
 
