@@ -537,6 +537,8 @@ class RotatingInputs:
         self.F = torch.from_numpy(F).to(dev)
         self.m = torch.from_numpy(m).to(dev)
         self.P = torch.from_numpy(synth.lu_params(d // 32, 4)).to(dev)
+        g, b = synth.adaln(2 if M % 2 == 0 else 1, d, 4)
+        self.gamma, self.beta = torch.from_numpy(g).to(dev), torch.from_numpy(b).to(dev)
 
 
 def time_launches(kind, inp, launches, warmup, stream, graph=True):
@@ -557,6 +559,8 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
             kq.sq_quantize(inp.xs[k], inp.m, inp.cs[k], inp.ss[k], stream=stream)
         elif kind == "mx":
             kq.mx_quantize(inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
+        elif kind == "norm_kq":
+            kq.norm_kq_quantize(inp.xs[k], inp.gamma, inp.beta, inp.F, 1e-6, False, inp.cs[k], inp.ss[k], stream=stream)
         elif kind == "kq_lu":
             kq.kq_quantize_lu(inp.xs[k], inp.P, False, inp.cs[k], inp.ss[k], stream=stream)
         elif kind.startswith("fwht"):
@@ -744,7 +748,7 @@ def main():
                     help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes; "
                          "sqnr: quantisation-error proxy per method")
     ap.add_argument("--kernel", default="kq",
-                    help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu or fwht<H>")
+                    help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H> or norm_kq")
     ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
     ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD")
     ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")

@@ -167,7 +167,10 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
  *   3  the arithmetic of 2 on input staged through shared memory by TMA,
  *   4  the block transform on the tcgen05 tensor cores: Y_j = X_j K_j^T with
  *      K_j expanded in fp32 and split into three bf16 parts (each product
- *      exact in the fp32 accumulator), TMA-fed, accumulators in tensor memory.
+ *      exact in the fp32 accumulator), TMA-fed, accumulators in tensor memory,
+ *   5  the arithmetic of 2 with the diagonal part of the factors in shared
+ *      memory (fewer registers, more resident warps, no prefetch),
+ *   6  the arithmetic of 2 with a two-deep register prefetch.
  * Other values return KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
                         int shared, uint8_t *out_codes, uint8_t *out_scales,

@@ -663,6 +663,118 @@ fwht_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *_
     }
 }
 
+// KroQuant quantizer, lean (variant 5): the arithmetic of variant 2 with the
+// column coefficients (the 32 values of D and the 10 off-diagonal
+// coefficients) kept in shared memory instead of registers, and no register
+// prefetch.  A thread's coefficients sit in its own 176-byte slot (11 x 16 B:
+// an odd number of 16-byte units, so the 8 lanes of a 16-byte shared-load
+// phase hit 8 distinct bank groups) and are re-read every block (11 shared
+// loads).  64 registers per thread instead of 108, so 4 CTAs (32 warps) per
+// SM hide the memory latency without a prefetch.
+constexpr int kLeanSlotFloats = 44;   // 32 D values + 12 pad (176 bytes)
+
+__global__ void __launch_bounds__(kThreads, 4)
+kq_lean_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+               uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
+{
+    __shared__ __align__(16) float dslot[kThreads * kLeanSlotFloats];
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    const bool active = t < T && t < nblocks;
+    const int j = active ? int(t % nb) : 0;
+    float *slot = dslot + threadIdx.x * kLeanSlotFloats;
+    bool fast;
+    {
+        float4 g[5];
+        load_factors(factors, shared, j, g);
+        KqFast st;
+        fast = kq_fast_setup(g, st);
+        float2 *myd = reinterpret_cast<float2 *>(slot);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) myd[i] = st.DP[i];
+        float4 *cq = reinterpret_cast<float4 *>(slot + 32);
+        cq[0] = make_float4(st.B[0], st.C[0], st.B[1], st.C[1]);
+        cq[1] = make_float4(st.B[2], st.C[2], st.B[3], st.C[3]);
+        cq[2] = make_float4(st.b4, st.c4, 0.0f, 0.0f);
+    }
+    if (!active) return;
+    const float4 *dq = reinterpret_cast<const float4 *>(slot);
+    for (int64_t gi = t; gi < nblocks; gi += T) {
+        uint4 raw[4];
+        load_block_nc(act, gi, raw);
+        float2 p[16];
+        unpack_pairs(raw, p);
+        if (fast) {
+            const float4 c01 = dq[8], c23 = dq[9], c4q = dq[10];
+            const float b4 = c4q.x, c4 = c4q.y;
+            unit_stage2<1>(p, bcast(c01.x), bcast(c01.y));
+            unit_stage2<2>(p, bcast(c01.z), bcast(c01.w));
+            unit_stage2<4>(p, bcast(c23.x), bcast(c23.y));
+            unit_stage2<8>(p, bcast(c23.z), bcast(c23.w));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 dd = dq[q];   // (D_2q, D_2q+16, D_2q+1, D_2q+17)
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int i = 2 * q + h2;
+                    const float lo = p[i].x, hi = p[i].y;
+                    const float2 dp = h2 ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y);
+                    p[i] = __ffma2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), dp, plus_zero2());
+                }
+            }
+        } else {   // rare: the factors are reloaded (L1) rather than kept live
+            float4 g[5];
+            load_factors(factors, shared, j, g);
+            kq_direct_apply(p, g);
+        }
+        kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+    }
+}
+
+// KroQuant quantizer, variant 6: the arithmetic of variant 2 with a two-deep
+// register prefetch (three 64-byte blocks per thread in flight), for more
+// memory-level parallelism at the same 2 CTAs per SM.
+__global__ void __launch_bounds__(kThreads, 2)
+kq_packed2_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
+{
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    if (t >= T || t >= nblocks) return;
+    const int j = int(t % nb);
+    KqFast st;
+    bool fast;
+    {
+        float4 g[5];
+        load_factors(factors, shared, j, g);
+        fast = kq_fast_setup(g, st);
+    }
+    int64_t gi = t;
+    uint4 r0[4], r1[4];
+    load_block_nc(act, gi, r0);
+    if (gi + T < nblocks) load_block_nc(act, gi + T, r1);
+    for (;;) {
+        const int64_t g2 = gi + 2 * T;
+        uint4 r2[4];
+        if (g2 < nblocks) load_block_nc(act, g2, r2);
+        float2 p[16];
+        unpack_pairs(r0, p);
+        if (fast) {
+            kq_fast_apply(p, st);
+        } else {   // rare: the factors are reloaded (L1) rather than kept live
+            float4 g[5];
+            load_factors(factors, shared, j, g);
+            kq_direct_apply(p, g);
+        }
+        kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+        if (gi + T >= nblocks) break;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            r0[q] = r1[q];
+            r1[q] = r2[q];
+        }
+        gi += T;
+    }
+}
+
 // SmoothQuant quantizer on the pair layout: y = fp32(x * m) per channel (one
 // correctly rounded packed multiply), then the MXFP4 block quantizer.
 __global__ void __launch_bounds__(kThreads)
@@ -1042,95 +1154,148 @@ mx_dequantize_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict_
 // variance, eps inside the square root), AdaLN modulation
 // x_mod = LN(h) (1 + gamma_b) + beta_b with per-sample vectors (rows grouped by
 // sample, rows_per consecutive rows each), then the KroQuant transform and
-// MXFP4 -- x_mod never leaves registers.  A CTA holds R rows x nb threads:
-// thread (row rl, column j) owns block j of its row, so its column's transform
-// coefficients are set up once; the row statistics are two deterministic tree
-// reductions over the row's nb partial sums in shared memory (two passes, so
-// the variance is the mean of squared deviations, not E[h^2] - mean^2).
-__global__ void __launch_bounds__(512)
+// MXFP4 -- x_mod never leaves registers.
+//
+// One warp per row.  Pass 1 streams the row from HBM; each lane folds the
+// blocks it reads into a running (count, mean, sum of squared deviations)
+// with the parallel-variance combination of Chan, Golub and LeVeque, and five
+// shuffle steps merge the lanes.  Pass 2 reads the row again (from L2: a row is
+// at most 32 KB and a wave of warps touches a few MB) and quantizes every
+// block with its column's coefficients, which the CTA computes once into a
+// shared-memory table: per column the 16 D pairs, the 10 off-diagonal
+// coefficients, a flag for the unit-diagonal form and the 20 raw factors (the
+// direct-form fallback), kNormSlot floats, an odd number of 16-byte units so
+// lanes reading consecutive columns hit distinct bank groups.
+constexpr int kNormSlot = 68;   // 32 DP + 12 (coefficients, flag, pad) + 20 raw + 4 pad = 272 B
+
+struct Welford {
+    float n, mean, m2;
+};
+
+__device__ __forceinline__ Welford welford_merge(Welford a, Welford b)
+{
+    const float n = a.n + b.n;
+    if (n == 0.0f) return a;
+    const float delta = b.mean - a.mean;
+    const float fb = b.n / n;
+    Welford r;
+    r.n = n;
+    r.mean = fmaf(delta, fb, a.mean);
+    r.m2 = a.m2 + b.m2 + delta * delta * a.n * fb;
+    return r;
+}
+
+__global__ void __launch_bounds__(kThreads)
 norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
                int64_t rows_per, float eps, const float *__restrict__ factors, int shared, uint4 *__restrict__ codes,
-               uint8_t *__restrict__ scales, int64_t M, int nb, int R, int npow)
+               uint8_t *__restrict__ scales, int64_t M, int nb)
 {
-    extern __shared__ float red[];   // [R * nb] partial sums
-    const int tid = threadIdx.x;
-    const int rl = tid / nb, j = tid - (tid / nb) * nb;
-    const int base = rl * nb;
-    const int d = nb * kBlk;
-    KqFastC st;
-    bool fast;
-    {
+    extern __shared__ __align__(16) float tab[];   // [nb][kNormSlot]
+    // coefficient table (every column of the row, computed once per CTA)
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
         float4 g[5];
         load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
-        fast = kq_fast_setup_c(g, st);
-    }
-
-    for (int64_t r0 = int64_t(blockIdx.x) * R; r0 < M; r0 += int64_t(gridDim.x) * R) {   // CTA-uniform
-        const int64_t r = r0 + rl;
-        const bool valid = r < M;
-        uint4 raw[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
-                        make_uint4(0, 0, 0, 0)};
-        if (valid) load_block_nc(h, r * nb + j, raw);
-        float2 p[16];
-        unpack_pairs(raw, p);
-        // row mean
-        float2 acc = p[0];
-#pragma unroll
-        for (int i = 1; i < 16; ++i) acc = __fadd2_rn(acc, p[i]);
-        red[tid] = acc.x + acc.y;
-        __syncthreads();
-        for (int s2 = npow >> 1; s2 > 0; s2 >>= 1) {
-            if (j < s2 && j + s2 < nb) red[base + j] += red[base + j + s2];
-            __syncthreads();
-        }
-        const float mu = red[base] / float(d);
-        __syncthreads();
-        // row variance (mean of squared deviations)
-        const float2 nmu = make_float2(-mu, -mu);
-        float2 q = make_float2(0.0f, 0.0f);
+        KqFast st;
+        const bool fast = kq_fast_setup(g, st);
+        float *e = tab + j * kNormSlot;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const float2 t = __fadd2_rn(p[i], nmu);
-            q = __ffma2_rn(t, t, q);
+            e[2 * i] = st.DP[i].x;
+            e[2 * i + 1] = st.DP[i].y;
         }
-        red[tid] = q.x + q.y;
-        __syncthreads();
-        for (int s2 = npow >> 1; s2 > 0; s2 >>= 1) {
-            if (j < s2 && j + s2 < nb) red[base + j] += red[base + j + s2];
-            __syncthreads();
-        }
-        const float var = red[base] / float(d);
-        __syncthreads();
-        if (!valid) continue;
-        const float inv = 1.0f / sqrtf(var + eps);
-        // modulation with this row's sample vectors
-        const int64_t b = r / rows_per;
-        const float4 *gp = reinterpret_cast<const float4 *>(gamma + b * d + j * kBlk);
-        const float4 *bp = reinterpret_cast<const float4 *>(beta + b * d + j * kBlk);
-        const float2 iv = make_float2(inv, inv);
-        // pair i holds elements (i, i + 16): gamma/beta of 4 consecutive pairs come
-        // from float4 q4 (elements 4 q4 ..) and q4 + 4 (elements 16 + 4 q4 ..)
+        float4 *q = reinterpret_cast<float4 *>(e + 32);
+        q[0] = make_float4(st.B[0], st.C[0], st.B[1], st.C[1]);
+        q[1] = make_float4(st.B[2], st.C[2], st.B[3], st.C[3]);
+        q[2] = make_float4(st.b4, st.c4, fast ? 1.0f : 0.0f, 0.0f);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 ga = __ldg(gp + q4), gb = __ldg(gp + q4 + 4);
-            const float4 ba = __ldg(bp + q4), bb = __ldg(bp + q4 + 4);
-            const float g_lo[4] = {ga.x, ga.y, ga.z, ga.w}, g_hi[4] = {gb.x, gb.y, gb.z, gb.w};
-            const float b_lo[4] = {ba.x, ba.y, ba.z, ba.w}, b_hi[4] = {bb.x, bb.y, bb.z, bb.w};
+        for (int k = 0; k < 5; ++k) q[3 + k] = g[k];
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int d = nb * kBlk;
+    const int64_t warps = int64_t(gridDim.x) * (blockDim.x / 32);
+    for (int64_t r = int64_t(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32; r < M; r += warps) {
+        const uint4 *hrow = h + r * nb * 4;
+        // ---- pass 1: row statistics
+        Welford w = {0.0f, 0.0f, 0.0f};
+        for (int j = lane; j < nb; j += 32) {
+            uint4 raw[4];
+            load_block_nc(hrow, j, raw);
+            float2 p[16];
+            unpack_pairs(raw, p);
+            float2 s2 = p[0];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int i = 4 * q4 + e;
-                const float2 t = __fmul2_rn(__fadd2_rn(p[i], nmu), iv);
-                p[i] = __ffma2_rn(t, make_float2(1.0f + g_lo[e], 1.0f + g_hi[e]), make_float2(b_lo[e], b_hi[e]));
+            for (int i = 1; i < 16; ++i) s2 = __fadd2_rn(s2, p[i]);
+            const float bmean = (s2.x + s2.y) * (1.0f / 32.0f);
+            const float2 nm = make_float2(-bmean, -bmean);
+            float2 q2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float2 t = __fadd2_rn(p[i], nm);
+                q2 = __ffma2_rn(t, t, q2);
             }
+            w = welford_merge(w, Welford{32.0f, bmean, q2.x + q2.y});
         }
-        if (fast) {
-            kq_fast_apply_c(p, st);
-        } else {   // rare: the factors are reloaded (L1) rather than kept live
-            float4 g[5];
-            load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
-            kq_direct_apply(p, g);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            Welford o;
+            o.n = __shfl_xor_sync(0xffffffffu, w.n, off);
+            o.mean = __shfl_xor_sync(0xffffffffu, w.mean, off);
+            o.m2 = __shfl_xor_sync(0xffffffffu, w.m2, off);
+            w = welford_merge(w, o);
         }
-        kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+        const float mu = w.mean;
+        const float inv = 1.0f / sqrtf(w.m2 / float(d) + eps);
+        // ---- pass 2: normalise, modulate, transform, quantize
+        const int64_t b = r / rows_per;
+        const float2 nmu = make_float2(-mu, -mu), iv = make_float2(inv, inv);
+        for (int j = lane; j < nb; j += 32) {
+            uint4 raw[4];
+            load_block_nc(hrow, j, raw);
+            float2 p[16];
+            unpack_pairs(raw, p);
+            const float4 *gp = reinterpret_cast<const float4 *>(gamma + b * d + j * kBlk);
+            const float4 *bp = reinterpret_cast<const float4 *>(beta + b * d + j * kBlk);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 ga = __ldg(gp + q4), gb = __ldg(gp + q4 + 4);
+                const float4 ba = __ldg(bp + q4), bb = __ldg(bp + q4 + 4);
+                const float g_lo[4] = {ga.x, ga.y, ga.z, ga.w}, g_hi[4] = {gb.x, gb.y, gb.z, gb.w};
+                const float b_lo[4] = {ba.x, ba.y, ba.z, ba.w}, b_hi[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = 4 * q4 + e;
+                    const float2 t = __fmul2_rn(__fadd2_rn(p[i], nmu), iv);
+                    p[i] = __ffma2_rn(t, make_float2(1.0f + g_lo[e], 1.0f + g_hi[e]), make_float2(b_lo[e], b_hi[e]));
+                }
+            }
+            const float4 *eq = reinterpret_cast<const float4 *>(tab + j * kNormSlot);
+            const float4 c4q = eq[10];
+            if (c4q.z != 0.0f) {
+                const float4 c01 = eq[8], c23 = eq[9];
+                unit_stage2<1>(p, bcast(c01.x), bcast(c01.y));
+                unit_stage2<2>(p, bcast(c01.z), bcast(c01.w));
+                unit_stage2<4>(p, bcast(c23.x), bcast(c23.y));
+                unit_stage2<8>(p, bcast(c23.z), bcast(c23.w));
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 dd = eq[q];   // (D_2q, D_2q+16, D_2q+1, D_2q+17)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int i = 2 * q + h2;
+                        const float lo = p[i].x, hi = p[i].y;
+                        const float2 dp = h2 ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y);
+                        p[i] = __ffma2_rn(make_float2(fmaf(c4q.x, hi, lo), fmaf(c4q.y, lo, hi)), dp, plus_zero2());
+                    }
+                }
+            } else {
+                float4 g[5];
+#pragma unroll
+                for (int k = 0; k < 5; ++k) g[k] = eq[11 + k];
+                kq_direct_apply(p, g);
+            }
+            kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+        }
     }
 }
 
@@ -1187,7 +1352,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 // per SM (occupancy query, cached per device and kernel).
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
-    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kNumKernels
+    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1410,8 +1575,30 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
     if (variant == 0) variant = kDefaultVariant;
-    if (variant < 1 || variant > 4)
+    if (variant < 1 || variant > 6)
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    if (variant == 6 && !f32) {
+        const int64_t nb6 = d / kBlk;
+        Geometry geo;
+        auto k = kq_packed2_kernel;
+        if ((rc = launch_pinned(fn, kKqPacked2, k, M, nb6, &geo)) != KQ_OK) return rc;
+        k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
+                                             shared, reinterpret_cast<uint4 *>(codes), scales, M * nb6, int(nb6),
+                                             geo.T);
+        return launch_check(fn);
+    }
+    if (variant == 6) variant = 2;
+    if (variant == 5 && !f32) {
+        const int64_t nb5 = d / kBlk;
+        Geometry geo;
+        auto k = kq_lean_kernel;
+        if ((rc = launch_pinned(fn, kKqLean, k, M, nb5, &geo)) != KQ_OK) return rc;
+        k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
+                                             shared, reinterpret_cast<uint4 *>(codes), scales, M * nb5, int(nb5),
+                                             geo.T);
+        return launch_check(fn);
+    }
+    if (variant == 5) variant = 2;   // the fp32 export: the same arithmetic in variant 2
     if (variant == 4 && M < (int64_t(1) << 31)) {
         const int64_t nb4 = d / kBlk;
         CUtensorMap map;
@@ -1717,25 +1904,30 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, 
         !aligned(beta, 16))
         return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
     const int nb = int(d / kBlk);
-    int R = 256 / nb;
-    if (R < 1) R = 1;
-    int npow = 1;
-    while (npow < nb) npow <<= 1;
-    const int threads = R * nb;
-    const size_t smem = size_t(threads) * sizeof(float);
+    const size_t smem = size_t(nb) * kNormSlot * sizeof(float);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (smem > 48 * 1024 && (dev < 0 || dev >= kMaxDevices || !g_smem_set[kNormKq][dev].load())) {
+        e = cudaFuncSetAttribute(norm_kq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(size_t(512) * kNormSlot * sizeof(float)));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_smem_set[kNormKq][dev].store(1);
+    }
     int sms = 0;
     int rc = sm_count(&sms);
     if (rc != KQ_OK) return rc;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel, threads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel, kThreads, smem);
     if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
     if (per_sm < 1) per_sm = 1;
-    const int64_t groups = (M + R - 1) / R;
+    const int64_t warps_needed = M;
     int64_t grid = int64_t(sms) * per_sm;
-    if (grid > groups) grid = groups;
-    norm_kq_kernel<<<unsigned(grid), threads, smem, stream>>>(
+    const int64_t need = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
+    if (grid > need) grid = need;
+    norm_kq_kernel<<<unsigned(grid), kThreads, smem, stream>>>(
         static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
-        reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb, R, npow);
+        reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb);
     return launch_check(fn);
 }
 
