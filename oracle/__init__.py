@@ -61,6 +61,16 @@ def lib():
         L.oracle_kq_inverse.restype = ci
         L.oracle_norm_kq.argtypes = [p, p, p, i64, ctypes.c_double, p, ci, i64, i64, p, p, p, p]
         L.oracle_norm_kq.restype = ci
+        L.oracle_sf_offset.argtypes = [i64, i64, i64]
+        L.oracle_sf_offset.restype = i64
+        L.oracle_sf_bytes.argtypes = [i64, i64]
+        L.oracle_sf_bytes.restype = i64
+        L.oracle_scales_to_sf.argtypes = [p, i64, i64, p]
+        L.oracle_scales_to_sf.restype = ci
+        L.oracle_mx_quantize_f32.argtypes = [p, i64, i64, p, p]
+        L.oracle_mx_quantize_f32.restype = ci
+        L.oracle_mxf4_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
+        L.oracle_mxf4_gemm.restype = ci
         _lib = L
     return _lib
 
@@ -282,3 +292,68 @@ def norm_kq(h_bf16, gamma, beta, eps, factors, shared=False, want=("codes",)):
     if ab is not None:
         out["absb"] = ab
     return out
+
+
+def sf_offset(r: int, j: int, nb: int) -> int:
+    """Byte offset of the scale (row r, block column j) in the scale-factor layout."""
+    return int(lib().oracle_sf_offset(r, j, nb))
+
+
+def sf_bytes(rows: int, nb: int) -> int:
+    """Size of a scale-factor-layout buffer for rows x nb scales (whole 512-byte units)."""
+    return int(lib().oracle_sf_bytes(rows, nb))
+
+
+def scales_to_sf(scales, fill=None):
+    """Row-major scales [rows, nb] -> scale-factor layout (uint8, sf_bytes long).
+
+    Entries the layout leaves undefined hold `fill` (default: 0xFF, so a test
+    that reads them by mistake sees NaN scales); the pad of an odd nb is 0x00.
+    """
+    sc = _c(scales, np.uint8)
+    rows, nb = sc.shape
+    out = np.full(sf_bytes(rows, nb), 0xFF if fill is None else fill, np.uint8)
+    _check(lib().oracle_scales_to_sf(_ptr(sc), rows, nb, _ptr(out)), "scales_to_sf")
+    return out
+
+
+def sf_defined_mask(rows: int, nb: int):
+    """Boolean mask over an SF buffer: the bytes scales_to_sf defines."""
+    mask = np.zeros(sf_bytes(rows, nb), bool)
+    r = np.arange(rows)[:, None]
+    cols = nb + 1 if nb % 2 else nb
+    j = np.arange(cols)[None, :]
+    ka = (nb + 3) // 4
+    off = ((r // 128) * ka + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (j % 4)
+    mask[off.ravel()] = True
+    return mask
+
+
+def mx_quantize_f32(x):
+    """Plain MXFP4 quantizer on fp32 input: (codes [M, d/2], scales [M, d/32])."""
+    xv = _c(x, np.float32)
+    M, d = _shape(xv)
+    codes = np.empty((M, d // 2), np.uint8)
+    scales = np.empty((M, d // 32), np.uint8)
+    _check(lib().oracle_mx_quantize_f32(_ptr(xv), M, d, _ptr(codes), _ptr(scales)), "mx_quantize_f32")
+    return codes, scales
+
+
+def mxf4_gemm(codes_a, scales_a, codes_b, scales_b, rows=None, want_absbound=False):
+    """D = A B^T over decoded MXFP4 operands, in double (kq_oracle.c R10).
+
+    codes_a [M, K/2], scales_a [M, K/32] (row-major), likewise B [N, ...].
+    `rows` restricts the output to those rows of A (sampled checks).
+    """
+    ca, sa = _c(codes_a, np.uint8), _c(scales_a, np.uint8)
+    cb, sb = _c(codes_b, np.uint8), _c(scales_b, np.uint8)
+    M, K = ca.shape[0], ca.shape[1] * 2
+    N = cb.shape[0]
+    assert cb.shape[1] * 2 == K and sa.shape == (M, K // 32) and sb.shape == (N, K // 32)
+    ms = None if rows is None else _c(rows, np.int64)
+    nm = M if ms is None else ms.size
+    D = np.empty((nm, N), np.float64)
+    ab = np.empty((nm, N), np.float64) if want_absbound else None
+    _check(lib().oracle_mxf4_gemm(_ptr(ca), _ptr(sa), _ptr(cb), _ptr(sb), _ptr(ms), nm, M, N, K, _ptr(D), _ptr(ab)),
+           "mxf4_gemm")
+    return (D, ab) if want_absbound else D

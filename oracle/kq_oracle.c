@@ -29,6 +29,11 @@
  *              2^(floor(log2(amax)) - emax_elem) with emax_elem = 2 for E2M1,
  *              stored as E8M0 (biased by 127); elements FP4 E2M1 with values
  *              {0, 0.5, 1, 1.5, 2, 3, 4, 6}, round-to-nearest-even, saturating.
+ *   [SF]       NVIDIA PTX ISA, tcgen05 block-scaled MMA, the scale-factor
+ *              operand: scale bytes of 128 consecutive rows x 4 consecutive
+ *              32-blocks form one 512-byte unit, seen as 32 lanes x 16 bytes;
+ *              lane l holds the rows l, l+32, l+64, l+96 (4 bytes each, in
+ *              that order), each as the 4 blocks in increasing order.
  *
  * Readings taken where the sources are silent (each one is listed in the
  * design notes of the repository):
@@ -54,6 +59,11 @@
  *      per-sample vectors gamma_b, beta_b of length d; rows are grouped by
  *      sample, M / nsamples consecutive rows per sample.  x_mod is not rounded
  *      to bf16 (nothing is written between the two steps).
+ *   R10 The W4A4 linear layer (the step after the quantizer, [KQ-abs]: both
+ *      operands in MXFP4) computes D[m][n] = sum_k a[m][k] b[n][k] with a and b
+ *      the decoded MXFP4 values of X T^T and W T^-1 ([KQ-Eq4]); D is exact in
+ *      double here.  Its scale bytes may be stored in the scale-factor layout
+ *      of the block-scaled tensor-core MMA ([SF] below).
  *   R8 The fixed-Hadamard baseline of block size H (a power of two, 32 <= H,
  *      H | d) is the orthonormal Sylvester transform H_H / sqrt(H) on every
  *      H consecutive channels, followed by the same MX quantizer (blocks of
@@ -611,5 +621,89 @@ int oracle_norm_kq(const uint16_t *h, const float *gamma, const float *beta, int
         free(xm);
     }
     free(K);
+    return 0;
+}
+
+/* [SF] byte offset of the scale of row r, block column j, for a matrix with
+ * nb block columns: 512-byte units ordered row-unit major, the ceil(nb/4)
+ * units of one 128-row group consecutive; inside a unit as stated above. */
+int64_t oracle_sf_offset(int64_t r, int64_t j, int64_t nb)
+{
+    int64_t ka = (nb + 3) / 4;
+    int64_t unit = (r / 128) * ka + j / 4;
+    int64_t lane = r % 32, group = (r % 128) / 32;
+    return unit * 512 + lane * 16 + group * 4 + (j % 4);
+}
+
+int64_t oracle_sf_bytes(int64_t rows, int64_t nb)
+{
+    return ((rows + 127) / 128) * ((nb + 3) / 4) * 512;
+}
+
+/* Row-major scales [rows][nb] -> [SF] layout.  With nb odd the byte of block
+ * column nb (padding inside the last unit) is set to 0x00 (2^-127, finite):
+ * a K=64 step of the MMA reads two consecutive block columns, and the last
+ * one then pairs the real column nb-1 with this pad.  Other padding bytes
+ * are left as they are. */
+int oracle_scales_to_sf(const uint8_t *scales, int64_t rows, int64_t nb, uint8_t *sf)
+{
+    if (rows < 0 || nb <= 0) return -2;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < nb; ++j) sf[oracle_sf_offset(r, j, nb)] = scales[r * nb + j];
+        if (nb & 1) sf[oracle_sf_offset(r, nb, nb)] = 0x00;
+    }
+    return 0;
+}
+
+/* [OCP-MX] the plain MXFP4 quantizer on fp32 input (the folded weights
+ * W T^-1 of [KQ-Eq4] are fp32). */
+int oracle_mx_quantize_f32(const float *x, int64_t M, int64_t d, uint8_t *codes, uint8_t *scales)
+{
+    if (d % BLK != 0 || M < 0) return -2;
+    int64_t nb = d / BLK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t j = 0; j < nb; ++j)
+            oracle_mx_block(x + r * d + j * BLK, codes + r * (d / 2) + j * (BLK / 2), scales + r * nb + j);
+    return 0;
+}
+
+/* One decoded MXFP4 element (R5 nibble order, [OCP-MX] value), in double. */
+static double mx_value(const uint8_t *codes, const uint8_t *scales, int64_t r, int64_t k, int64_t K)
+{
+    uint8_t byte = codes[r * (K / 2) + k / 2];
+    uint8_t c = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+    double v = E2M1_GRID[c & 7];
+    if (c & 8) v = -v;
+    uint8_t sb = scales[r * (K / BLK) + k / BLK];
+    return sb == 0xFF ? NAN : ldexp(v, (int)sb - 127);
+}
+
+/* R10: D[m][n] = sum_k a[m][k] b[n][k] over the decoded operands (row-major
+ * scales), summed in double.  Each product is exact (E2M1 values carry at
+ * most 2 significant bits, scales are powers of two); the double sum rounds
+ * far below any fp32 accumulation.  If absd is not NULL it receives
+ * sum_k |a[m][k] b[n][k]| for tolerances.  Rows ms[0..nm) of A only when ms
+ * is not NULL (sampled checks); D and absd are then [nm][N]. */
+int oracle_mxf4_gemm(const uint8_t *ca, const uint8_t *sa, const uint8_t *cb, const uint8_t *sbb,
+                     const int64_t *ms, int64_t nm, int64_t M, int64_t N, int64_t K, double *D, double *absd)
+{
+    if (K <= 0 || K % BLK != 0 || M < 0 || N < 0) return -2;
+    int64_t rows = ms ? nm : M;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < rows; ++i) {
+        int64_t m = ms ? ms[i] : i;
+        if (m < 0 || m >= M) continue;
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = mx_value(ca, sa, m, k, K) * mx_value(cb, sbb, n, k, K);
+                acc += p;
+                aacc += fabs(p);
+            }
+            D[i * N + n] = acc;
+            if (absd) absd[i * N + n] = aacc;
+        }
+    }
     return 0;
 }
