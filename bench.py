@@ -628,6 +628,82 @@ def kernel_mode(args):
                       "frac_of_peak": round(gbs / peak, 4), "peak": peak, "peak_source": src}), flush=True)
 
 
+def gemm_mode(args):
+    """The W4A4 linear layer on MXFP4 operands (tcgen05 block-scaled MMA) at
+    M x N x K, alone and chained after the KroQuant quantizer that feeds it.
+
+    Operands rotate over enough sets that each launch reads A and writes D
+    outside L2 (>= 3x L2 between reuses).  The roofline is the tensor pipe:
+    2 M N K flops against the measured bf16 GEMM peak x 4, the nominal
+    fp4 / bf16 dense ratio (9 / 2.25 PFLOP/s).
+    """
+    import torch
+
+    import w4a4_mxfp4_post_b200 as kq
+    from w4a4_mxfp4_post_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda:0")
+    M, N, K = (int(t) for t in args.shape.lower().split("x"))
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    x = synth.activation("pixart", M, K, 5)
+    F = synth.factors(K // 32, 5)
+    W = torch.from_numpy(synth.weights(N, K, 5)).to(dev)
+    Wf = kq.kq_fold_weights(W, torch.from_numpy(F).to(dev))
+    bc, bsf = kq.mx_quantize_f32(Wf, sf_layout=True)
+    set_bytes = M * K * 2 + M * K // 2 + kq.kq_sf_bytes(M, K) + M * N * 2
+    nsets = max(2, min(64, math.ceil(3 * l2 / set_bytes)))
+    Fd = torch.from_numpy(F).to(dev)
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16).clone() for _ in range(nsets)]
+    acs, asfs = zip(*[kq.kq_quantize_sf(xs[i], Fd) for i in range(nsets)])
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def run(kind, n):
+        for i in range(n):
+            k = i % nsets
+            if kind == "chain":
+                kq.kq_quantize_sf(xs[k], Fd, out_codes=acs[k], out_sf=asfs[k], stream=stream)
+            kq.mxf4_gemm(acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
+
+    res = {}
+    for kind in ("gemm", "chain"):
+        with torch.cuda.stream(stream):
+            run(kind, max(3, args.warmup))
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run(kind, args.launches)
+        t_end = time.perf_counter() + SPINUP_S
+        while time.perf_counter() < t_end:
+            g.replay()
+            stream.synchronize()
+        reps = max(1, int(0.3 / max(1e-6, _replay_seconds(g, stream))))
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            t1.record(stream)
+        stream.synchronize()
+        res[kind] = 1e3 * t0.elapsed_time(t1) / (args.launches * reps)
+    flops = 2.0 * M * N * K
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            bf16 = float(json.load(fh)["bf16_tflops"])
+        src = "measured bf16 burst (MEASURED_PEAKS.json) x 4 (nominal fp4/bf16 dense ratio)"
+    except Exception:
+        bf16, src = 1590.0, "fallback bf16 1.59 PFLOP/s x 4 (nominal fp4/bf16 dense ratio)"
+    peak = 4.0 * bf16
+    tflops = flops / (res["gemm"] * 1e-6) / 1e12
+    out_bytes = M * N * 2 + M * K // 2 + N * K // 2
+    print(json.dumps({"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets, "gemm_us": round(res["gemm"], 3),
+                      "chain_us": round(res["chain"], 3), "tflops": round(tflops, 1), "peak_tflops": peak,
+                      "frac_of_peak": round(tflops / peak, 4), "peak_source": src,
+                      "hbm_gbs_min_bytes": round(out_bytes / (res["gemm"] * 1e-6) / 1e9, 1)}), flush=True)
+
+
 def sweep_mode(args):
     """Bandwidth sweep: every quantizer at every (M, d) of the sweep workload."""
     import torch
@@ -745,13 +821,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the cpu_baseline block")
     ap.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the reference arm")
     ap.add_argument("--json-out", default="")
-    ap.add_argument("--mode", choices=["step", "kernel", "sweep", "sqnr"], default="step",
+    ap.add_argument("--mode", choices=["step", "kernel", "sweep", "sqnr", "gemm"], default="step",
                     help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes; "
                          "sqnr: quantisation-error proxy per method")
     ap.add_argument("--kernel", default="kq",
                     help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H> or norm_kq")
     ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
-    ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD")
+    ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD; gemm mode: MxNxK")
     ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")
     ap.add_argument("--no-graph", action="store_true", help="kernel mode: eager launches")
     ap.add_argument("--launches", type=int, default=100, help="kernel / sweep mode: timed launches")
@@ -762,6 +838,8 @@ def main():
         return sweep_mode(args)
     if args.mode == "sqnr":
         return sqnr_mode(args)
+    if args.mode == "gemm":
+        return gemm_mode(args)
     if args.steps < 1 or args.warmup < 3:
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
 

@@ -154,6 +154,63 @@ int kq_inverse_f32(const float *y, const float *factors, int shared,
 int mx_dequantize(const uint8_t *codes, const uint8_t *scales, float *out,
                   int64_t M, int64_t d, cudaStream_t stream);
 
+/* ---- W4A4 consumer: the linear layer on the quantized operands ----------
+ *
+ * Scale-factor layout ("sf"): the E8M0 scales of a [rows][d] MXFP4 matrix as
+ * the block-scaled tensor-core MMA reads them (NVIDIA PTX ISA, tcgen05.mma
+ * block scaling, the scale-factor operand).  With nb = d/32 block columns,
+ * the scales of 128 consecutive rows x 4 consecutive block columns form one
+ * 512-byte unit; the scale of row r, block column j sits at byte
+ *   ((r / 128) * ceil(nb / 4) + j / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4.
+ * A buffer holds kq_sf_bytes(rows, d) bytes (whole units: rows rounded up to
+ * 128, block columns to 4).  The writers below fill every real scale and,
+ * when nb is odd, the byte of block column nb (set to 0x00): mxf4_gemm reads
+ * it beside column nb-1.  Other padding bytes are left untouched and are
+ * never read for an output element. */
+#define KQ_SCALES_ROWMAJOR 0
+#define KQ_SCALES_SF 1
+
+/* Bytes of a scale-factor-layout buffer for a [rows][d] matrix; -1 for
+ * rows < 0 or d not a positive multiple of 32.  Host only, no CUDA call. */
+int64_t kq_sf_bytes(int64_t rows, int64_t d);
+
+/* kq_quantize (shared != 0: kq_quantize_shared) with the scales written in
+ * the scale-factor layout to out_sf (kq_sf_bytes(M, d) bytes, 1-byte
+ * aligned); codes exactly as kq_quantize. */
+int kq_quantize_sf(const void *act_bf16, const float *factors, int shared,
+                   uint8_t *out_codes, uint8_t *out_sf,
+                   int64_t M, int64_t d, cudaStream_t stream);
+
+/* The plain MXFP4 quantizer on float32 input x [M][d] (for the folded weights
+ * W T^-1 from kq_fold_weights, which are fp32): the block rule above on the
+ * fp32 values.  scale_layout KQ_SCALES_ROWMAJOR writes out_scales [M][d/32],
+ * KQ_SCALES_SF the scale-factor layout (kq_sf_bytes(M, d) bytes); any other
+ * value -> KQ_ERR_SHAPE.  x and out_codes 16-byte aligned. */
+int mx_quantize_f32(const float *x, uint8_t *out_codes, uint8_t *out_scales,
+                    int scale_layout, int64_t M, int64_t d, cudaStream_t stream);
+
+/* Row-major scales [M][d/32] (from any quantizer here) -> the scale-factor
+ * layout (kq_sf_bytes(M, d) bytes; the buffers may not overlap). */
+int mx_scales_to_sf(const uint8_t *scales, uint8_t *out_sf,
+                    int64_t M, int64_t d, cudaStream_t stream);
+
+/* The W4A4 linear layer ("KroQuant ...", abstract: W4A4 at MXFP4; section
+ * 3.2, Eq. (4): the inverse folded into the weights, so that
+ * X W^T = (X T^T)(W T^-1)^T):
+ *   out[m][n] = sum_k a[m][k] * b[n][k]
+ * with a the decoded MXFP4 activation (a_codes [M][K/2], a_sf its scales in
+ * the scale-factor layout, kq_sf_bytes(M, K) bytes) and b the decoded MXFP4
+ * weight (b_codes [N][K/2], b_sf, kq_sf_bytes(N, K) bytes).  Products are
+ * exact and accumulate in fp32 on the tensor cores (tcgen05 block-scaled
+ * MMA); out is bf16 (out_f32 == 0, rounded to nearest even) or float32,
+ * [M][N] row-major.  Needs K a positive multiple of 32, N a multiple of 8,
+ * M, N, K < 2^31; every pointer 16-byte aligned; out may not overlap the
+ * inputs.  A scale byte 0xFF (NaN) makes the outputs it reaches NaN. */
+int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf,
+              const uint8_t *b_codes, const uint8_t *b_sf,
+              void *out, int out_f32, int64_t M, int64_t N, int64_t K,
+              cudaStream_t stream);
+
 /* Test export: the fp32 transform y = T x (float32 [M][d]) exactly as the
  * quantizer computes it before the amax, for the transform-accuracy check. */
 int kq_transform_f32(const void *act_bf16, const float *factors, int shared,

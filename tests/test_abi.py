@@ -149,6 +149,39 @@ def test_norm_inverse_dequant_argument_errors(L):
     assert L.mx_dequantize(None, None, None, 0, 64, None) == 0
 
 
+def test_w4a4_argument_errors(L):
+    L.kq_sf_bytes.restype = ctypes.c_int64
+    L.kq_sf_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    assert L.kq_sf_bytes(300, 2240) == 3 * 18 * 512
+    assert L.kq_sf_bytes(0, 64) == 0
+    assert L.kq_sf_bytes(4, 40) == -1
+    # kq_quantize_sf
+    assert L.kq_quantize_sf(P(16), P(16), 0, P(16), P(16), 4, 40, None) == -2
+    assert L.kq_quantize_sf(P(16), None, 0, P(16), P(16), 4, 64, None) == -1
+    assert L.kq_quantize_sf(P(8), P(16), 0, P(16), P(16), 4, 64, None) == -3
+    assert L.kq_quantize_sf(None, None, 0, None, None, 0, 64, None) == 0
+    # mx_quantize_f32
+    assert L.mx_quantize_f32(P(16), P(16), P(16), 2, 4, 64, None) == -2
+    assert L.mx_quantize_f32(P(16), P(16), P(16), 0, 4, 48, None) == -2
+    assert L.mx_quantize_f32(P(16), None, P(16), 1, 4, 64, None) == -1
+    assert L.mx_quantize_f32(P(16), P(8), P(16), 1, 4, 64, None) == -3
+    assert L.mx_quantize_f32(None, None, None, 1, 0, 64, None) == 0
+    # mx_scales_to_sf
+    assert L.mx_scales_to_sf(P(16), P(16), -1, 64, None) == -2
+    assert L.mx_scales_to_sf(None, P(16), 4, 64, None) == -1
+    assert L.mx_scales_to_sf(None, None, 0, 64, None) == 0
+    # mxf4_gemm: a_codes, a_sf, b_codes, b_sf, out, out_f32, M, N, K, stream
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(16), 0, 4, 8, 48, None) == -2      # K % 32
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(16), 0, 4, 12, 64, None) == -2     # N % 8
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(16), 0, 4, 8, 0, None) == -2       # K <= 0
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(16), 0, 1 << 31, 8, 64, None) == -2
+    assert L.mxf4_gemm(P(16), None, P(16), P(16), P(16), 0, 4, 8, 64, None) == -1
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(8), P(16), 0, 4, 8, 64, None) == -3
+    assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(4), 1, 4, 8, 64, None) == -3
+    assert L.mxf4_gemm(None, None, None, None, None, 0, 0, 8, 64, None) == 0
+    assert L.mxf4_gemm(None, None, None, None, None, 0, 4, 0, 64, None) == 0
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
 

@@ -14,6 +14,12 @@ every function raises if the library is missing or returns an error.
     codes, scales = mx_quantize(act)
     W_folded      = kq_fold_weights(W, factors, shared=False)
     y             = kq_transform_f32(act, factors, shared=False)
+
+W4A4 consumer (scales in the tensor core's scale-factor layout):
+
+    codes, sf     = kq_quantize_sf(act, factors)         # [M, d/2], [kq_sf_bytes(M, d)] uint8
+    wcodes, wsf   = mx_quantize_f32(W_folded, sf_layout=True)
+    out           = mxf4_gemm(codes, sf, wcodes, wsf)    # bf16 [M, N] = X W^T, W4A4
 """
 from __future__ import annotations
 
@@ -26,11 +32,14 @@ __all__ = [
     "mx_quantize", "kq_fold_weights", "kq_transform_f32", "kq_last_error", "kq_abi_version",
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
     "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize", "kq_inverse_f32", "mx_dequantize", "norm_kq_quantize",
+    "KQ_SCALES_ROWMAJOR", "KQ_SCALES_SF", "kq_sf_bytes", "kq_quantize_sf", "mx_quantize_f32", "mx_scales_to_sf",
+    "mxf4_gemm",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
 
 KQ_OK, KQ_ERR_NULL, KQ_ERR_SHAPE, KQ_ERR_ALIGN, KQ_ERR_CUDA, KQ_ERR_VARIANT = 0, -1, -2, -3, -4, -5
+KQ_SCALES_ROWMAJOR, KQ_SCALES_SF = 0, 1
 
 # Entry points and their argument types (p = pointer, i = int, q = int64).
 _SIGS = {
@@ -49,6 +58,10 @@ _SIGS = {
     "fwht_quantize": "pqppqqp",
     "kq_inverse_f32": "ppipqqp",
     "mx_dequantize": "pppqqp",
+    "kq_quantize_sf": "ppippqqp",
+    "mx_quantize_f32": "pppiqqp",
+    "mx_scales_to_sf": "ppqqp",
+    "mxf4_gemm": "pppppiqqqp",
 }
 
 _lib = None
@@ -86,6 +99,8 @@ def lib() -> ctypes.CDLL:
                                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                                 ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
         L.norm_kq_quantize.restype = ctypes.c_int
+        L.kq_sf_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+        L.kq_sf_bytes.restype = ctypes.c_int64
         _lib = L
     return _lib
 
@@ -353,4 +368,99 @@ def kq_transform_f32(act, factors, shared=False, out=None, stream=None):
         out = torch.empty((M, d), dtype=torch.float32, device=act.device)
     _need(out, "out", torch.float32, act.device, (M, d))
     _call("kq_transform_f32", _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d, _stream(stream))
+    return out
+
+
+def kq_sf_bytes(rows: int, d: int) -> int:
+    """Bytes of a scale-factor-layout buffer for a [rows, d] MXFP4 matrix."""
+    n = lib().kq_sf_bytes(int(rows), int(d))
+    if n < 0:
+        raise ValueError(f"kq_sf_bytes: bad shape rows={rows}, d={d}")
+    return n
+
+
+def _sf_out(out_sf, rows, d, device):
+    torch = _torch()
+    n = kq_sf_bytes(rows, d)
+    if out_sf is None:
+        out_sf = torch.empty((n,), dtype=torch.uint8, device=device)
+    _need(out_sf, "out_sf", torch.uint8, device, (n,))
+    return out_sf
+
+
+def kq_quantize_sf(act, factors, shared=False, out_codes=None, out_sf=None, stream=None):
+    """kq_quantize with the scales in the tensor core's scale-factor layout (1-D uint8)."""
+    torch = _torch()
+    M, d = _act(act)
+    _factors(factors, d, shared, act.device)
+    if out_codes is None:
+        out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=act.device)
+    _need(out_codes, "out_codes", torch.uint8, act.device, (M, d // 2))
+    out_sf = _sf_out(out_sf, M, d, act.device)
+    _call("kq_quantize_sf", _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M, d,
+          _stream(stream))
+    return out_codes, out_sf
+
+
+def mx_quantize_f32(x, sf_layout=False, out_codes=None, out_scales=None, stream=None):
+    """Plain MXFP4 quantizer on fp32 input [M, d] (the folded weights).
+
+    Scales row-major [M, d/32], or with sf_layout=True in the scale-factor layout (1-D).
+    """
+    torch = _torch()
+    _need(x, "x", torch.float32)
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [M, d]")
+    M, d = x.shape
+    if out_codes is None:
+        out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    _need(out_codes, "out_codes", torch.uint8, x.device, (M, d // 2))
+    if sf_layout:
+        out_scales = _sf_out(out_scales, M, d, x.device)
+    else:
+        if out_scales is None:
+            out_scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
+        _need(out_scales, "out_scales", torch.uint8, x.device, (M, d // 32))
+    _call("mx_quantize_f32", _ptr(x), _ptr(out_codes), _ptr(out_scales),
+          KQ_SCALES_SF if sf_layout else KQ_SCALES_ROWMAJOR, M, d, _stream(stream))
+    return out_codes, out_scales
+
+
+def mx_scales_to_sf(scales, out_sf=None, stream=None):
+    """Row-major scales [M, d/32] -> the scale-factor layout (1-D uint8)."""
+    torch = _torch()
+    _need(scales, "scales", torch.uint8)
+    if scales.dim() != 2:
+        raise ValueError("scales must be 2-D [M, d/32]")
+    M, d = scales.shape[0], scales.shape[1] * 32
+    out_sf = _sf_out(out_sf, M, d, scales.device)
+    _call("mx_scales_to_sf", _ptr(scales), _ptr(out_sf), M, d, _stream(stream))
+    return out_sf
+
+
+def mxf4_gemm(a_codes, a_sf, b_codes, b_sf, out=None, out_dtype=None, stream=None):
+    """W4A4 linear layer: out[m, n] = sum_k a[m, k] b[n, k] over decoded MXFP4 operands.
+
+    a_codes [M, K/2], b_codes [N, K/2] uint8; a_sf, b_sf their scales in the
+    scale-factor layout; out bf16 (default) or float32 [M, N].
+    """
+    torch = _torch()
+    _need(a_codes, "a_codes", torch.uint8)
+    if a_codes.dim() != 2 or b_codes.dim() != 2:
+        raise ValueError("a_codes and b_codes must be 2-D")
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    dev = a_codes.device
+    _need(b_codes, "b_codes", torch.uint8, dev)
+    N = b_codes.shape[0]
+    if b_codes.shape[1] * 2 != K:
+        raise ValueError(f"b_codes must be [N, {K // 2}], got {tuple(b_codes.shape)}")
+    _need(a_sf, "a_sf", torch.uint8, dev, (kq_sf_bytes(M, K),))
+    _need(b_sf, "b_sf", torch.uint8, dev, (kq_sf_bytes(N, K),))
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=dev)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, dev, (M, N))
+    _call("mxf4_gemm", _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
+          int(out.dtype == torch.float32), M, N, K, _stream(stream))
     return out

@@ -411,72 +411,6 @@ __device__ __forceinline__ void kq_fast_apply(float2 (&p)[16], const KqFast &st)
     }
 }
 
-// Compact column state (used where registers are scarce: the fused
-// normalisation kernel).  D = (x)_k diag(g00_k, g11_k) is kept factored as
-// diag_G1 (x) D_rest: the pair (g00, g11) of G1 (index
-// bit 4, the two halves of every register pair) and the 16 values of D_rest
-// (bits 0..3), which multiply both halves of pair i alike.  All coefficients
-// are then scalars used as broadcast operands of the packed instructions,
-// 28 registers in all, at the cost of one more packed multiply per pair than
-// the paired form below.
-struct KqFastC {
-    float Dr[16];             // D_rest_i, i = 0..15
-    float d40, d41;           // diagonal of G1
-    float B[4], C[4];         // stages on bits 0..3 (G5, G4, G3, G2)
-    float b4, c4;             // stage on bit 4 (G1)
-};
-
-__device__ __forceinline__ bool kq_fast_setup_c(const float4 (&g)[5], KqFastC &st)
-{
-    float d0[5], d1[5], bb[5], cc[5];
-    bool fast = true;
-#pragma unroll
-    for (int k = 0; k < 5; ++k) fast &= unit_split(g[k], d0[k], d1[k], bb[k], cc[k]);
-    // D_rest_i = prod over bits 0..3 of (bit b of i ? g11 : g00) of G_(5-b)
-    float dd[16];
-    dd[0] = 1.0f;
-#pragma unroll
-    for (int bit = 0; bit < 4; ++bit) {
-        const int k = 4 - bit;
-#pragma unroll
-        for (int i = 0; i < (1 << bit); ++i) {
-            dd[i + (1 << bit)] = dd[i] * d1[k];
-            dd[i] = dd[i] * d0[k];
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) st.Dr[i] = dd[i];
-    st.d40 = d0[0];
-    st.d41 = d1[0];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        st.B[b] = bb[4 - b];
-        st.C[b] = cc[4 - b];
-    }
-    st.b4 = bb[0];
-    st.c4 = cc[0];
-    return fast;
-}
-
-__device__ __forceinline__ void kq_fast_apply_c(float2 (&p)[16], const KqFastC &st)
-{
-    unit_stage2<1>(p, bcast(st.B[0]), bcast(st.C[0]));
-    unit_stage2<2>(p, bcast(st.B[1]), bcast(st.C[1]));
-    unit_stage2<4>(p, bcast(st.B[2]), bcast(st.C[2]));
-    unit_stage2<8>(p, bcast(st.B[3]), bcast(st.C[3]));
-    // stage on bit 4, then D = diag_G1 (x) D_rest.  The last multiply is an FMA
-    // with +0: the same value, except that an exact zero comes out +0 whatever
-    // the signs (as a sum of products that cancels exactly does in
-    // round-to-nearest).
-    const float2 d4 = make_float2(st.d40, st.d41);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float lo = p[i].x, hi = p[i].y;
-        const float2 t = __fmul2_rn(make_float2(fmaf(st.b4, hi, lo), fmaf(st.c4, lo, hi)), d4);
-        p[i] = __ffma2_rn(t, bcast(st.Dr[i]), plus_zero2());
-    }
-}
-
 // The direct form, y_lo = g00 lo + g01 hi, y_hi = g10 lo + g11 hi per stage.
 __device__ __forceinline__ void kq_direct_apply(float2 (&p)[16], const float4 (&g)[5])
 {
@@ -513,6 +447,53 @@ __device__ __forceinline__ void kq_emit(float2 (&p)[16], int64_t gi, uint4 *__re
     }
 }
 
+// Scale-factor layout of the block-scaled tensor-core MMA (PTX ISA, tcgen05
+// block scaling, the scale-factor operand): the scales of 128 rows x 4
+// consecutive blocks form one 512-byte unit, 32 lanes x 16 bytes, lane l
+// holding rows l, l+32, l+64, l+96 at bytes 4*((r / 32) % 4), each as its 4
+// blocks in order; units are ordered row-group major (the ceil(nb/4) units of
+// 128 rows are consecutive).  For odd nb the byte of block column nb is
+// written as 0x00 (2^-127): the MMA's last K=64 step reads it beside the real
+// column nb-1, against zero codes, and it must be finite.
+struct SfPos {
+    int64_t row;     // current row (advances by rstep per step of the thread)
+    int64_t rstep;
+    int64_t ka512;   // 512 * ceil(nb / 4): bytes per 128-row group
+    int64_t col;     // column part of the offset: 512 * (j / 4) + j % 4
+    bool pad;        // this thread writes the odd-nb pad byte
+};
+
+__device__ __forceinline__ SfPos sf_pos(int64_t t, int64_t T, int nb)
+{
+    SfPos s;
+    const int j = int(t % nb);
+    s.row = t / nb;
+    s.rstep = T / nb;
+    s.ka512 = int64_t((nb + 3) >> 2) * 512;
+    s.col = int64_t(j >> 2) * 512 + (j & 3);
+    s.pad = (nb & 1) && j == nb - 1;
+    return s;
+}
+
+__device__ __forceinline__ int64_t sf_offset(const SfPos &s)
+{
+    return (s.row >> 7) * s.ka512 + (s.row & 31) * 16 + ((s.row >> 5) & 3) * 4 + s.col;
+}
+
+// Codes as kq_emit; the scale byte at its scale-factor-layout offset.
+__device__ __forceinline__ void kq_emit_sf(float2 (&p)[16], int64_t gi, uint4 *__restrict__ codes,
+                                           uint8_t *__restrict__ sf, SfPos &sp)
+{
+    uint4 c;
+    uint32_t sb;
+    mx_quantize_pairs(p, c, sb);
+    codes[gi] = c;
+    const int64_t off = sf_offset(sp);
+    sf[off] = uint8_t(sb);
+    if (sp.pad) sf[off + 1] = 0;
+    sp.row += sp.rstep;
+}
+
 __device__ __forceinline__ void load_factors(const float4 *__restrict__ factors, int shared, int j, float4 (&g)[5])
 {
     const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
@@ -547,7 +528,9 @@ __device__ __forceinline__ void load_lu(const float *__restrict__ lu, int shared
 // A thread whose column has a factor with |g00| or |g11| outside
 // [2^-16, 2^16] or |b| or |c| above 16 (where U's intermediate values could
 // grow by more than 17^5) runs the direct form instead.
-template <KqOut OUT, bool LU = false>
+// With SF the scales go to the scale-factor layout (requires T a multiple of
+// nb, as the pinned geometry gives).
+template <KqOut OUT, bool LU = false, bool SF = false>
 __global__ void __launch_bounds__(kThreads, 2)
 kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params, int shared,
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
@@ -555,6 +538,8 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
 {
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
+    SfPos sp{};
+    if constexpr (SF) sp = sf_pos(t, T, nb);
     float4 g[5];
     if constexpr (LU)
         load_lu(params, shared, int(t % nb), g);
@@ -574,7 +559,10 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
             float2 p[16];
             unpack_pairs(raw, p);
             kq_fast_apply(p, st);
-            kq_emit<OUT>(p, gi, codes, scales, y_out);
+            if constexpr (SF)
+                kq_emit_sf(p, gi, codes, scales, sp);
+            else
+                kq_emit<OUT>(p, gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
@@ -588,7 +576,10 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
             float2 p[16];
             unpack_pairs(raw, p);
             kq_direct_apply(p, g);
-            kq_emit<OUT>(p, gi, codes, scales, y_out);
+            if constexpr (SF)
+                kq_emit_sf(p, gi, codes, scales, sp);
+            else
+                kq_emit<OUT>(p, gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
@@ -1148,6 +1139,56 @@ mx_dequantize_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict_
     }
 }
 
+// Plain MXFP4 quantizer on fp32 input, for the folded weights W T^-1 of
+// KroQuant section 3.2, Eq. (4) (fp32 after the fold): one 32-block per
+// thread, the same block quantizer as the activation kernels; scales
+// row-major [M][nb] or, with SF, in the scale-factor layout.
+template <bool SF>
+__global__ void __launch_bounds__(kThreads)
+mx_f32_kernel(const float4 *__restrict__ x, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
+              int64_t nblocks, int nb)
+{
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < nblocks; g += stride) {
+        float v[32];
+        const float4 *src = x + g * 8;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 f = __ldg(src + q);
+            v[4 * q] = f.x;
+            v[4 * q + 1] = f.y;
+            v[4 * q + 2] = f.z;
+            v[4 * q + 3] = f.w;
+        }
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_block(v, c, sb);
+        codes[g] = c;
+        if constexpr (SF) {
+            SfPos sp = sf_pos(g, g + 1, nb);   // row g / nb, column g % nb (rstep unused)
+            const int64_t off = sf_offset(sp);
+            scales[off] = uint8_t(sb);
+            if (sp.pad) scales[off + 1] = 0;
+        } else {
+            scales[g] = uint8_t(sb);
+        }
+    }
+}
+
+// Row-major scales [M][nb] -> the scale-factor layout (one byte per thread),
+// with the odd-nb pad byte; lets every quantizer feed the W4A4 product.
+__global__ void __launch_bounds__(kThreads)
+sf_relayout_kernel(const uint8_t *__restrict__ scales, uint8_t *__restrict__ sf, int64_t n, int nb)
+{
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < n; g += stride) {
+        SfPos sp = sf_pos(g, g + 1, nb);
+        const int64_t off = sf_offset(sp);
+        sf[off] = __ldg(scales + g);
+        if (sp.pad) sf[off + 1] = 0;
+    }
+}
+
 // The quantizer fused with the normalisation that produces its input (KroQuant
 // abstract: normalisation layers force the transform online).  For every token
 // row h of a bf16 activation: LayerNorm without affine (mean, biased
@@ -1300,6 +1341,7 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
 }
 
 #include "kq_mma.cuh"
+#include "mxf4_gemm.cuh"
 
 // ---------------------------------------------------------------------------
 // launch geometry
@@ -1352,7 +1394,8 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 // per SM (occupancy query, cached per device and kernel).
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
-    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2, kNumKernels
+    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2,
+    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kGemmBf16, kGemmF32, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1541,6 +1584,40 @@ int mma_prepare(KernelId id, const void *fn)
     }
     return KQ_OK;
 }
+
+int smem_prepare(KernelId id, const void *fn, size_t bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices || !g_smem_set[id][dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_smem_set[id][dev].store(1, std::memory_order_release);
+    }
+    return KQ_OK;
+}
+
+// MXFP4 codes [rows][K/2] as a uint8 matrix read by the W4A4 product: boxes of
+// {128 bytes x box_rows}, 128-byte swizzle, rows and bytes past the matrix
+// read as zero.
+int encode_gemm_map(const void *codes, int64_t rows, int64_t K, int box_rows, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(K / 2)};
+    const cuuint32_t box[2] = {cuuint32_t(gemm::kChunkBytes), cuuint32_t(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
+int64_t sf_bytes_of(int64_t rows, int64_t nb) { return ((rows + 127) / 128) * ((nb + 3) / 4) * 512; }
 
 // Default clock budget of a bounded wait: 2^31 cycles, about a second.
 constexpr long long kWaitBudget = 1LL << 31;
@@ -1928,6 +2005,100 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, 
     norm_kq_kernel<<<unsigned(grid), kThreads, smem, stream>>>(
         static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
         reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb);
+    return launch_check(fn);
+}
+
+int64_t kq_sf_bytes(int64_t rows, int64_t d)
+{
+    if (rows < 0 || d <= 0 || d % kBlk != 0) return -1;
+    return sf_bytes_of(rows, d / kBlk);
+}
+
+int kq_quantize_sf(const void *act_bf16, const float *factors, int shared, uint8_t *out_codes, uint8_t *out_sf,
+                   int64_t M, int64_t d, cudaStream_t stream)
+{
+    const char *fn = "kq_quantize_sf";
+    int rc = check_quant_args(fn, act_bf16, factors, true, out_codes, out_sf, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    Geometry geo;
+    auto k = kq_packed_kernel<KqOut::kCodes, false, true>;
+    if ((rc = launch_pinned(fn, kKqPackedSf, k, M, nb, &geo)) != KQ_OK) return rc;
+    k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16), factors, shared ? 1 : 0,
+                                         reinterpret_cast<uint4 *>(out_codes), out_sf, nullptr, M * nb, int(nb),
+                                         geo.T);
+    return launch_check(fn);
+}
+
+int mx_quantize_f32(const float *x, uint8_t *out_codes, uint8_t *out_scales, int scale_layout, int64_t M, int64_t d,
+                    cudaStream_t stream)
+{
+    const char *fn = "mx_quantize_f32";
+    if (scale_layout != KQ_SCALES_ROWMAJOR && scale_layout != KQ_SCALES_SF)
+        return fail(KQ_ERR_SHAPE, "%s: scale_layout must be KQ_SCALES_ROWMAJOR or KQ_SCALES_SF", fn);
+    int rc = check_quant_args(fn, x, nullptr, false, out_codes, out_scales, M, d);
+    if (rc == 1) return ok();
+    if (rc != KQ_OK) return rc;
+    const int64_t nb = d / kBlk;
+    const int64_t nblocks = M * nb;
+    const bool sf = scale_layout == KQ_SCALES_SF;
+    auto k = sf ? mx_f32_kernel<true> : mx_f32_kernel<false>;
+    int64_t target = 0;
+    if ((rc = resident_threads(sf ? kMxF32Sf : kMxF32, reinterpret_cast<const void *>(k), &target)) != KQ_OK)
+        return rc;
+    const int64_t T = target < nblocks ? target : nblocks;
+    k<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(
+        reinterpret_cast<const float4 *>(x), reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks, int(nb));
+    return launch_check(fn);
+}
+
+int mx_scales_to_sf(const uint8_t *scales, uint8_t *out_sf, int64_t M, int64_t d, cudaStream_t stream)
+{
+    const char *fn = "mx_scales_to_sf";
+    if (M < 0 || d <= 0 || d % kBlk != 0)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32", fn);
+    if (d / kBlk > INT32_MAX || (M > 0 && M > INT64_MAX / d)) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (M == 0) return ok();
+    if (!scales || !out_sf) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    const int64_t n = M * (d / kBlk);
+    int64_t target = 0;
+    int rc = resident_threads(kSfRelayout, reinterpret_cast<const void *>(sf_relayout_kernel), &target);
+    if (rc != KQ_OK) return rc;
+    const int64_t T = target < n ? target : n;
+    sf_relayout_kernel<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(scales, out_sf, n,
+                                                                                          int(d / kBlk));
+    return launch_check(fn);
+}
+
+int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes, const uint8_t *b_sf, void *out,
+              int out_f32, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    const char *fn = "mxf4_gemm";
+    if (M < 0 || N < 0 || K <= 0 || K % kBlk != 0 || N % 8 != 0)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0, N >= 0 a multiple of 8, K a positive multiple of 32 "
+                    "(M=%lld, N=%lld, K=%lld)", fn, (long long)M, (long long)N, (long long)K);
+    if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+        return fail(KQ_ERR_SHAPE, "%s: M, N and K must be below 2^31", fn);
+    if (M == 0 || N == 0) return ok();
+    if (!a_codes || !a_sf || !b_codes || !b_sf || !out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
+        !aligned(out, 16))
+        return fail(KQ_ERR_ALIGN, "%s: every pointer must be 16-byte aligned", fn);
+    CUtensorMap amap, bmap;
+    int rc = encode_gemm_map(a_codes, M, K, gemm::kBM, &amap);
+    if (rc != KQ_OK) return rc;
+    if ((rc = encode_gemm_map(b_codes, N, K, gemm::kBN, &bmap)) != KQ_OK) return rc;
+    const int64_t tiles = ((M + gemm::kBM - 1) / gemm::kBM) * ((N + gemm::kBN - 1) / gemm::kBN);
+    if (tiles >= (int64_t(1) << 31)) return fail(KQ_ERR_SHAPE, "%s: too many output tiles", fn);
+    int sms = 0;
+    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+    const unsigned grid = unsigned(tiles < sms ? tiles : sms);
+    auto k = out_f32 ? gemm::mxf4_gemm_kernel<true> : gemm::mxf4_gemm_kernel<false>;
+    if ((rc = smem_prepare(out_f32 ? kGemmF32 : kGemmBf16, reinterpret_cast<const void *>(k), gemm::kSmem)) != KQ_OK)
+        return rc;
+    k<<<grid, gemm::kThreads, gemm::kSmem, stream>>>(amap, bmap, a_sf, b_sf, out, int(M), int(N), int(K),
+                                                     kWaitBudget);
     return launch_check(fn);
 }
 

@@ -1,0 +1,299 @@
+// mxf4_gemm.cuh -- the W4A4 linear layer that consumes the quantizer's output.
+// Included by kroquant.cu; uses its helpers (mbarriers, TMA, descriptors of
+// kq_mma.cuh).
+//
+// D[m][n] = sum_k a[m][k] b[n][k], where a = MXFP4(X T^T) [M x K] is the
+// quantized activation and b = MXFP4(W T^-1) [N x K] the quantized folded
+// weight ("KroQuant: Kronecker-Structured Block Transforms for Efficient
+// Post-Training Quantization of Diffusion Transformers", abstract: W4A4 at
+// MXFP4; section 3.2, Eq. (4): the inverse folded into the weights).  Both
+// operands are K-major as the quantizers write them (codes [rows][K/2], even
+// element in the low nibble), with their E8M0 scales in the scale-factor
+// layout (SfPos in kroquant.cu).  D is bf16 or fp32, [M][N] row-major.
+//
+// One tcgen05 block-scaled MMA (kind::mxf4, block32) is M128 x N256 x K64: the
+// tensor core decodes E2M1 and applies the two E8M0 scales of every 32-block,
+// accumulating in fp32 in tensor memory.  The scale bytes reach tensor memory
+// by tcgen05.cp from shared memory (one 512-byte unit = 128 rows x 4 blocks
+// per copy, 32 lanes x 128 bits replicated to the four lane quarters).
+//
+// A CTA owns one SM (persistent) and walks the 128 x 256 output tiles
+// t = blockIdx.x, + gridDim.x, ...; a k-chunk is 256 elements (128 bytes of
+// codes per row, one 128-byte swizzle atom).
+//   warp 0     producer: per chunk, TMA loads of the A box {128 B x 128 rows}
+//              and the B box {128 B x 256 rows} (128-byte swizzle; rows and
+//              bytes past the matrix read as zero) and bulk copies of the
+//              scale units (A: the row group's 2 units of the chunk, B: 2 row
+//              groups x 2 units) into a kStages ring
+//   warp 1     allocates tensor memory; one thread copies a stage's scale
+//              units to tensor memory, issues the chunk's four MMAs (only the
+//              K=64 steps below K) and commits the stage back to the producer;
+//              after a tile's last chunk it commits the accumulator
+//   warps 2-9  epilogue: warp w reads accumulator lanes 32 (w % 4) .. +31 (tile
+//              rows) and columns 128 ((w - 2) / 4) .. +127 into registers,
+//              hands the accumulator back at once, then converts and stores its
+//              row segment while the MMAs of the next tile run
+// Every mbarrier wait is bounded (g_wait_timeouts); every path drains the
+// copies in flight, waits for its MMAs and frees the tensor memory.
+
+namespace gemm {
+
+constexpr int kBM = 128;                                  // tile rows (MMA M)
+constexpr int kBN = 256;                                  // tile columns (MMA N)
+constexpr int kChunkBytes = 128;                          // codes bytes per row per k-chunk (256 elements)
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kChunkBytes;                // 16 KB
+constexpr int kBBytes = kBN * kChunkBytes;                // 32 KB
+constexpr int kSfUnit = 512;                              // 128 rows x 4 blocks
+constexpr int kSfaBytes = 2 * kSfUnit;                    // the chunk's 2 units of the A row group
+constexpr int kSfbBytes = 4 * kSfUnit;                    // 2 row groups x 2 units
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 51 KB, a multiple of 1 KB
+constexpr int kTmemCols = 512;                            // power of two >= 256 + 8 + 16
+constexpr uint32_t kAccCol = 0;                           // 256 fp32 accumulator columns
+constexpr uint32_t kSfaCol = 256;                         // 2 units x 4 columns
+constexpr uint32_t kSfbCol = 264;                         // 2 units x 8 columns (N = 256: 8 row groups of 32)
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;             // 320
+constexpr size_t kSmem = size_t(kStages) * kStageBytes + 1024 + (2 * kStages + 4) * sizeof(uint64_t) + 16;
+
+static_assert(kStageBytes % 1024 == 0, "stages must keep the 1 KB alignment of the 128-byte swizzle");
+
+// Instruction descriptor, block-scaled kinds: b_sf_id bits 4-5, A format
+// bits 7-9 and B format bits 10-12 (1 = E2M1 for kind::mxf4), K-major A and B
+// (bits 15, 16 = 0), N >> 3 in bits 17-22, scale format bit 23 (1 = E8M0),
+// M >> 4 in bits 24-28, a_sf_id bits 29-30, bit 31 = 0 (K = 64).
+constexpr uint32_t kIdescBase =
+    (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24);
+
+// sf_id selects the byte pair of each 32-bit scale word: the K=64 step j of a
+// 128-element unit reads blocks 2j and 2j+1, i.e. bytes 2j, 2j+1.
+__device__ __forceinline__ uint32_t idesc(uint32_t sf_id) { return kIdescBase | (sf_id << 4) | (sf_id << 29); }
+
+__device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t id,
+                                          uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                     tmem_d),
+                 "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
+                 : "memory");
+}
+
+// One 512-byte scale unit (shared memory, 32 rows x 16 bytes, no swizzle) to
+// 4 tensor-memory columns, replicated to the four 32-lane quarters.
+__device__ __forceinline__ void tmem_copy_unit(uint32_t taddr, uint32_t saddr)
+{
+    const uint64_t desc = mma::smem_desc(saddr, 128, 0);
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// Plain (untiled) bulk copy global -> shared, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 32 fp32 columns of this thread's lane, no wait (the caller waits once).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float *v)
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <bool F32OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap b_map,
+                 const uint8_t *__restrict__ a_sf, const uint8_t *__restrict__ b_sf, void *__restrict__ out, int M,
+                 int N, int K, long long budget)
+{
+    extern __shared__ uint8_t smem_dyn[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + size_t(kStages) * kStageBytes);
+    uint64_t *full = bars;                    // [kStages] stage landed (TMA / bulk tx)
+    uint64_t *empty = bars + kStages;         // [kStages] MMAs reading the stage done (commit)
+    uint64_t *acc_full = bars + 2 * kStages;  // accumulator holds a finished tile (commit)
+    uint64_t *acc_empty = acc_full + 1;       // accumulator read by the 8 epilogue warps
+    uint64_t *done = acc_full + 2;            // every MMA of this CTA completed (final commit)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 4);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    const int MT = (M + kBM - 1) / kBM;
+    const int NT = (N + kBN - 1) / kBN;
+    const int tiles = MT * NT;
+    const int KC = (K + 255) / 256;           // k-chunks
+    const int KS = (K + 63) / 64;             // MMA K steps
+    const int Ka = (K + 127) / 128;           // scale units per 128-row group
+    const int NRa = (N + 127) / 128;          // B row groups with scale units
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, kEpiWarps);
+        mbar_init(done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    mma::tc_fence_before();
+    __syncthreads();
+    mma::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- producer
+            int k = 0, filled = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int mt = t / NT, nt = t % NT;
+                const bool b_hi = 2 * nt + 1 < NRa;        // the tile's second B row group exists
+                for (int c = 0; c < KC; ++c, ++k) {
+                    const int s = k % kStages;
+                    if (k >= kStages && !mbar_wait(&empty[s], ((k / kStages) - 1) & 1, budget)) {
+                        atomicAdd(&g_wait_timeouts, 1);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = base + size_t(s) * kStageBytes;
+                    uint8_t *sfa = st + kABytes + kBBytes;
+                    uint8_t *sfb = sfa + kSfaBytes;
+                    const int ka0 = 2 * c;
+                    const uint32_t sfbytes = uint32_t(Ka - ka0 >= 2 ? 2 : 1) * kSfUnit;
+                    mbar_expect_tx(&full[s], uint32_t(kABytes + kBBytes) + sfbytes * (b_hi ? 3u : 2u));
+                    mma::tma_load_2d(st, &a_map, c * kChunkBytes, mt * kBM, &full[s]);
+                    mma::tma_load_2d(st + kABytes, &b_map, c * kChunkBytes, nt * kBN, &full[s]);
+                    bulk_load(sfa, a_sf + (int64_t(mt) * Ka + ka0) * kSfUnit, sfbytes, &full[s]);
+                    bulk_load(sfb, b_sf + (int64_t(2 * nt) * Ka + ka0) * kSfUnit, sfbytes, &full[s]);
+                    if (b_hi) bulk_load(sfb + 2 * kSfUnit, b_sf + (int64_t(2 * nt + 1) * Ka + ka0) * kSfUnit, sfbytes,
+                                        &full[s]);
+                    filled = k + 1;
+                }
+            }
+            // drain: the copies issued have landed before the CTA may exit
+            for (int kk = (filled > kStages ? filled - kStages : 0); kk < filled; ++kk)
+                if (!mbar_wait(&full[kk % kStages], (kk / kStages) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    break;
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- scale copies and MMAs (one thread)
+            int k = 0, it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+                if (it > 0 && !mbar_wait(acc_empty, (it - 1) & 1, budget)) {
+                    atomicAdd(&g_wait_timeouts, 1);
+                    break;
+                }
+                mma::tc_fence_after();
+                for (int c = 0; c < KC; ++c, ++k) {
+                    const int s = k % kStages;
+                    if (!mbar_wait(&full[s], (k / kStages) & 1, budget)) {
+                        atomicAdd(&g_wait_timeouts, 1);
+                        ok = false;
+                        break;
+                    }
+                    mma::tc_fence_after();
+                    const uint32_t a0 = smem_addr(base + size_t(s) * kStageBytes);
+                    const uint32_t b0 = a0 + kABytes;
+                    const uint32_t sfa = b0 + kBBytes;
+                    const uint32_t sfb = sfa + kSfaBytes;
+                    // units of a missing B row group or past K are stale data;
+                    // they only reach output columns >= N or K steps not issued
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        tmem_copy_unit(tmem_base + kSfaCol + 4 * u, sfa + u * kSfUnit);
+                        tmem_copy_unit(tmem_base + kSfbCol + 8 * u, sfb + u * kSfUnit);
+                        tmem_copy_unit(tmem_base + kSfbCol + 8 * u + 4, sfb + (2 + u) * kSfUnit);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (c * 4 + j >= KS) break;
+                        const uint32_t sf_id = (j & 1) * 2;
+                        const uint32_t u = j >> 1;
+                        const uint64_t ad = mma::smem_desc(a0 + j * 32, 1024, mma::kLayoutSw128);
+                        const uint64_t bd = mma::smem_desc(b0 + j * 32, 1024, mma::kLayoutSw128);
+                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(sf_id),
+                                  (tmem_base + kSfaCol + 4 * u) | (sf_id << 30),
+                                  (tmem_base + kSfbCol + 8 * u) | (sf_id << 30), (c | j) != 0);
+                    }
+                    mma::umma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                mma::umma_commit(acc_full);
+            }
+            // every MMA issued has completed before the tensor memory is freed
+            mma::umma_commit(done);
+            if (!mbar_wait(done, 0, budget)) atomicAdd(&g_wait_timeouts, 1);
+        }
+    } else {
+        // ---------------- epilogue
+        const int q = warp & 3;                   // lane quarter this warp may read
+        const int h = (warp - 2) >> 2;            // column half of the tile
+        int it = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+            const int mt = t / NT, nt = t % NT;
+            const bool ready = mbar_wait(acc_full, it & 1, budget);
+            if (!__all_sync(0xffffffffu, ready)) {   // tcgen05.ld below is warp-collective
+                if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
+                break;
+            }
+            mma::tc_fence_after();
+            float v[128];
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(h * 128);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tmem_ld32_nowait(taddr + 32 * i, v + 32 * i);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            mma::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+
+            const int row = mt * kBM + q * 32 + lane;
+            const int col0 = nt * kBN + h * 128;
+            if (row < M) {
+                if constexpr (F32OUT) {
+                    float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + int64_t(row) * N + col0);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + 4 * i < N) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                } else {
+                    uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + int64_t(row) * N + col0);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (col0 + 8 * i < N)
+                            o[i] = make_uint4(mma::pack_bf16x2(v[8 * i], v[8 * i + 1]),
+                                              mma::pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                              mma::pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
+                                              mma::pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                }
+            }
+        }
+    }
+
+    mma::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        mma::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace gemm

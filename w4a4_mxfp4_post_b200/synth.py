@@ -45,6 +45,10 @@ WORKLOADS = {
 
 MODELS = ("tiny", "pixart", "sana", "flux")
 
+# The W4A4 linear layers fed by the quantizer: the PixArt-Sigma MLP at 8192
+# tokens, (N, K) per layer: fc1 1152 -> 4608 and fc2 4608 -> 1152.
+GEMM_LAYERS = {"pixart_mlp": {"M": 8192, "layers": ((4608, 1152), (1152, 4608)), "seed": 5}}
+
 
 def _rng(*key: int) -> np.random.Generator:
     return np.random.default_rng(np.random.SeedSequence([int(k) for k in key]))
@@ -203,3 +207,13 @@ def workload_layers(name: str):
     shared = w["factors"] == "shared"
     Ms = w.get("Ms", (w.get("M"),))
     return [(M, d, w["model"], shared, w["seed"]) for M in Ms for d in w["ds"]]
+
+
+def mx_operand(rows: int, K: int, seed: int, scale_lo: int = 112, scale_hi: int = 142):
+    """A random MXFP4 operand: codes [rows, K/2] (every byte value equally
+    likely, so every E2M1 code and sign) and E8M0 scale bytes [rows, K/32]
+    uniform in [scale_lo, scale_hi)."""
+    g = _rng(seed, 7, rows, K)
+    codes = g.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    scales = g.integers(scale_lo, scale_hi, (rows, K // 32), dtype=np.uint8)
+    return codes, scales
