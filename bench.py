@@ -659,15 +659,19 @@ def gemm_mode(args):
     outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
     stream = torch.cuda.Stream(device=dev)
 
+    variants = [int(v) for v in args.kernels.split(",")] if args.kernels[0].isdigit() else [0]
+
     def run(kind, n):
         for i in range(n):
             k = i % nsets
             if kind == "chain":
                 kq.kq_quantize_sf(xs[k], Fd, out_codes=acs[k], out_sf=asfs[k], stream=stream)
-            kq.mxf4_gemm(acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
+                kq.mxf4_gemm(acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
+            else:
+                kq.mxf4_gemm_variant(int(kind[1:]), acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
 
     res = {}
-    for kind in ("gemm", "chain"):
+    for kind in [f"v{v}" for v in variants] + ["chain"]:
         with torch.cuda.stream(stream):
             run(kind, max(3, args.warmup))
         stream.synchronize()
@@ -696,12 +700,14 @@ def gemm_mode(args):
     except Exception:
         bf16, src = 1590.0, "fallback bf16 1.59 PFLOP/s x 4 (nominal fp4/bf16 dense ratio)"
     peak = 4.0 * bf16
-    tflops = flops / (res["gemm"] * 1e-6) / 1e12
+    first = f"v{variants[0]}"
+    tflops = flops / (res[first] * 1e-6) / 1e12
     out_bytes = M * N * 2 + M * K // 2 + N * K // 2
-    print(json.dumps({"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets, "gemm_us": round(res["gemm"], 3),
+    print(json.dumps({"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets,
+                      "gemm_us": {k: round(v, 3) for k, v in res.items() if k != "chain"},
                       "chain_us": round(res["chain"], 3), "tflops": round(tflops, 1), "peak_tflops": peak,
                       "frac_of_peak": round(tflops / peak, 4), "peak_source": src,
-                      "hbm_gbs_min_bytes": round(out_bytes / (res["gemm"] * 1e-6) / 1e9, 1)}), flush=True)
+                      "hbm_gbs_min_bytes": round(out_bytes / (res[first] * 1e-6) / 1e9, 1)}), flush=True)
 
 
 def sweep_mode(args):
@@ -826,7 +832,8 @@ def main():
                          "sqnr: quantisation-error proxy per method")
     ap.add_argument("--kernel", default="kq",
                     help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H> or norm_kq")
-    ap.add_argument("--kernels", default="kq,sq,mx", help="sweep mode: comma-separated kernels")
+    ap.add_argument("--kernels", default="kq,sq,mx",
+                    help="sweep mode: comma-separated kernels; gemm mode: comma-separated tile configurations")
     ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD; gemm mode: MxNxK")
     ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")
     ap.add_argument("--no-graph", action="store_true", help="kernel mode: eager launches")

@@ -211,6 +211,21 @@ int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf,
               void *out, int out_f32, int64_t M, int64_t N, int64_t K,
               cudaStream_t stream);
 
+/* Test export: mxf4_gemm through a chosen tile configuration (all 128 x 256
+ * output tiles, one CTA per SM; a k-chunk is CB bytes of codes per row):
+ *   0  the default (what mxf4_gemm runs: 4),
+ *   1  CB = 128, 4 stages, epilogue stores from registers,
+ *   2  CB = 64, 6 stages, bf16 epilogue through shared memory and TMA stores,
+ *   3  CB = 64, 4 stages, TMA stores,
+ *   4  CB = 128, 3 stages, TMA stores,
+ *   5  CB = 64, 8 stages, stores from registers.
+ * Same results for every configuration (the K order of the MMAs is the same).
+ * Other values return KQ_ERR_VARIANT. */
+int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf,
+                      const uint8_t *b_codes, const uint8_t *b_sf,
+                      void *out, int out_f32, int64_t M, int64_t N, int64_t K,
+                      cudaStream_t stream);
+
 /* Test export: the fp32 transform y = T x (float32 [M][d]) exactly as the
  * quantizer computes it before the amax, for the transform-accuracy check. */
 int kq_transform_f32(const void *act_bf16, const float *factors, int shared,

@@ -130,6 +130,25 @@ def test_mxf4_gemm_random_operands(cuda_device, M, N, K, f32):
     assert kq.kq_wait_timeouts() == 0
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 520, 1152), (77, 136, 5600), (256, 264, 96)])
+def test_mxf4_gemm_configurations_agree(cuda_device, M, N, K):
+    """Every tile configuration gives the same bits (same K order), and the
+    oracle's bound holds for each."""
+    import torch
+
+    ca, sa = synth.mx_operand(M, K, 51)
+    cb, sb = synth.mx_operand(N, K, 52)
+    args = [dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
+            dev(oracle.scales_to_sf(sb), cuda_device)]
+    D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+    for dtype in (torch.float32, torch.bfloat16):
+        ref = kq.mxf4_gemm_variant(1, *args, out_dtype=dtype)
+        check_gemm(ref.float().cpu().numpy(), D, absd, K, dtype == torch.bfloat16)
+        for v in (0, 2, 3, 4, 5):
+            got = kq.mxf4_gemm_variant(v, *args, out_dtype=dtype)
+            assert torch.equal(got, ref), (v, dtype)
+
+
 def test_mxf4_gemm_repeated_calls_and_other_stream(cuda_device):
     import torch
 

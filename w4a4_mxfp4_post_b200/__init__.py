@@ -33,7 +33,7 @@ __all__ = [
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
     "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize", "kq_inverse_f32", "mx_dequantize", "norm_kq_quantize",
     "KQ_SCALES_ROWMAJOR", "KQ_SCALES_SF", "kq_sf_bytes", "kq_quantize_sf", "mx_quantize_f32", "mx_scales_to_sf",
-    "mxf4_gemm",
+    "mxf4_gemm", "mxf4_gemm_variant",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -62,6 +62,7 @@ _SIGS = {
     "mx_quantize_f32": "pppiqqp",
     "mx_scales_to_sf": "ppqqp",
     "mxf4_gemm": "pppppiqqqp",
+    "mxf4_gemm_variant": "ipppppiqqqp",
 }
 
 _lib = None
@@ -444,6 +445,11 @@ def mxf4_gemm(a_codes, a_sf, b_codes, b_sf, out=None, out_dtype=None, stream=Non
     a_codes [M, K/2], b_codes [N, K/2] uint8; a_sf, b_sf their scales in the
     scale-factor layout; out bf16 (default) or float32 [M, N].
     """
+    return mxf4_gemm_variant(0, a_codes, a_sf, b_codes, b_sf, out, out_dtype, stream)
+
+
+def mxf4_gemm_variant(variant, a_codes, a_sf, b_codes, b_sf, out=None, out_dtype=None, stream=None):
+    """mxf4_gemm through a chosen tile configuration (0 = the default; test export)."""
     torch = _torch()
     _need(a_codes, "a_codes", torch.uint8)
     if a_codes.dim() != 2 or b_codes.dim() != 2:
@@ -461,6 +467,6 @@ def mxf4_gemm(a_codes, a_sf, b_codes, b_sf, out=None, out_dtype=None, stream=Non
     if out.dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("out must be bfloat16 or float32")
     _need(out, "out", out.dtype, dev, (M, N))
-    _call("mxf4_gemm", _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
+    _call("mxf4_gemm_variant", int(variant), _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
           int(out.dtype == torch.float32), M, N, K, _stream(stream))
     return out

@@ -1395,7 +1395,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
     kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2,
-    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kGemmBf16, kGemmF32, kNumKernels
+    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1599,19 +1599,38 @@ int smem_prepare(KernelId id, const void *fn, size_t bytes)
 }
 
 // MXFP4 codes [rows][K/2] as a uint8 matrix read by the W4A4 product: boxes of
-// {128 bytes x box_rows}, 128-byte swizzle, rows and bytes past the matrix
-// read as zero.
-int encode_gemm_map(const void *codes, int64_t rows, int64_t K, int box_rows, CUtensorMap *map)
+// {cb bytes x box_rows}, cb-byte swizzle (cb = 64 or 128), rows and bytes past
+// the matrix read as zero.
+int encode_gemm_map(const void *codes, int64_t rows, int64_t K, int cb, int box_rows, CUtensorMap *map)
 {
     EncodeTiledFn enc;
     int rc = encode_fn(&enc);
     if (rc != KQ_OK) return rc;
     const cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
     const cuuint64_t strides[1] = {cuuint64_t(K / 2)};
-    const cuuint32_t box[2] = {cuuint32_t(gemm::kChunkBytes), cuuint32_t(box_rows)};
+    const cuuint32_t box[2] = {cuuint32_t(cb), cuuint32_t(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(codes), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           cb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
+// The bf16 output D [M][N] of the W4A4 product: boxes of {64 columns x 32
+// rows} (one epilogue warp's half row segment), 128-byte swizzle.
+int encode_gemm_out_map(void *out, int64_t M, int64_t N, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
+    const cuuint64_t strides[1] = {cuuint64_t(N) * 2};
+    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
     return KQ_OK;
@@ -1743,6 +1762,59 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
         }
     }
     return launch_check(fn);
+}
+
+// The W4A4 product, one tile configuration: tensor maps, grid (one CTA per
+// SM or per tile), shared-memory attribute (set once per device and
+// instantiation), launch.
+struct GemmArgs {
+    const uint8_t *a_codes, *a_sf, *b_codes, *b_sf;
+    void *out;
+    bool f32;
+    int64_t M, N, K, tiles;
+    cudaStream_t stream;
+};
+
+constexpr int kDefaultGemmVariant = 4;
+
+template <class C, bool F32>
+std::atomic<int> g_gemm_smem_set[kMaxDevices];
+
+template <class C, bool F32>
+int gemm_launch_out(const GemmArgs &g, const CUtensorMap &amap, const CUtensorMap &bmap, const CUtensorMap &omap,
+                    unsigned grid)
+{
+    auto k = gemm::mxf4_gemm_kernel<C, F32>;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices || !g_gemm_smem_set<C, F32>[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_gemm_smem_set<C, F32>[dev].store(1, std::memory_order_release);
+    }
+    k<<<grid, gemm::kThreads, C::kSmem, g.stream>>>(amap, bmap, omap, g.a_sf, g.b_sf, g.out, int(g.M), int(g.N),
+                                                     int(g.K), kWaitBudget);
+    return launch_check("mxf4_gemm");
+}
+
+template <class C>
+int gemm_launch(const GemmArgs &g)
+{
+    CUtensorMap amap, bmap, omap;
+    int rc = encode_gemm_map(g.a_codes, g.M, g.K, C::kCB, gemm::kBM, &amap);
+    if (rc != KQ_OK) return rc;
+    if ((rc = encode_gemm_map(g.b_codes, g.N, g.K, C::kCB, gemm::kBN, &bmap)) != KQ_OK) return rc;
+    // only the TMA-store epilogue reads the output map; the others get a placeholder
+    if (C::kTmaOut && !g.f32) {
+        if ((rc = encode_gemm_out_map(g.out, g.M, g.N, &omap)) != KQ_OK) return rc;
+    } else {
+        omap = amap;
+    }
+    int sms = 0;
+    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
+    const unsigned grid = unsigned(g.tiles < sms ? g.tiles : sms);
+    return g.f32 ? gemm_launch_out<C, true>(g, amap, bmap, omap, grid) : gemm_launch_out<C, false>(g, amap, bmap, omap, grid);
 }
 
 }  // namespace
@@ -2071,8 +2143,8 @@ int mx_scales_to_sf(const uint8_t *scales, uint8_t *out_sf, int64_t M, int64_t d
     return launch_check(fn);
 }
 
-int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes, const uint8_t *b_sf, void *out,
-              int out_f32, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes,
+                      const uint8_t *b_sf, void *out, int out_f32, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
 {
     const char *fn = "mxf4_gemm";
     if (M < 0 || N < 0 || K <= 0 || K % kBlk != 0 || N % 8 != 0)
@@ -2080,26 +2152,29 @@ int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_code
                     "(M=%lld, N=%lld, K=%lld)", fn, (long long)M, (long long)N, (long long)K);
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return fail(KQ_ERR_SHAPE, "%s: M, N and K must be below 2^31", fn);
+    if (variant == 0) variant = kDefaultGemmVariant;
+    if (variant < 1 || variant > 5) return fail(KQ_ERR_VARIANT, "%s: variant %d is not available", fn, variant);
     if (M == 0 || N == 0) return ok();
     if (!a_codes || !a_sf || !b_codes || !b_sf || !out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
     if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
         !aligned(out, 16))
         return fail(KQ_ERR_ALIGN, "%s: every pointer must be 16-byte aligned", fn);
-    CUtensorMap amap, bmap;
-    int rc = encode_gemm_map(a_codes, M, K, gemm::kBM, &amap);
-    if (rc != KQ_OK) return rc;
-    if ((rc = encode_gemm_map(b_codes, N, K, gemm::kBN, &bmap)) != KQ_OK) return rc;
     const int64_t tiles = ((M + gemm::kBM - 1) / gemm::kBM) * ((N + gemm::kBN - 1) / gemm::kBN);
     if (tiles >= (int64_t(1) << 31)) return fail(KQ_ERR_SHAPE, "%s: too many output tiles", fn);
-    int sms = 0;
-    if ((rc = sm_count(&sms)) != KQ_OK) return rc;
-    const unsigned grid = unsigned(tiles < sms ? tiles : sms);
-    auto k = out_f32 ? gemm::mxf4_gemm_kernel<true> : gemm::mxf4_gemm_kernel<false>;
-    if ((rc = smem_prepare(out_f32 ? kGemmF32 : kGemmBf16, reinterpret_cast<const void *>(k), gemm::kSmem)) != KQ_OK)
-        return rc;
-    k<<<grid, gemm::kThreads, gemm::kSmem, stream>>>(amap, bmap, a_sf, b_sf, out, int(M), int(N), int(K),
-                                                     kWaitBudget);
-    return launch_check(fn);
+    const GemmArgs g{a_codes, a_sf, b_codes, b_sf, out, out_f32 != 0, M, N, K, tiles, stream};
+    switch (variant) {
+    case 1: return gemm_launch<gemm::Cfg1>(g);
+    case 2: return gemm_launch<gemm::Cfg2>(g);
+    case 3: return gemm_launch<gemm::Cfg3>(g);
+    case 4: return gemm_launch<gemm::Cfg4>(g);
+    default: return gemm_launch<gemm::Cfg5>(g);
+    }
+}
+
+int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf, const uint8_t *b_codes, const uint8_t *b_sf, void *out,
+              int out_f32, int64_t M, int64_t N, int64_t K, cudaStream_t stream)
+{
+    return mxf4_gemm_variant(0, a_codes, a_sf, b_codes, b_sf, out, out_f32, M, N, K, stream);
 }
 
 int kq_wait_timeouts(int *count, int reset)

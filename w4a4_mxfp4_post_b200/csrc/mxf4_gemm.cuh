@@ -18,21 +18,27 @@
 // per copy, 32 lanes x 128 bits replicated to the four lane quarters).
 //
 // A CTA owns one SM (persistent) and walks the 128 x 256 output tiles
-// t = blockIdx.x, + gridDim.x, ...; a k-chunk is 256 elements (128 bytes of
-// codes per row, one 128-byte swizzle atom).
-//   warp 0     producer: per chunk, TMA loads of the A box {128 B x 128 rows}
-//              and the B box {128 B x 256 rows} (128-byte swizzle; rows and
+// t = blockIdx.x, + gridDim.x, ...; a k-chunk is CB bytes of codes per row
+// (2 CB elements, one CB-byte swizzle atom; CB / 64 scale units per row
+// group), CB and the ring depth ST being compile-time choices (Cfg).
+//   warp 0     producer: per chunk, TMA loads of the A box {CB x 128 rows}
+//              and the B box {CB x 256 rows} (CB-byte swizzle; rows and
 //              bytes past the matrix read as zero) and bulk copies of the
-//              scale units (A: the row group's 2 units of the chunk, B: 2 row
-//              groups x 2 units) into a kStages ring
+//              chunk's scale units (A: its row group's, B: both row groups')
+//              into an ST-stage ring
 //   warp 1     allocates tensor memory; one thread copies a stage's scale
-//              units to tensor memory, issues the chunk's four MMAs (only the
-//              K=64 steps below K) and commits the stage back to the producer;
-//              after a tile's last chunk it commits the accumulator
+//              units to that stage's own tensor-memory columns (so a copy
+//              never waits on MMAs still reading an older stage), issues the
+//              chunk's CB / 32 MMAs (only the K=64 steps below K) and commits the
+//              stage back to the producer; after a tile's last chunk it
+//              commits the accumulator
 //   warps 2-9  epilogue: warp w reads accumulator lanes 32 (w % 4) .. +31 (tile
-//              rows) and columns 128 ((w - 2) / 4) .. +127 into registers,
-//              hands the accumulator back at once, then converts and stores its
-//              row segment while the MMAs of the next tile run
+//              rows) and columns 128 ((w - 2) / 4) .. +127 into registers and
+//              hands the accumulator back at once; then, while the MMAs of the
+//              next tile run, it stores its segment: with TMA_OUT (bf16) through
+//              the warp's 8 KB of shared memory (128-byte swizzle) and two TMA
+//              tensor stores of {64 columns x 32 rows} (rows and columns past D
+//              are clipped), otherwise with 16-byte stores from registers
 // Every mbarrier wait is bounded (g_wait_timeouts); every path drains the
 // copies in flight, waits for its MMAs and frees the tensor memory.
 
@@ -40,23 +46,41 @@ namespace gemm {
 
 constexpr int kBM = 128;                                  // tile rows (MMA M)
 constexpr int kBN = 256;                                  // tile columns (MMA N)
-constexpr int kChunkBytes = 128;                          // codes bytes per row per k-chunk (256 elements)
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kChunkBytes;                // 16 KB
-constexpr int kBBytes = kBN * kChunkBytes;                // 32 KB
 constexpr int kSfUnit = 512;                              // 128 rows x 4 blocks
-constexpr int kSfaBytes = 2 * kSfUnit;                    // the chunk's 2 units of the A row group
-constexpr int kSfbBytes = 4 * kSfUnit;                    // 2 row groups x 2 units
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;   // 51 KB, a multiple of 1 KB
-constexpr int kTmemCols = 512;                            // power of two >= 256 + 8 + 16
+constexpr int kTmemCols = 512;                            // power of two >= 256 + scale columns
 constexpr uint32_t kAccCol = 0;                           // 256 fp32 accumulator columns
-constexpr uint32_t kSfaCol = 256;                         // 2 units x 4 columns
-constexpr uint32_t kSfbCol = 264;                         // 2 units x 8 columns (N = 256: 8 row groups of 32)
+constexpr uint32_t kSfCol = 256;                          // scale columns, per stage
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;             // 320
-constexpr size_t kSmem = size_t(kStages) * kStageBytes + 1024 + (2 * kStages + 4) * sizeof(uint64_t) + 16;
+constexpr int kStageOutBytes = 32 * 128 * 2;              // a warp's 32 rows x 128 bf16 columns
+constexpr size_t kSmemMax = 232448;                       // 227 KB per CTA
 
-static_assert(kStageBytes % 1024 == 0, "stages must keep the 1 KB alignment of the 128-byte swizzle");
+// Tile configuration: CB codes bytes per row per k-chunk (64 or 128), ST ring
+// stages, TMA_OUT = bf16 output through shared memory and TMA stores.
+template <int CB, int ST, bool TMA_OUT>
+struct Cfg {
+    static constexpr int kCB = CB;
+    static constexpr int kST = ST;
+    static constexpr bool kTmaOut = TMA_OUT;
+    static constexpr int kUnits = CB / 64;                // scale units per row group per chunk
+    static constexpr int kMmas = CB / 32;                 // K=64 MMAs per chunk
+    static constexpr int kABytes = kBM * CB;
+    static constexpr int kBBytes = kBN * CB;
+    static constexpr int kSfaBytes = kUnits * kSfUnit;
+    static constexpr int kSfbBytes = 2 * kUnits * kSfUnit;
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr uint32_t kSfStageCols = 12 * kUnits; // A: 4 per unit, B: 8 per unit
+    static constexpr uint64_t kLayout = CB == 128 ? mma::kLayoutSw128 : mma::kLayoutSw64;
+    static constexpr uint32_t kSbo = 8 * CB;              // 8-row swizzle atom
+    static constexpr size_t kRing = size_t(ST) * kStageBytes;
+    static constexpr size_t kSmem = kRing + (TMA_OUT ? size_t(kEpiWarps) * kStageOutBytes : 0) + 1024 +
+                                    (2 * ST + 4) * sizeof(uint64_t) + 16;
+    static_assert(CB == 64 || CB == 128, "chunk bytes");
+    static_assert(kStageBytes % (8 * CB) == 0, "stages keep the alignment of the swizzle atom");
+    static_assert(!TMA_OUT || kRing % 1024 == 0, "the output staging keeps the 1 KB alignment of its swizzle");
+    static_assert(kSfCol + ST * kSfStageCols <= kTmemCols, "tensor memory columns");
+    static_assert(kSmem <= kSmemMax, "shared memory");
+};
 
 // Instruction descriptor, block-scaled kinds: b_sf_id bits 4-5, A format
 // bits 7-9 and B format bits 10-12 (1 = E2M1 for kind::mxf4), K-major A and B
@@ -66,7 +90,7 @@ constexpr uint32_t kIdescBase =
     (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24);
 
 // sf_id selects the byte pair of each 32-bit scale word: the K=64 step j of a
-// 128-element unit reads blocks 2j and 2j+1, i.e. bytes 2j, 2j+1.
+// 128-element unit reads blocks 2j and 2j+1, i.e. bytes 2j, 2j+1 (sf_id 2j).
 __device__ __forceinline__ uint32_t idesc(uint32_t sf_id) { return kIdescBase | (sf_id << 4) | (sf_id << 29); }
 
 __device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t id,
@@ -108,18 +132,21 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float *v)
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-template <bool F32OUT>
+template <class C, bool F32OUT>
 __global__ void __launch_bounds__(kThreads, 1)
 mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap b_map,
-                 const uint8_t *__restrict__ a_sf, const uint8_t *__restrict__ b_sf, void *__restrict__ out, int M,
-                 int N, int K, long long budget)
+                 const __grid_constant__ CUtensorMap out_map, const uint8_t *__restrict__ a_sf,
+                 const uint8_t *__restrict__ b_sf, void *__restrict__ out, int M, int N, int K, long long budget)
 {
+    constexpr int ST = C::kST;
+    constexpr bool kStaged = C::kTmaOut && !F32OUT;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + size_t(kStages) * kStageBytes);
-    uint64_t *full = bars;                    // [kStages] stage landed (TMA / bulk tx)
-    uint64_t *empty = bars + kStages;         // [kStages] MMAs reading the stage done (commit)
-    uint64_t *acc_full = bars + 2 * kStages;  // accumulator holds a finished tile (commit)
+    uint8_t *stage_out = base + C::kRing;                // [kEpiWarps] x 8 KB output staging (TMA_OUT)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(stage_out + (C::kTmaOut ? size_t(kEpiWarps) * kStageOutBytes : 0));
+    uint64_t *full = bars;                    // [ST] stage landed (TMA / bulk tx)
+    uint64_t *empty = bars + ST;              // [ST] MMAs reading the stage done (commit)
+    uint64_t *acc_full = bars + 2 * ST;       // accumulator holds a finished tile (commit)
     uint64_t *acc_empty = acc_full + 1;       // accumulator read by the 8 epilogue warps
     uint64_t *done = acc_full + 2;            // every MMA of this CTA completed (final commit)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 4);
@@ -128,13 +155,13 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
     const int MT = (M + kBM - 1) / kBM;
     const int NT = (N + kBN - 1) / kBN;
     const int tiles = MT * NT;
-    const int KC = (K + 255) / 256;           // k-chunks
-    const int KS = (K + 63) / 64;             // MMA K steps
-    const int Ka = (K + 127) / 128;           // scale units per 128-row group
-    const int NRa = (N + 127) / 128;          // B row groups with scale units
+    const int KC = (K + 2 * C::kCB - 1) / (2 * C::kCB);   // k-chunks
+    const int Ka = (K + 127) / 128;                       // scale units per 128-row group
+    const int KS = (K + 63) / 64;                         // MMA K steps
+    const int NRa = (N + 127) / 128;                      // B row groups with scale units
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < ST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -163,30 +190,32 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 const int mt = t / NT, nt = t % NT;
                 const bool b_hi = 2 * nt + 1 < NRa;        // the tile's second B row group exists
                 for (int c = 0; c < KC; ++c, ++k) {
-                    const int s = k % kStages;
-                    if (k >= kStages && !mbar_wait(&empty[s], ((k / kStages) - 1) & 1, budget)) {
+                    const int s = k % ST;
+                    if (k >= ST && !mbar_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
                         atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
-                    uint8_t *st = base + size_t(s) * kStageBytes;
-                    uint8_t *sfa = st + kABytes + kBBytes;
-                    uint8_t *sfb = sfa + kSfaBytes;
-                    const int ka0 = 2 * c;
-                    const uint32_t sfbytes = uint32_t(Ka - ka0 >= 2 ? 2 : 1) * kSfUnit;
-                    mbar_expect_tx(&full[s], uint32_t(kABytes + kBBytes) + sfbytes * (b_hi ? 3u : 2u));
-                    mma::tma_load_2d(st, &a_map, c * kChunkBytes, mt * kBM, &full[s]);
-                    mma::tma_load_2d(st + kABytes, &b_map, c * kChunkBytes, nt * kBN, &full[s]);
-                    bulk_load(sfa, a_sf + (int64_t(mt) * Ka + ka0) * kSfUnit, sfbytes, &full[s]);
-                    bulk_load(sfb, b_sf + (int64_t(2 * nt) * Ka + ka0) * kSfUnit, sfbytes, &full[s]);
-                    if (b_hi) bulk_load(sfb + 2 * kSfUnit, b_sf + (int64_t(2 * nt + 1) * Ka + ka0) * kSfUnit, sfbytes,
-                                        &full[s]);
+                    uint8_t *st = base + size_t(s) * C::kStageBytes;
+                    uint8_t *sfa = st + C::kABytes + C::kBBytes;
+                    uint8_t *sfb = sfa + C::kSfaBytes;
+                    const int u0 = c * C::kUnits;
+                    const int nu = Ka - u0 < C::kUnits ? Ka - u0 : C::kUnits;   // units of this chunk, >= 1
+                    const uint32_t sfbytes = uint32_t(nu) * kSfUnit;
+                    mbar_expect_tx(&full[s], uint32_t(C::kABytes + C::kBBytes) + sfbytes * (b_hi ? 3u : 2u));
+                    mma::tma_load_2d(st, &a_map, c * C::kCB, mt * kBM, &full[s]);
+                    mma::tma_load_2d(st + C::kABytes, &b_map, c * C::kCB, nt * kBN, &full[s]);
+                    bulk_load(sfa, a_sf + (int64_t(mt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
+                    bulk_load(sfb, b_sf + (int64_t(2 * nt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
+                    if (b_hi)
+                        bulk_load(sfb + C::kUnits * kSfUnit, b_sf + (int64_t(2 * nt + 1) * Ka + u0) * kSfUnit, sfbytes,
+                                  &full[s]);
                     filled = k + 1;
                 }
             }
             // drain: the copies issued have landed before the CTA may exit
-            for (int kk = (filled > kStages ? filled - kStages : 0); kk < filled; ++kk)
-                if (!mbar_wait(&full[kk % kStages], (kk / kStages) & 1, budget)) {
+            for (int kk = (filled > ST ? filled - ST : 0); kk < filled; ++kk)
+                if (!mbar_wait(&full[kk % ST], (kk / ST) & 1, budget)) {
                     atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
@@ -203,35 +232,36 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 }
                 mma::tc_fence_after();
                 for (int c = 0; c < KC; ++c, ++k) {
-                    const int s = k % kStages;
-                    if (!mbar_wait(&full[s], (k / kStages) & 1, budget)) {
+                    const int s = k % ST;
+                    if (!mbar_wait(&full[s], (k / ST) & 1, budget)) {
                         atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
                     mma::tc_fence_after();
-                    const uint32_t a0 = smem_addr(base + size_t(s) * kStageBytes);
-                    const uint32_t b0 = a0 + kABytes;
-                    const uint32_t sfa = b0 + kBBytes;
-                    const uint32_t sfb = sfa + kSfaBytes;
-                    // units of a missing B row group or past K are stale data;
-                    // they only reach output columns >= N or K steps not issued
+                    const uint32_t a0 = smem_addr(base + size_t(s) * C::kStageBytes);
+                    const uint32_t b0 = a0 + C::kABytes;
+                    const uint32_t sfa = b0 + C::kBBytes;
+                    const uint32_t sfb = sfa + C::kSfaBytes;
+                    const uint32_t tsfa = tmem_base + kSfCol + uint32_t(s) * C::kSfStageCols;   // + 4 u
+                    const uint32_t tsfb = tsfa + 4 * C::kUnits;                               // + 8 u (+ 4: group 1)
+                    // units past K or of a missing B row group are stale data:
+                    // they reach only K steps not issued or output columns >= N
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        tmem_copy_unit(tmem_base + kSfaCol + 4 * u, sfa + u * kSfUnit);
-                        tmem_copy_unit(tmem_base + kSfbCol + 8 * u, sfb + u * kSfUnit);
-                        tmem_copy_unit(tmem_base + kSfbCol + 8 * u + 4, sfb + (2 + u) * kSfUnit);
+                    for (int u = 0; u < C::kUnits; ++u) {
+                        tmem_copy_unit(tsfa + 4 * u, sfa + u * kSfUnit);
+                        tmem_copy_unit(tsfb + 8 * u, sfb + u * kSfUnit);
+                        tmem_copy_unit(tsfb + 8 * u + 4, sfb + (C::kUnits + u) * kSfUnit);
                     }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (c * 4 + j >= KS) break;
-                        const uint32_t sf_id = (j & 1) * 2;
+                    for (int j = 0; j < C::kMmas; ++j) {
+                        if (c * C::kMmas + j >= KS) break;
+                        const uint32_t sf_id = 2 * (j & 1);
                         const uint32_t u = j >> 1;
-                        const uint64_t ad = mma::smem_desc(a0 + j * 32, 1024, mma::kLayoutSw128);
-                        const uint64_t bd = mma::smem_desc(b0 + j * 32, 1024, mma::kLayoutSw128);
-                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(sf_id),
-                                  (tmem_base + kSfaCol + 4 * u) | (sf_id << 30),
-                                  (tmem_base + kSfbCol + 8 * u) | (sf_id << 30), (c | j) != 0);
+                        const uint64_t ad = mma::smem_desc(a0 + j * 32, C::kSbo, C::kLayout);
+                        const uint64_t bd = mma::smem_desc(b0 + j * 32, C::kSbo, C::kLayout);
+                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(sf_id), (tsfa + 4 * u) | (sf_id << 30),
+                                  (tsfb + 8 * u) | (sf_id << 30), (c | j) != 0);
                     }
                     mma::umma_commit(&empty[s]);
                 }
@@ -255,34 +285,73 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 break;
             }
             mma::tc_fence_after();
-            float v[128];
             const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(h * 128);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tmem_ld32_nowait(taddr + 32 * i, v + 32 * i);
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            mma::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-
-            const int row = mt * kBM + q * 32 + lane;
+            const int row0 = mt * kBM + q * 32;
             const int col0 = nt * kBN + h * 128;
-            if (row < M) {
-                if constexpr (F32OUT) {
+            if constexpr (F32OUT) {
+                float v[128];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tmem_ld32_nowait(taddr + 32 * i, v + 32 * i);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                mma::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+                const int row = row0 + lane;
+                if (row < M) {
                     float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + int64_t(row) * N + col0);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (col0 + 4 * i < N) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-                } else {
-                    uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + int64_t(row) * N + col0);
+                }
+            } else {
+                // 64 columns at a time into packed bf16 pairs (keeps 64 + 64 registers live)
+                uint32_t w[64];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (col0 + 8 * i < N)
-                            o[i] = make_uint4(mma::pack_bf16x2(v[8 * i], v[8 * i + 1]),
-                                              mma::pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                              mma::pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
-                                              mma::pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                for (int half = 0; half < 2; ++half) {
+                    float v[64];
+                    tmem_ld32_nowait(taddr + 64 * half, v);
+                    tmem_ld32_nowait(taddr + 64 * half + 32, v + 32);
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[32 * half + i] = mma::pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                }
+                mma::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+                if constexpr (kStaged) {
+                    // the previous tile's stores have finished reading the staging buffer
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    __syncwarp();
+                    uint8_t *stg = stage_out + size_t(warp - 2) * kStageOutBytes;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        // 16-byte chunk i of this lane's row: box i / 8, chunk i % 8
+                        // swizzled by the row (128-byte swizzle: chunk ^ (row % 8))
+                        const int b = i >> 3, cc = i & 7;
+                        *reinterpret_cast<uint4 *>(stg + b * 4096 + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
+                            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    // boxes that start past D are not issued; the rest is clipped
+                    if (lane == 0 && row0 < M && col0 < N) {
+                        mma::tma_store_2d(&out_map, col0, row0, stg);
+                        if (col0 + 64 < N) mma::tma_store_2d(&out_map, col0 + 64, row0, stg + 4096);
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    }
+                } else {
+                    const int row = row0 + lane;
+                    if (row < M) {
+                        uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + int64_t(row) * N + col0);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (col0 + 8 * i < N) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    }
                 }
             }
+        }
+        if constexpr (kStaged) {
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
     }
 
@@ -295,5 +364,14 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                      : "memory");
     }
 }
+
+// Configurations (mxf4_gemm_variant): 1 = 128-byte chunks, 4 stages, stores
+// from registers; 2 = 64-byte chunks, 6 stages, TMA-store epilogue; 3 = 64, 4,
+// TMA stores; 4 = 128, 3, TMA stores; 5 = 64, 8, stores from registers.
+using Cfg1 = Cfg<128, 4, false>;
+using Cfg2 = Cfg<64, 6, true>;
+using Cfg3 = Cfg<64, 4, true>;
+using Cfg4 = Cfg<128, 3, true>;
+using Cfg5 = Cfg<64, 8, false>;
 
 }  // namespace gemm
