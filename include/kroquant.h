@@ -242,7 +242,10 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
  *      exact in the fp32 accumulator), TMA-fed, accumulators in tensor memory,
  *   5  the arithmetic of 2 with the diagonal part of the factors in shared
  *      memory (fewer registers, more resident warps, no prefetch),
- *   6  the arithmetic of 2 with a two-deep register prefetch.
+ *   6  the arithmetic of 2 with a two-deep register prefetch,
+ *   7  the arithmetic of 2 with the input prefetched by cp.async into a
+ *      per-thread shared-memory ring, 3 blocks in flight per thread,
+ *   8  as 7 with 5 blocks in flight.
  * Other values return KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
                         int shared, uint8_t *out_codes, uint8_t *out_scales,

@@ -203,24 +203,24 @@ def test_baseline_variants_bit_exact(cuda_device, M, d):
 
 @pytest.mark.parametrize("M,d", VARIANT_SHAPES, ids=[f"{M}x{d}" for M, d in VARIANT_SHAPES])
 def test_kq_variants_sharing_arithmetic_are_identical(cuda_device, M, d):
-    """Variants 2, 3, 5 and 6 share the arithmetic, so their outputs are identical."""
+    """Variants 2, 3, 5, 6, 7 and 8 share the arithmetic, so their outputs are identical."""
     x = synth.activation("pixart", M, d, seed=M * 3 + d)
     F = synth.factors(d // 32, seed=d + 1)
     xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
     c2, s2 = kq.kq_quantize_variant(2, xd, Fd)
-    for v in (3, 5, 6):
+    for v in (3, 5, 6, 7, 8):
         cv, sv = kq.kq_quantize_variant(v, xd, Fd)
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
     F1 = synth.factors(1, seed=d, shared=True)
     c2, s2 = kq.kq_quantize_variant(2, xd, dev_f32(F1, cuda_device), shared=True)
-    for v in (3, 5, 6):
+    for v in (3, 5, 6, 7, 8):
         cv, sv = kq.kq_quantize_variant(v, xd, dev_f32(F1, cuda_device), shared=True)
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
     # a column that falls back to the direct form (swap factor) alongside split ones
     F2 = F.copy()
     F2[0, 2] = np.array([[0, 1], [1, 0]], np.float32)
     c2, s2 = kq.kq_quantize_variant(2, xd, dev_f32(F2, cuda_device))
-    for v in (3, 5, 6):
+    for v in (3, 5, 6, 7, 8):
         cv, sv = kq.kq_quantize_variant(v, xd, dev_f32(F2, cuda_device))
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
 

@@ -24,7 +24,7 @@ def dev_bf16(bits, device):
     return dev(bits.view(np.int16), device).view(torch.bfloat16)
 
 
-CASES = [(64, 128, 1, False), (37, 96, 1, False), (8192, 1152, 2, False), (2048, 5600, 2, False),
+CASES = [(64, 128, 1, False), (37, 96, 1, False), (8192, 1152, 2, False), (2048, 5600, 2, False), (1000, 4608, 4, False),
          (2048, 2240, 4, True), (512, 12288, 2, False), (300, 4608, 3, False)]
 
 

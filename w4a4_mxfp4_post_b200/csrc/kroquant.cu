@@ -766,6 +766,86 @@ kq_packed2_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ fact
     }
 }
 
+// KroQuant quantizer, variants 7 and 8: the arithmetic of variant 2, with the
+// input prefetched by cp.async into a per-warp ring in shared memory (D steps,
+// D - 1 of them in flight): the copies hold no registers, so the memory-level
+// parallelism does not cost occupancy.  At every step a warp's 32 threads own
+// 32 consecutive blocks (2 KB); the warp copies them cooperatively, each
+// cp.async instruction covering 512 contiguous bytes, into its ring slot with
+// the 16-byte piece p of block b at b * 64 + 16 (p ^ ((b >> 1) & 3)), so the
+// per-thread reads of a block are free of bank conflicts.  The loop is
+// warp-uniform (a warp's first thread has the most steps); a thread without a
+// block at a step only helps copy and synchronise.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *g)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+kq_async_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
+                uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
+{
+    extern __shared__ uint4 ring[];   // [warp][D][128 pieces of 16 bytes]
+    const int lane = threadIdx.x & 31;
+    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t t0 = t - lane;                          // the warp's first thread
+    const bool live = t < T && t < nblocks;
+    const int j = live ? int(t % nb) : 0;
+    KqFast st;
+    bool fast = false;
+    if (live) {
+        float4 g[5];
+        load_factors(factors, shared, j, g);
+        fast = kq_fast_setup(g, st);
+    }
+    uint4 *wring = ring + size_t(threadIdx.x >> 5) * D * 128;
+    const uint32_t wbase = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
+    const int64_t nsteps = (t0 < T && t0 < nblocks) ? (nblocks - t0 + T - 1) / T : 0;   // warp-uniform
+    auto issue = [&](int64_t i, int slot) {
+        const int64_t b0 = t0 + i * T;                    // the warp's first block at step i
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c = q * 32 + lane;                  // piece c of the warp's 2 KB
+            const int b = c >> 2, pc = c & 3;
+            if (t0 + b < T && b0 + b < nblocks)
+                cp_async16(wbase + uint32_t(slot * 2048 + b * 64 + ((pc ^ ((b >> 1) & 3)) << 4)), act + (b0 + b) * 4 + pc);
+        }
+    };
+#pragma unroll
+    for (int s = 0; s < D - 1; ++s) {
+        if (s < nsteps) issue(s, s);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    int slot = 0;
+    for (int64_t i = 0; i < nsteps; ++i) {
+        // one group per step (possibly empty): step i + D - 1 into the slot read at step i - 1
+        if (i + D - 1 < nsteps) issue(i + D - 1, slot == 0 ? D - 1 : slot - 1);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group %0;" ::"n"(D - 1) : "memory");   // step i has landed (own copies)
+        __syncwarp();                                                       // ... and the other lanes'
+        const int64_t gi = t + i * T;
+        if (live && gi < nblocks) {
+            uint4 raw[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) raw[q] = wring[slot * 128 + lane * 4 + (q ^ ((lane >> 1) & 3))];
+            float2 p[16];
+            unpack_pairs(raw, p);
+            if (fast) {
+                kq_fast_apply(p, st);
+            } else {   // rare: the factors are reloaded (L1) rather than kept live
+                float4 g[5];
+                load_factors(factors, shared, j, g);
+                kq_direct_apply(p, g);
+            }
+            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+        }
+        __syncwarp();   // every lane has read the slot before it is refilled
+        slot = slot == D - 1 ? 0 : slot + 1;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // SmoothQuant quantizer on the pair layout: y = fp32(x * m) per channel (one
 // correctly rounded packed multiply), then the MXFP4 block quantizer.
 __global__ void __launch_bounds__(kThreads)
@@ -1340,6 +1420,174 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
     }
 }
 
+// Single-pass form of the fused normalisation + quantizer, used wherever its
+// shared memory fits (the kernel above is the general fallback).  Each CTA
+// owns a contiguous range of rows of one sample; its shared-memory table holds,
+// per column, the transform coefficients (as above) and that sample's 1 + gamma
+// and beta (kNormRowSlot float4, an odd number of 16-byte units; a column in
+// the direct form, which is rare, reloads its raw factors).  Each warp
+// streams whole rows into a ring of nbuf row buffers with cp.async (every
+// instruction of a warp copies 512 contiguous bytes; the 16-byte piece p of
+// block b lands at b * 64 + 16 (p ^ ((b >> 1) & 3)), so the per-lane block
+// reads of the second sweep are free of bank conflicts), the next row in
+// flight while the current one is processed: the row is read from HBM once.
+// From shared memory a warp takes the mean (one sweep), the sum of squared
+// deviations from it (a second sweep: the two-pass variance), then normalises,
+// modulates, transforms and quantizes every block.
+constexpr int kNormRowSlot = 27;   // 8 D + 2 B/C + 1 (b4, c4, flag) + 8 (1 + gamma) + 8 beta
+
+__global__ void __launch_bounds__(512, 1)
+norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
+                    int64_t rows_per, float eps, const float *__restrict__ factors, int shared,
+                    uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int nb, int cps, int nbuf)
+{
+    extern __shared__ float4 smf[];
+    float4 *tab = smf;                                                        // [nb][kNormRowSlot]
+    uint4 *rowbuf = reinterpret_cast<uint4 *>(smf + size_t(nb) * kNormRowSlot);   // [warps][nbuf][nb * 4]
+    const int warps = int(blockDim.x) / 32, wid = int(threadIdx.x) / 32, lane = int(threadIdx.x) & 31;
+    const int64_t smp = blockIdx.x / cps;
+    const int part = int(blockIdx.x % cps);
+    const int64_t r0 = smp * rows_per + rows_per * part / cps;
+    const int64_t r1 = smp * rows_per + rows_per * (part + 1) / cps;
+    const int d = nb * kBlk;
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+        float4 g[5];
+        load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
+        KqFast st;
+        const bool fast = kq_fast_setup(g, st);
+        float4 *e = tab + size_t(j) * kNormRowSlot;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            e[q] = make_float4(st.DP[2 * q].x, st.DP[2 * q].y, st.DP[2 * q + 1].x, st.DP[2 * q + 1].y);
+        e[8] = make_float4(st.B[0], st.C[0], st.B[1], st.C[1]);
+        e[9] = make_float4(st.B[2], st.C[2], st.B[3], st.C[3]);
+        e[10] = make_float4(st.b4, st.c4, fast ? 1.0f : 0.0f, 0.0f);
+        const float4 *gp = reinterpret_cast<const float4 *>(gamma + smp * d + int64_t(j) * kBlk);
+        const float4 *bp = reinterpret_cast<const float4 *>(beta + smp * d + int64_t(j) * kBlk);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 ga = __ldg(gp + q);
+            e[11 + q] = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
+            e[19 + q] = __ldg(bp + q);
+        }
+    }
+    __syncthreads();
+
+    const int npieces = nb * 4;                                   // 16-byte pieces per row
+    uint4 *wbuf = rowbuf + size_t(wid) * nbuf * npieces;
+    const uint32_t wbase = static_cast<uint32_t>(__cvta_generic_to_shared(wbuf));
+    const int64_t nrows = (r1 - r0 > wid) ? (r1 - r0 - wid + warps - 1) / warps : 0;   // this warp's rows
+    // Piece c = lane + 32 k is piece (lane & 3) of block (lane >> 2) + 8 k, whose
+    // swizzle term ((block >> 1) & 3) = (lane >> 3) & 3 does not depend on k: a
+    // lane's pieces sit at a fixed offset plus 512 k bytes.
+    const int lslot = (lane & ~3) + ((lane & 3) ^ ((lane >> 3) & 3));
+    const int nk = (npieces - lane + 31) / 32;                    // this lane's pieces per row
+    auto issue = [&](int64_t r, int buf) {
+        const uint4 *src = h + r * npieces + lane;
+        uint32_t dst = wbase + uint32_t((buf * npieces + lslot) * 16);
+        for (int k = 0; k < nk; ++k, src += 32, dst += 512) cp_async16(dst, src);
+    };
+    if (nrows > 0) issue(r0 + wid, 0);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t r = r0 + wid + i * warps;
+        const int buf = nbuf == 2 ? int(i & 1) : 0;
+        if (nbuf == 2) {
+            if (i + 1 < nrows) issue(r + warps, buf ^ 1);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            if (i > 0) {
+                issue(r, 0);
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            }
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncwarp();
+        const uint4 *rb = wbuf + size_t(buf) * npieces;
+        // ---- statistics: mean, then the sum of squared deviations from it
+        const uint4 *lp = rb + lslot;                             // this lane's pieces, 32 apart
+        float2 s2 = make_float2(0.0f, 0.0f);
+        for (int k = 0; k < nk; ++k) {
+            const uint4 w = lp[32 * k];
+            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.x), bf16_hi(w.x)));
+            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.y), bf16_hi(w.y)));
+            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.z), bf16_hi(w.z)));
+            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.w), bf16_hi(w.w)));
+        }
+        float sum = s2.x + s2.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float mu = sum / float(d);
+        const float2 nmu = make_float2(-mu, -mu);
+        float2 q2 = make_float2(0.0f, 0.0f);
+        for (int k = 0; k < nk; ++k) {
+            const uint4 w = lp[32 * k];
+            float2 t;
+            t = __fadd2_rn(make_float2(bf16_lo(w.x), bf16_hi(w.x)), nmu);
+            q2 = __ffma2_rn(t, t, q2);
+            t = __fadd2_rn(make_float2(bf16_lo(w.y), bf16_hi(w.y)), nmu);
+            q2 = __ffma2_rn(t, t, q2);
+            t = __fadd2_rn(make_float2(bf16_lo(w.z), bf16_hi(w.z)), nmu);
+            q2 = __ffma2_rn(t, t, q2);
+            t = __fadd2_rn(make_float2(bf16_lo(w.w), bf16_hi(w.w)), nmu);
+            q2 = __ffma2_rn(t, t, q2);
+        }
+        float m2 = q2.x + q2.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+        const float inv = 1.0f / sqrtf(m2 / float(d) + eps);
+        const float2 iv = make_float2(inv, inv);
+        // ---- normalise, modulate, transform, quantize
+        for (int jb = lane; jb < nb; jb += 32) {
+            uint4 raw[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) raw[q] = rb[jb * 4 + (q ^ ((jb >> 1) & 3))];
+            float2 p[16];
+            unpack_pairs(raw, p);
+            const float4 *eq = tab + size_t(jb) * kNormRowSlot;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 ga = eq[11 + q4], gb = eq[15 + q4], ba = eq[19 + q4], bb = eq[23 + q4];
+                const float g_lo[4] = {ga.x, ga.y, ga.z, ga.w}, g_hi[4] = {gb.x, gb.y, gb.z, gb.w};
+                const float b_lo[4] = {ba.x, ba.y, ba.z, ba.w}, b_hi[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i2 = 4 * q4 + e;
+                    const float2 t = __fmul2_rn(__fadd2_rn(p[i2], nmu), iv);
+                    p[i2] = __ffma2_rn(t, make_float2(g_lo[e], g_hi[e]), make_float2(b_lo[e], b_hi[e]));
+                }
+            }
+            const float4 c4q = eq[10];
+            if (c4q.z != 0.0f) {
+                const float4 c01 = eq[8], c23 = eq[9];
+                unit_stage2<1>(p, bcast(c01.x), bcast(c01.y));
+                unit_stage2<2>(p, bcast(c01.z), bcast(c01.w));
+                unit_stage2<4>(p, bcast(c23.x), bcast(c23.y));
+                unit_stage2<8>(p, bcast(c23.z), bcast(c23.w));
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 dd = eq[q];   // (D_2q, D_2q+16, D_2q+1, D_2q+17)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int i2 = 2 * q + h2;
+                        const float lo = p[i2].x, hi = p[i2].y;
+                        const float2 dp = h2 ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y);
+                        p[i2] = __ffma2_rn(make_float2(fmaf(c4q.x, hi, lo), fmaf(c4q.y, lo, hi)), dp, plus_zero2());
+                    }
+                }
+            } else {   // rare: the raw factors, from L1
+                float4 g[5];
+                load_factors(reinterpret_cast<const float4 *>(factors), shared, jb, g);
+                kq_direct_apply(p, g);
+            }
+            kq_emit<KqOut::kCodes>(p, r * nb + jb, codes, scales, nullptr);
+        }
+        __syncwarp();   // every lane is done with the buffer before it is refilled
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 #include "kq_mma.cuh"
 #include "mxf4_gemm.cuh"
 
@@ -1395,7 +1643,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
     kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2,
-    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kNumKernels
+    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kKqAsync4, kKqAsync6, kNormRows, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1485,6 +1733,8 @@ int encode_act_map(const void *act, int64_t nblocks, CUtensorMap *map)
 }
 
 std::atomic<int> g_smem_set[kNumKernels][kMaxDevices];
+constexpr size_t kNormRowsSmemMax = size_t(227) * 1024;
+std::atomic<int> g_norm_cfg[kMaxDevices][513];   // chosen single-pass norm configuration per row width
 
 // Dynamic shared memory above 48 KB needs an opt-in per kernel and device.
 int staged_prepare(KernelId id, const void *fn, int64_t *ctas_total)
@@ -1644,6 +1894,28 @@ constexpr long long kWaitBudget = 1LL << 31;
 // Largest block count the staged path takes (row coordinates are int32).
 constexpr int64_t kStagedMaxBlocks = (int64_t(1) << 31) - kStageRows;
 
+// As launch_pinned, for a kernel with dynamic shared memory (the occupancy
+// query then accounts for it).
+template <typename Kernel>
+int launch_pinned_smem(const char *fn, KernelId id, Kernel kernel, size_t smem, int64_t M, int64_t nb, Geometry *geo)
+{
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    int c = (dev >= 0 && dev < kMaxDevices) ? g_ctas_per_sm[id][dev].load(std::memory_order_relaxed) : 0;
+    if (c <= 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, reinterpret_cast<const void *>(kernel), kThreads, smem);
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "%s: occupancy query: %s", fn, cudaGetErrorString(e));
+        if (c < 1) c = 1;
+        if (dev >= 0 && dev < kMaxDevices) g_ctas_per_sm[id][dev].store(c, std::memory_order_relaxed);
+    }
+    *geo = pinned_geometry(M, nb, int64_t(sms) * c * kThreads);
+    return KQ_OK;
+}
+
 template <typename Kernel>
 int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t nb, Geometry *geo)
 {
@@ -1671,8 +1943,22 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
     if (variant == 0) variant = kDefaultVariant;
-    if (variant < 1 || variant > 6)
+    if (variant < 1 || variant > 8)
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
+    if ((variant == 7 || variant == 8) && !f32) {
+        const int64_t nb7 = d / kBlk;
+        const int depth = variant == 7 ? 4 : 6;
+        auto k = variant == 7 ? kq_async_kernel<4> : kq_async_kernel<6>;
+        const KernelId id = variant == 7 ? kKqAsync4 : kKqAsync6;
+        const size_t smem = size_t(depth) * kThreads * 64;   // per warp depth x 2 KB
+        if ((rc = smem_prepare(id, reinterpret_cast<const void *>(k), smem)) != KQ_OK) return rc;
+        Geometry geo;
+        if ((rc = launch_pinned_smem(fn, id, k, smem, M, nb7, &geo)) != KQ_OK) return rc;
+        k<<<geo.grid, kThreads, smem, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
+                                                shared, reinterpret_cast<uint4 *>(codes), scales, M * nb7, int(nb7), geo.T);
+        return launch_check(fn);
+    }
+    if (variant == 7 || variant == 8) variant = 2;   // the fp32 export: the same arithmetic in variant 2
     if (variant == 6 && !f32) {
         const int64_t nb6 = d / kBlk;
         Geometry geo;
@@ -2053,6 +2339,53 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, 
         !aligned(beta, 16))
         return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
     const int nb = int(d / kBlk);
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    {
+        // single-pass kernel: the first (warps, row buffers) whose shared memory
+        // fits, chosen once per device and row width (cached: warps << 8 | nbuf
+        // << 4 | CTAs per SM; -1 = none fits)
+        int devc = 0;
+        cudaError_t e2 = cudaGetDevice(&devc);
+        if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e2));
+        const size_t tab = size_t(nb) * kNormRowSlot * 16, row = size_t(nb) * 64;
+        int packed = (devc >= 0 && devc < kMaxDevices) ? g_norm_cfg[devc][nb].load(std::memory_order_acquire) : 0;
+        if (packed == 0) {
+            packed = -1;
+            e2 = cudaFuncSetAttribute(norm_kq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(kNormRowsSmemMax));
+            if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e2));
+            // fewer than 4 row buffers per CTA would leave the SM nearly idle: the
+            // fallback kernel is then faster
+            const int cfg[7][2] = {{16, 1}, {8, 2}, {12, 1}, {4, 2}, {8, 1}, {2, 2}, {4, 1}};
+            for (const auto &c : cfg) {
+                const size_t smem_r = tab + size_t(c[0]) * c[1] * row;
+                if (smem_r > kNormRowsSmemMax) continue;
+                int per_sm = 0;
+                e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_rows_kernel, 32 * c[0], smem_r);
+                if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e2));
+                if (per_sm < 1) continue;
+                packed = (c[0] << 8) | (c[1] << 4) | (per_sm > 15 ? 15 : per_sm);
+                break;
+            }
+            if (devc >= 0 && devc < kMaxDevices) g_norm_cfg[devc][nb].store(packed, std::memory_order_release);
+        }
+        if (packed > 0) {
+            const int warps = packed >> 8, nbuf = (packed >> 4) & 15, per_sm = packed & 15;
+            const int64_t rows_per = M / nsamples;
+            int64_t cps = int64_t(sms) * per_sm / nsamples;
+            const int64_t most = rows_per / warps;          // at least one row per warp per CTA
+            if (cps > most) cps = most;
+            if (cps < 1) cps = 1;
+            if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
+            const size_t smem_r = tab + size_t(warps) * nbuf * row;
+            norm_kq_rows_kernel<<<unsigned(cps * nsamples), 32 * warps, smem_r, stream>>>(
+                static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps, factors, shared ? 1 : 0,
+                reinterpret_cast<uint4 *>(out_codes), out_scales, nb, int(cps), nbuf);
+            return launch_check(fn);
+        }
+    }
     const size_t smem = size_t(nb) * kNormSlot * sizeof(float);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -2063,9 +2396,6 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, 
         if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         if (dev >= 0 && dev < kMaxDevices) g_smem_set[kNormKq][dev].store(1);
     }
-    int sms = 0;
-    int rc = sm_count(&sms);
-    if (rc != KQ_OK) return rc;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel, kThreads, smem);
     if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
