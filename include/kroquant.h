@@ -211,14 +211,17 @@ int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf,
               void *out, int out_f32, int64_t M, int64_t N, int64_t K,
               cudaStream_t stream);
 
-/* Test export: mxf4_gemm through a chosen tile configuration (all 128 x 256
- * output tiles, one CTA per SM; a k-chunk is CB bytes of codes per row):
- *   0  the default (what mxf4_gemm runs: 4),
+/* Test export: mxf4_gemm through a chosen tile configuration (128 x 256
+ * output tiles unless stated, one CTA per SM; a k-chunk is CB bytes of codes
+ * per row):
+ *   0  the default (what mxf4_gemm runs: 4, or 6 where 256-column tiles
+ *      fill the last wave of SMs badly),
  *   1  CB = 128, 4 stages, epilogue stores from registers,
  *   2  CB = 64, 6 stages, bf16 epilogue through shared memory and TMA stores,
  *   3  CB = 64, 4 stages, TMA stores,
  *   4  CB = 128, 3 stages, TMA stores,
- *   5  CB = 64, 8 stages, stores from registers.
+ *   5  CB = 64, 8 stages, stores from registers,
+ *   6  as 4 with 192-column tiles.
  * Same results for every configuration (the K order of the MMAs is the same).
  * Other values return KQ_ERR_VARIANT. */
 int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf,

@@ -144,7 +144,7 @@ def test_mxf4_gemm_configurations_agree(cuda_device, M, N, K):
     for dtype in (torch.float32, torch.bfloat16):
         ref = kq.mxf4_gemm_variant(1, *args, out_dtype=dtype)
         check_gemm(ref.float().cpu().numpy(), D, absd, K, dtype == torch.bfloat16)
-        for v in (0, 2, 3, 4, 5):
+        for v in (0, 2, 3, 4, 5, 6):
             got = kq.mxf4_gemm_variant(v, *args, out_dtype=dtype)
             assert torch.equal(got, ref), (v, dtype)
 

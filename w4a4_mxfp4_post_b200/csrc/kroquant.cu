@@ -1868,20 +1868,22 @@ int encode_gemm_map(const void *codes, int64_t rows, int64_t K, int cb, int box_
     return KQ_OK;
 }
 
-// The bf16 output D [M][N] of the W4A4 product: boxes of {64 columns x 32
-// rows} (one epilogue warp's half row segment), 128-byte swizzle.
-int encode_gemm_out_map(void *out, int64_t M, int64_t N, CUtensorMap *map)
+// The bf16 output D [M][N] of the W4A4 product: boxes of {box_cols x 32 rows}
+// (part of one epilogue warp's row segment), 128-byte swizzle for 64 columns,
+// 64-byte swizzle for 32.
+int encode_gemm_out_map(void *out, int64_t M, int64_t N, int box_cols, CUtensorMap *map)
 {
     EncodeTiledFn enc;
     int rc = encode_fn(&enc);
     if (rc != KQ_OK) return rc;
     const cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
     const cuuint64_t strides[1] = {cuuint64_t(N) * 2};
-    const cuuint32_t box[2] = {64, 32};
+    const cuuint32_t box[2] = {cuuint32_t(box_cols), 32};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
     return KQ_OK;
 }
@@ -2057,11 +2059,20 @@ struct GemmArgs {
     const uint8_t *a_codes, *a_sf, *b_codes, *b_sf;
     void *out;
     bool f32;
-    int64_t M, N, K, tiles;
+    int64_t M, N, K;
     cudaStream_t stream;
 };
 
-constexpr int kDefaultGemmVariant = 4;
+// Default tile configuration: 4 (256-column tiles) or 6 (192-column tiles),
+// whichever the cost model waves x (128 + BN) -- rounds of one tile per SM,
+// each moving A and B rows -- rates cheaper.
+int default_gemm_variant(int64_t M, int64_t N, int sms)
+{
+    const int64_t mt = (M + gemm::kBM - 1) / gemm::kBM;
+    const int64_t w256 = (mt * ((N + 255) / 256) + sms - 1) / sms;
+    const int64_t w192 = (mt * ((N + 191) / 192) + sms - 1) / sms;
+    return w192 * (128 + 192) < w256 * (128 + 256) ? 6 : 4;
+}
 
 template <class C, bool F32>
 std::atomic<int> g_gemm_smem_set[kMaxDevices];
@@ -2087,19 +2098,21 @@ int gemm_launch_out(const GemmArgs &g, const CUtensorMap &amap, const CUtensorMa
 template <class C>
 int gemm_launch(const GemmArgs &g)
 {
+    const int64_t tiles = ((g.M + gemm::kBM - 1) / gemm::kBM) * ((g.N + C::kBN - 1) / C::kBN);
+    if (tiles >= (int64_t(1) << 31)) return fail(KQ_ERR_SHAPE, "mxf4_gemm: too many output tiles");
     CUtensorMap amap, bmap, omap;
     int rc = encode_gemm_map(g.a_codes, g.M, g.K, C::kCB, gemm::kBM, &amap);
     if (rc != KQ_OK) return rc;
-    if ((rc = encode_gemm_map(g.b_codes, g.N, g.K, C::kCB, gemm::kBN, &bmap)) != KQ_OK) return rc;
+    if ((rc = encode_gemm_map(g.b_codes, g.N, g.K, C::kCB, C::kBN, &bmap)) != KQ_OK) return rc;
     // only the TMA-store epilogue reads the output map; the others get a placeholder
     if (C::kTmaOut && !g.f32) {
-        if ((rc = encode_gemm_out_map(g.out, g.M, g.N, &omap)) != KQ_OK) return rc;
+        if ((rc = encode_gemm_out_map(g.out, g.M, g.N, C::kBN == 256 ? 64 : 32, &omap)) != KQ_OK) return rc;
     } else {
         omap = amap;
     }
     int sms = 0;
     if ((rc = sm_count(&sms)) != KQ_OK) return rc;
-    const unsigned grid = unsigned(g.tiles < sms ? g.tiles : sms);
+    const unsigned grid = unsigned(tiles < sms ? tiles : sms);
     return g.f32 ? gemm_launch_out<C, true>(g, amap, bmap, omap, grid) : gemm_launch_out<C, false>(g, amap, bmap, omap, grid);
 }
 
@@ -2482,22 +2495,26 @@ int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf, 
                     "(M=%lld, N=%lld, K=%lld)", fn, (long long)M, (long long)N, (long long)K);
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return fail(KQ_ERR_SHAPE, "%s: M, N and K must be below 2^31", fn);
-    if (variant == 0) variant = kDefaultGemmVariant;
-    if (variant < 1 || variant > 5) return fail(KQ_ERR_VARIANT, "%s: variant %d is not available", fn, variant);
+    if (variant < 0 || variant > 6) return fail(KQ_ERR_VARIANT, "%s: variant %d is not available", fn, variant);
     if (M == 0 || N == 0) return ok();
     if (!a_codes || !a_sf || !b_codes || !b_sf || !out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
     if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
         !aligned(out, 16))
         return fail(KQ_ERR_ALIGN, "%s: every pointer must be 16-byte aligned", fn);
-    const int64_t tiles = ((M + gemm::kBM - 1) / gemm::kBM) * ((N + gemm::kBN - 1) / gemm::kBN);
-    if (tiles >= (int64_t(1) << 31)) return fail(KQ_ERR_SHAPE, "%s: too many output tiles", fn);
-    const GemmArgs g{a_codes, a_sf, b_codes, b_sf, out, out_f32 != 0, M, N, K, tiles, stream};
+    if (variant == 0) {
+        int sms = 0;
+        int rc = sm_count(&sms);
+        if (rc != KQ_OK) return rc;
+        variant = default_gemm_variant(M, N, sms);
+    }
+    const GemmArgs g{a_codes, a_sf, b_codes, b_sf, out, out_f32 != 0, M, N, K, stream};
     switch (variant) {
     case 1: return gemm_launch<gemm::Cfg1>(g);
     case 2: return gemm_launch<gemm::Cfg2>(g);
     case 3: return gemm_launch<gemm::Cfg3>(g);
     case 4: return gemm_launch<gemm::Cfg4>(g);
-    default: return gemm_launch<gemm::Cfg5>(g);
+    case 5: return gemm_launch<gemm::Cfg5>(g);
+    default: return gemm_launch<gemm::Cfg6>(g);
     }
 }
 

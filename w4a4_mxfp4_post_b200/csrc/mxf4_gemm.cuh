@@ -45,53 +45,59 @@
 namespace gemm {
 
 constexpr int kBM = 128;                                  // tile rows (MMA M)
-constexpr int kBN = 256;                                  // tile columns (MMA N)
 constexpr int kSfUnit = 512;                              // 128 rows x 4 blocks
 constexpr int kTmemCols = 512;                            // power of two >= 256 + scale columns
 constexpr uint32_t kAccCol = 0;                           // 256 fp32 accumulator columns
-constexpr uint32_t kSfCol = 256;                          // scale columns, per stage
+constexpr uint32_t kSfCol = 256;                          // scale columns: 16 per stage and k-unit
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;             // 320
 constexpr int kStageOutBytes = 32 * 128 * 2;              // a warp's 32 rows x 128 bf16 columns
 constexpr size_t kSmemMax = 232448;                       // 227 KB per CTA
 
 // Tile configuration: CB codes bytes per row per k-chunk (64 or 128), ST ring
-// stages, TMA_OUT = bf16 output through shared memory and TMA stores.
-template <int CB, int ST, bool TMA_OUT>
+// stages, TMA_OUT = bf16 output through shared memory and TMA stores, BN tile
+// columns (256, or 192 where 256-column tiles fill the last wave badly).
+// Scale columns per stage and k-unit: A's unit at +0, B's two units at +8 and
+// +12 (every tcgen05.cp destination a multiple of 4 columns).  A 192-column
+// tile may start in the middle of a 128-row scale unit (odd tiles start at its
+// third 32-row group): the MMA then reads B's scales from +10 instead of +8.
+template <int CB, int ST, bool TMA_OUT, int BN = 256>
 struct Cfg {
     static constexpr int kCB = CB;
     static constexpr int kST = ST;
     static constexpr bool kTmaOut = TMA_OUT;
+    static constexpr int kBN = BN;
     static constexpr int kUnits = CB / 64;                // scale units per row group per chunk
     static constexpr int kMmas = CB / 32;                 // K=64 MMAs per chunk
     static constexpr int kABytes = kBM * CB;
-    static constexpr int kBBytes = kBN * CB;
+    static constexpr int kBBytes = BN * CB;
     static constexpr int kSfaBytes = kUnits * kSfUnit;
     static constexpr int kSfbBytes = 2 * kUnits * kSfUnit;
     static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-    static constexpr uint32_t kSfStageCols = 12 * kUnits; // A: 4 per unit, B: 8 per unit
+    static constexpr uint32_t kSfStageCols = 16 * kUnits;
+    static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (1u << 23) |
+                                       (uint32_t(kBM >> 4) << 24);
+    static constexpr int kEpiCols = BN / 2;               // columns per epilogue warp
     static constexpr uint64_t kLayout = CB == 128 ? mma::kLayoutSw128 : mma::kLayoutSw64;
     static constexpr uint32_t kSbo = 8 * CB;              // 8-row swizzle atom
     static constexpr size_t kRing = size_t(ST) * kStageBytes;
     static constexpr size_t kSmem = kRing + (TMA_OUT ? size_t(kEpiWarps) * kStageOutBytes : 0) + 1024 +
                                     (2 * ST + 4) * sizeof(uint64_t) + 16;
     static_assert(CB == 64 || CB == 128, "chunk bytes");
+    static_assert(BN == 256 || BN == 192, "tile columns");
     static_assert(kStageBytes % (8 * CB) == 0, "stages keep the alignment of the swizzle atom");
     static_assert(!TMA_OUT || kRing % 1024 == 0, "the output staging keeps the 1 KB alignment of its swizzle");
     static_assert(kSfCol + ST * kSfStageCols <= kTmemCols, "tensor memory columns");
     static_assert(kSmem <= kSmemMax, "shared memory");
 };
 
-// Instruction descriptor, block-scaled kinds: b_sf_id bits 4-5, A format
-// bits 7-9 and B format bits 10-12 (1 = E2M1 for kind::mxf4), K-major A and B
-// (bits 15, 16 = 0), N >> 3 in bits 17-22, scale format bit 23 (1 = E8M0),
-// M >> 4 in bits 24-28, a_sf_id bits 29-30, bit 31 = 0 (K = 64).
-constexpr uint32_t kIdescBase =
-    (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24);
-
+// Instruction descriptor (Cfg::kIdesc), block-scaled kinds: b_sf_id bits 4-5,
+// A format bits 7-9 and B format bits 10-12 (1 = E2M1 for kind::mxf4),
+// K-major A and B (bits 15, 16 = 0), N >> 3 in bits 17-22, scale format bit 23
+// (1 = E8M0), M >> 4 in bits 24-28, a_sf_id bits 29-30, bit 31 = 0 (K = 64).
 // sf_id selects the byte pair of each 32-bit scale word: the K=64 step j of a
 // 128-element unit reads blocks 2j and 2j+1, i.e. bytes 2j, 2j+1 (sf_id 2j).
-__device__ __forceinline__ uint32_t idesc(uint32_t sf_id) { return kIdescBase | (sf_id << 4) | (sf_id << 29); }
+__device__ __forceinline__ uint32_t idesc(uint32_t base, uint32_t sf_id) { return base | (sf_id << 4) | (sf_id << 29); }
 
 __device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t id,
                                           uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate)
@@ -139,6 +145,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                  const uint8_t *__restrict__ b_sf, void *__restrict__ out, int M, int N, int K, long long budget)
 {
     constexpr int ST = C::kST;
+    constexpr int kBN = C::kBN;
     constexpr bool kStaged = C::kTmaOut && !F32OUT;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -188,7 +195,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 const int mt = t / NT, nt = t % NT;
-                const bool b_hi = 2 * nt + 1 < NRa;        // the tile's second B row group exists
+                const int g0 = nt * kBN / 128;                // first B row group of the tile
+                const bool b_hi = g0 + 1 < NRa;               // its second row group exists
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
                     if (k >= ST && !mbar_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
@@ -206,9 +214,9 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     mma::tma_load_2d(st, &a_map, c * C::kCB, mt * kBM, &full[s]);
                     mma::tma_load_2d(st + C::kABytes, &b_map, c * C::kCB, nt * kBN, &full[s]);
                     bulk_load(sfa, a_sf + (int64_t(mt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
-                    bulk_load(sfb, b_sf + (int64_t(2 * nt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
+                    bulk_load(sfb, b_sf + (int64_t(g0) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
                     if (b_hi)
-                        bulk_load(sfb + C::kUnits * kSfUnit, b_sf + (int64_t(2 * nt + 1) * Ka + u0) * kSfUnit, sfbytes,
+                        bulk_load(sfb + C::kUnits * kSfUnit, b_sf + (int64_t(g0 + 1) * Ka + u0) * kSfUnit, sfbytes,
                                   &full[s]);
                     filled = k + 1;
                 }
@@ -226,6 +234,9 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
             int k = 0, it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+                // a tile starting mid-unit (192-column tiles): the MMA reads B's
+                // scales off = 0 or 2 columns (32-row groups) into the first unit
+                const uint32_t off = uint32_t(((t % NT) * kBN % 128) / 32);
                 if (it > 0 && !mbar_wait(acc_empty, (it - 1) & 1, budget)) {
                     atomicAdd(&g_wait_timeouts, 1);
                     break;
@@ -243,15 +254,14 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     const uint32_t b0 = a0 + C::kABytes;
                     const uint32_t sfa = b0 + C::kBBytes;
                     const uint32_t sfb = sfa + C::kSfaBytes;
-                    const uint32_t tsfa = tmem_base + kSfCol + uint32_t(s) * C::kSfStageCols;   // + 4 u
-                    const uint32_t tsfb = tsfa + 4 * C::kUnits;                               // + 8 u (+ 4: group 1)
+                    const uint32_t tsf = tmem_base + kSfCol + uint32_t(s) * C::kSfStageCols;   // + 16 u
                     // units past K or of a missing B row group are stale data:
                     // they reach only K steps not issued or output columns >= N
 #pragma unroll
                     for (int u = 0; u < C::kUnits; ++u) {
-                        tmem_copy_unit(tsfa + 4 * u, sfa + u * kSfUnit);
-                        tmem_copy_unit(tsfb + 8 * u, sfb + u * kSfUnit);
-                        tmem_copy_unit(tsfb + 8 * u + 4, sfb + (C::kUnits + u) * kSfUnit);
+                        tmem_copy_unit(tsf + 16 * u, sfa + u * kSfUnit);
+                        tmem_copy_unit(tsf + 16 * u + 8, sfb + u * kSfUnit);
+                        tmem_copy_unit(tsf + 16 * u + 12, sfb + (C::kUnits + u) * kSfUnit);
                     }
 #pragma unroll
                     for (int j = 0; j < C::kMmas; ++j) {
@@ -260,8 +270,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                         const uint32_t u = j >> 1;
                         const uint64_t ad = mma::smem_desc(a0 + j * 32, C::kSbo, C::kLayout);
                         const uint64_t bd = mma::smem_desc(b0 + j * 32, C::kSbo, C::kLayout);
-                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(sf_id), (tsfa + 4 * u) | (sf_id << 30),
-                                  (tsfb + 8 * u) | (sf_id << 30), (c | j) != 0);
+                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(C::kIdesc, sf_id), (tsf + 16 * u) | (sf_id << 30),
+                                  (tsf + 16 * u + 8 + off) | (sf_id << 30), (c | j) != 0);
                     }
                     mma::umma_commit(&empty[s]);
                 }
@@ -285,13 +295,14 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 break;
             }
             mma::tc_fence_after();
-            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(h * 128);
+            constexpr int EC = C::kEpiCols;           // 128 or 96 columns per warp
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(h * EC);
             const int row0 = mt * kBM + q * 32;
-            const int col0 = nt * kBN + h * 128;
+            const int col0 = nt * kBN + h * EC;
             if constexpr (F32OUT) {
-                float v[128];
+                float v[EC];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) tmem_ld32_nowait(taddr + 32 * i, v + 32 * i);
+                for (int i = 0; i < EC / 32; ++i) tmem_ld32_nowait(taddr + 32 * i, v + 32 * i);
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 mma::tc_fence_before();
                 __syncwarp();
@@ -300,20 +311,19 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 if (row < M) {
                     float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + int64_t(row) * N + col0);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
+                    for (int i = 0; i < EC / 4; ++i)
                         if (col0 + 4 * i < N) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
             } else {
-                // 64 columns at a time into packed bf16 pairs (keeps 64 + 64 registers live)
-                uint32_t w[64];
+                // 32 columns at a time into packed bf16 pairs
+                uint32_t w[EC / 2];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float v[64];
-                    tmem_ld32_nowait(taddr + 64 * half, v);
-                    tmem_ld32_nowait(taddr + 64 * half + 32, v + 32);
+                for (int i = 0; i < EC / 32; ++i) {
+                    float v[32];
+                    tmem_ld32_nowait(taddr + 32 * i, v);
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) w[32 * half + i] = mma::pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    for (int e = 0; e < 16; ++e) w[16 * i + e] = mma::pack_bf16x2(v[2 * e], v[2 * e + 1]);
                 }
                 mma::tc_fence_before();
                 __syncwarp();
@@ -323,20 +333,31 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                     __syncwarp();
                     uint8_t *stg = stage_out + size_t(warp - 2) * kStageOutBytes;
+                    if constexpr (EC == 128) {
+                        // two boxes of 64 columns, 128-byte swizzle: chunk ^ (row % 8)
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        // 16-byte chunk i of this lane's row: box i / 8, chunk i % 8
-                        // swizzled by the row (128-byte swizzle: chunk ^ (row % 8))
-                        const int b = i >> 3, cc = i & 7;
-                        *reinterpret_cast<uint4 *>(stg + b * 4096 + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
-                            make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        for (int i = 0; i < 16; ++i) {
+                            const int bx = i >> 3, cc = i & 7;
+                            *reinterpret_cast<uint4 *>(stg + bx * 4096 + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
+                                make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        }
+                    } else {
+                        // three boxes of 32 columns, 64-byte swizzle: chunk ^ ((row / 2) % 4)
+#pragma unroll
+                        for (int i = 0; i < 12; ++i) {
+                            const int bx = i >> 2, cc = i & 3;
+                            *reinterpret_cast<uint4 *>(stg + bx * 2048 + lane * 64 + ((cc ^ ((lane >> 1) & 3)) << 4)) =
+                                make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        }
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     // boxes that start past D are not issued; the rest is clipped
                     if (lane == 0 && row0 < M && col0 < N) {
-                        mma::tma_store_2d(&out_map, col0, row0, stg);
-                        if (col0 + 64 < N) mma::tma_store_2d(&out_map, col0 + 64, row0, stg + 4096);
+                        constexpr int BW = EC == 128 ? 64 : 32;            // box width (columns)
+#pragma unroll
+                        for (int bx = 0; bx < EC / BW; ++bx)
+                            if (col0 + BW * bx < N) mma::tma_store_2d(&out_map, col0 + BW * bx, row0, stg + bx * BW * 64);
                         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                     }
                 } else {
@@ -344,7 +365,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     if (row < M) {
                         uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + int64_t(row) * N + col0);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
+                        for (int i = 0; i < EC / 8; ++i)
                             if (col0 + 8 * i < N) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                     }
                 }
@@ -367,11 +388,13 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
 
 // Configurations (mxf4_gemm_variant): 1 = 128-byte chunks, 4 stages, stores
 // from registers; 2 = 64-byte chunks, 6 stages, TMA-store epilogue; 3 = 64, 4,
-// TMA stores; 4 = 128, 3, TMA stores; 5 = 64, 8, stores from registers.
+// TMA stores; 4 = 128, 3, TMA stores; 5 = 64, 8, stores from registers;
+// 6 = as 4 with 192-column tiles.
 using Cfg1 = Cfg<128, 4, false>;
 using Cfg2 = Cfg<64, 6, true>;
 using Cfg3 = Cfg<64, 4, true>;
 using Cfg4 = Cfg<128, 3, true>;
 using Cfg5 = Cfg<64, 8, false>;
+using Cfg6 = Cfg<128, 3, true, 192>;
 
 }  // namespace gemm
