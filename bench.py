@@ -703,11 +703,29 @@ def gemm_mode(args):
     first = f"v{variants[0]}"
     tflops = flops / (res[first] * 1e-6) / 1e12
     out_bytes = M * N * 2 + M * K // 2 + N * K // 2
-    print(json.dumps({"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets,
-                      "gemm_us": {k: round(v, 3) for k, v in res.items() if k != "chain"},
-                      "chain_us": round(res["chain"], 3), "tflops": round(tflops, 1), "peak_tflops": peak,
-                      "frac_of_peak": round(tflops / peak, 4), "peak_source": src,
-                      "hbm_gbs_min_bytes": round(out_bytes / (res[first] * 1e-6) / 1e9, 1)}), flush=True)
+    line = {"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets,
+            "gemm_us": {k: round(v, 3) for k, v in res.items() if k != "chain"},
+            "chain_us": round(res["chain"], 3), "tflops": round(tflops, 1), "peak_tflops": peak,
+            "frac_of_peak": round(tflops / peak, 4), "peak_source": src,
+            "hbm_gbs_min_bytes": round(out_bytes / (res[first] * 1e-6) / 1e9, 1)}
+    if args.cpu_seconds > 0:
+        # the oracle's product (double, OpenMP over rows) on a row sample of the
+        # same operands, quantized by the oracle
+        import oracle
+
+        wc, ws = oracle.mx_quantize_f32(Wf.cpu().numpy())
+        xc, xs = oracle.kq_quantize(x[: min(M, 64)], F)
+        t0 = time.perf_counter()
+        n = 0
+        while n < xc.shape[0] and time.perf_counter() - t0 < min(args.cpu_seconds, 10.0):
+            step = min(8, xc.shape[0] - n)
+            oracle.mxf4_gemm(xc[n:n + step], xs[n:n + step], wc, ws)
+            n += step
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(2.0 * n * N * K / dt / 1e12, 6), "unit": "TFLOP/s",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{n} rows of A x all {N} rows of B, K = {K}, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
 
 
 def sweep_mode(args):
