@@ -43,6 +43,7 @@ METRIC = "KroQuant quantizer HBM GB/s (bf16→MXFP4+E8M0) and % of B200 peak vs 
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
 WORKLOAD = "pixart"
 GRAPH_STEPS = 200          # launches per captured graph
+E2E_CHUNKS = 4             # row chunks per layer in the end-to-end (host buffer) pipeline
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.cu")]
@@ -402,7 +403,12 @@ def gpu_arm(args, rank, local, world, pg):
 
 
 def e2e_kq(args, layers, dev, stream, kq, pg, world):
-    """KroQuant through the public API with host buffers: H2D, quantize, D2H, per step."""
+    """KroQuant through the public API with host buffers, per step: every layer's
+    bf16 input goes host -> device, is quantized, and its codes and scales go
+    device -> host.  The rows of a layer are pipelined in E2E_CHUNKS chunks over
+    three streams (H2D, quantize, D2H), so a chunk's D2H overlaps the next
+    chunk's H2D (PCIe is full duplex); events order every reuse of a device
+    chunk across steps.  All copies are inside the timed region."""
     import torch
 
     host = []
@@ -416,36 +422,63 @@ def e2e_kq(args, layers, dev, stream, kq, pg, world):
             "dc": torch.empty((M, d // 2), dtype=torch.uint8, device=dev),
             "ds": torch.empty((M, d // 32), dtype=torch.uint8, device=dev),
             "F": torch.from_numpy(L["F"]).to(dev), "shared": L["shared"],
+            "chunks": [(M * c // E2E_CHUNKS, M * (c + 1) // E2E_CHUNKS) for c in range(E2E_CHUNKS)],
         })
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    # per (layer, chunk): the quantize that last read dx, the D2H that last read dc/ds
+    last_q = {}
+    last_out = {}
 
     def one():
-        for h in host:
-            h["dx"].copy_(h["x"], non_blocking=True)
+        for li, h in enumerate(host):
             fn = kq.kq_quantize_shared if h["shared"] else kq.kq_quantize
-            fn(h["dx"], h["F"], h["dc"], h["ds"], stream=stream)
-            h["codes"].copy_(h["dc"], non_blocking=True)
-            h["scales"].copy_(h["ds"], non_blocking=True)
+            for ci, (r0, r1) in enumerate(h["chunks"]):
+                key = (li, ci)
+                if key in last_q:
+                    s_in.wait_event(last_q[key])
+                with torch.cuda.stream(s_in):
+                    h["dx"][r0:r1].copy_(h["x"][r0:r1], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+                stream.wait_event(ev_in)
+                if key in last_out:
+                    stream.wait_event(last_out[key])
+                fn(h["dx"][r0:r1], h["F"], h["dc"][r0:r1], h["ds"][r0:r1], stream=stream)
+                ev_q = torch.cuda.Event()
+                ev_q.record(stream)
+                last_q[key] = ev_q
+                s_out.wait_event(ev_q)
+                with torch.cuda.stream(s_out):
+                    h["codes"][r0:r1].copy_(h["dc"][r0:r1], non_blocking=True)
+                    h["scales"][r0:r1].copy_(h["ds"][r0:r1], non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(s_out)
+                last_out[key] = ev_o
 
     n = max(3, min(args.e2e_steps, args.steps))
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
-        stream.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        barrier(pg)
-        a.record(stream)
-        for _ in range(n):
-            one()
-        b.record(stream)
-        b.synchronize()
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    a.record(s_in)
+    for _ in range(n):
+        one()
+    # the end waits for all three streams
+    s_in.wait_stream(stream)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
+    b.synchronize()
     ms = allreduce_max(pg, [a.elapsed_time(b)], dev)[0]
     elems = sum(L["M"] * L["d"] for L in layers)
     h2d = sum(L["M"] * L["d"] * 2 for L in layers)
     d2h = sum(L["M"] * (L["d"] // 2 + L["d"] // 32) for L in layers)
     return {"value": round(world * BYTES_PER_ELEM * elems * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
-            "path": "pinned host bf16 -> cudaMemcpyAsync -> kq_quantize -> cudaMemcpyAsync -> pinned host"}
+            "path": f"pinned host bf16 -> cudaMemcpyAsync -> kq_quantize -> cudaMemcpyAsync -> pinned host, "
+                    f"{E2E_CHUNKS} row chunks per layer pipelined over H2D / quantize / D2H streams"}
 
 
 def cpu_baseline_block(layers, seconds):
