@@ -663,7 +663,9 @@ def kernel_mode(args):
 
 def gemm_mode(args):
     """The W4A4 linear layer on MXFP4 operands (tcgen05 block-scaled MMA) at
-    M x N x K, alone and chained after the KroQuant quantizer that feeds it.
+    M x N x K, alone, chained after the KroQuant quantizer that feeds it
+    (chain_us), and after the quantizer fused with LayerNorm + AdaLN
+    (norm_chain_us: residual stream in, layer output out).
 
     Operands rotate over enough sets that each launch reads A and writes D
     outside L2 (>= 3x L2 between reuses).  The roofline is the tensor pipe:
@@ -690,6 +692,8 @@ def gemm_mode(args):
     xs = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16).clone() for _ in range(nsets)]
     acs, asfs = zip(*[kq.kq_quantize_sf(xs[i], Fd) for i in range(nsets)])
     outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    g_ad, b_ad = synth.adaln(2 if M % 2 == 0 else 1, K, 5)
+    gd, bd = torch.from_numpy(g_ad).to(dev), torch.from_numpy(b_ad).to(dev)
     stream = torch.cuda.Stream(device=dev)
 
     variants = [int(v) for v in args.kernels.split(",")] if args.kernels[0].isdigit() else [0]
@@ -700,11 +704,14 @@ def gemm_mode(args):
             if kind == "chain":
                 kq.kq_quantize_sf(xs[k], Fd, out_codes=acs[k], out_sf=asfs[k], stream=stream)
                 kq.mxf4_gemm(acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
+            elif kind == "norm_chain":
+                kq.norm_kq_quantize_sf(xs[k], gd, bd, Fd, out_codes=acs[k], out_sf=asfs[k], stream=stream)
+                kq.mxf4_gemm(acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
             else:
                 kq.mxf4_gemm_variant(int(kind[1:]), acs[k], asfs[k], bc, bsf, out=outs[k], stream=stream)
 
     res = {}
-    for kind in [f"v{v}" for v in variants] + ["chain"]:
+    for kind in [f"v{v}" for v in variants] + ["chain", "norm_chain"]:
         with torch.cuda.stream(stream):
             run(kind, max(3, args.warmup))
         stream.synchronize()
@@ -737,8 +744,9 @@ def gemm_mode(args):
     tflops = flops / (res[first] * 1e-6) / 1e12
     out_bytes = M * N * 2 + M * K // 2 + N * K // 2
     line = {"mode": "gemm", "M": M, "N": N, "K": K, "nsets": nsets,
-            "gemm_us": {k: round(v, 3) for k, v in res.items() if k != "chain"},
-            "chain_us": round(res["chain"], 3), "tflops": round(tflops, 1), "peak_tflops": peak,
+            "gemm_us": {k: round(v, 3) for k, v in res.items() if k not in ("chain", "norm_chain")},
+            "chain_us": round(res["chain"], 3), "norm_chain_us": round(res["norm_chain"], 3),
+            "tflops": round(tflops, 1), "peak_tflops": peak,
             "frac_of_peak": round(tflops / peak, 4), "peak_source": src,
             "hbm_gbs_min_bytes": round(out_bytes / (res[first] * 1e-6) / 1e9, 1)}
     if args.cpu_seconds > 0:

@@ -189,6 +189,16 @@ int kq_quantize_sf(const void *act_bf16, const float *factors, int shared,
 int mx_quantize_f32(const float *x, uint8_t *out_codes, uint8_t *out_scales,
                     int scale_layout, int64_t M, int64_t d, cudaStream_t stream);
 
+/* norm_kq_quantize with the scales written in the scale-factor layout to
+ * out_sf (kq_sf_bytes(M, d) bytes, 1-byte aligned); codes exactly as
+ * norm_kq_quantize.  With mxf4_gemm this is the whole W4A4 layer input path:
+ * residual stream h -> LayerNorm + AdaLN -> transform -> MXFP4 -> product,
+ * with no intermediate written in bf16 and no scale relayout. */
+int norm_kq_quantize_sf(const void *h_bf16, const float *gamma, const float *beta,
+                        int64_t nsamples, float eps, const float *factors, int shared,
+                        uint8_t *out_codes, uint8_t *out_sf,
+                        int64_t M, int64_t d, cudaStream_t stream);
+
 /* Row-major scales [M][d/32] (from any quantizer here) -> the scale-factor
  * layout (kq_sf_bytes(M, d) bytes; the buffers may not overlap). */
 int mx_scales_to_sf(const uint8_t *scales, uint8_t *out_sf,

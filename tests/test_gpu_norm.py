@@ -50,3 +50,21 @@ def test_norm_kq_shape_errors(cuda_device):
     with pytest.raises(kq.KroQuantError) as ei:          # 6 rows, 4 samples
         kq.norm_kq_quantize(h, g, g.clone(), F)
     assert ei.value.status == kq.KQ_ERR_SHAPE
+
+
+@pytest.mark.parametrize("M,d,ns", [(300, 4608, 3), (129, 96, 1), (512, 12288, 2), (2048, 5600, 2)])
+def test_norm_kq_sf_layout_matches_row_major_path(cuda_device, M, d, ns):
+    """Same codes as norm_kq_quantize; the scales are its row-major scales in the
+    oracle's scale-factor layout, including the odd-block pad (whole buffer,
+    pre-filled with 0xFF, compared)."""
+    import torch
+
+    h = synth.activation("pixart", M, d, seed=M + 2 * d)
+    gamma, beta = synth.adaln(ns, d, seed=d + 1)
+    F = synth.factors(d // 32, seed=d + 2)
+    args = (dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device), dev(F, cuda_device))
+    c, s = kq.norm_kq_quantize(*args, eps=EPS)
+    sf0 = torch.full((kq.kq_sf_bytes(M, d),), 0xFF, dtype=torch.uint8, device=cuda_device)
+    c2, sf = kq.norm_kq_quantize_sf(*args, eps=EPS, out_sf=sf0)
+    np.testing.assert_array_equal(c2.cpu().numpy(), c.cpu().numpy())
+    np.testing.assert_array_equal(sf.cpu().numpy(), oracle.scales_to_sf(s.cpu().numpy()))

@@ -33,7 +33,7 @@ __all__ = [
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
     "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize", "kq_inverse_f32", "mx_dequantize", "norm_kq_quantize",
     "KQ_SCALES_ROWMAJOR", "KQ_SCALES_SF", "kq_sf_bytes", "kq_quantize_sf", "mx_quantize_f32", "mx_scales_to_sf",
-    "mxf4_gemm", "mxf4_gemm_variant",
+    "mxf4_gemm", "mxf4_gemm_variant", "norm_kq_quantize_sf",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
                                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                                 ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
         L.norm_kq_quantize.restype = ctypes.c_int
+        L.norm_kq_quantize_sf.argtypes = L.norm_kq_quantize.argtypes
+        L.norm_kq_quantize_sf.restype = ctypes.c_int
         L.kq_sf_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
         L.kq_sf_bytes.restype = ctypes.c_int64
         _lib = L
@@ -470,3 +472,21 @@ def mxf4_gemm_variant(variant, a_codes, a_sf, b_codes, b_sf, out=None, out_dtype
     _call("mxf4_gemm_variant", int(variant), _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
           int(out.dtype == torch.float32), M, N, K, _stream(stream))
     return out
+
+
+def norm_kq_quantize_sf(h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=None, out_sf=None, stream=None):
+    """norm_kq_quantize with the scales in the tensor core's scale-factor layout (1-D uint8)."""
+    torch = _torch()
+    M, d = _act(h)
+    _need(gamma, "gamma", torch.float32, h.device)
+    _need(beta, "beta", torch.float32, h.device, tuple(gamma.shape))
+    if gamma.dim() != 2 or gamma.shape[1] != d:
+        raise ValueError("gamma and beta must be [nsamples, d]")
+    _factors(factors, d, shared, h.device)
+    if out_codes is None:
+        out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=h.device)
+    _need(out_codes, "out_codes", torch.uint8, h.device, (M, d // 2))
+    out_sf = _sf_out(out_sf, M, d, h.device)
+    _call("norm_kq_quantize_sf", _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps), _ptr(factors),
+          int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M, d, _stream(stream))
+    return out_codes, out_sf

@@ -1306,6 +1306,27 @@ __device__ __forceinline__ Welford welford_merge(Welford a, Welford b)
     return r;
 }
 
+// Codes and scale of block (r, j); with SF the scale byte goes to the
+// scale-factor layout (see SfPos), with the odd-nb pad byte.
+template <bool SF>
+__device__ __forceinline__ void norm_emit(float2 (&p)[16], int64_t r, int j, int nb, uint4 *__restrict__ codes,
+                                          uint8_t *__restrict__ scales)
+{
+    if constexpr (SF) {
+        uint4 c;
+        uint32_t sb;
+        mx_quantize_pairs(p, c, sb);
+        codes[r * nb + j] = c;
+        const int64_t off = (r >> 7) * (int64_t((nb + 3) >> 2) * 512) + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
+                            int64_t(j >> 2) * 512 + (j & 3);
+        scales[off] = uint8_t(sb);
+        if ((nb & 1) && j == nb - 1) scales[off + 1] = 0;
+    } else {
+        kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+    }
+}
+
+template <bool SF>
 __global__ void __launch_bounds__(kThreads)
 norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
                int64_t rows_per, float eps, const float *__restrict__ factors, int shared, uint4 *__restrict__ codes,
@@ -1415,7 +1436,7 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
                 for (int k = 0; k < 5; ++k) g[k] = eq[11 + k];
                 kq_direct_apply(p, g);
             }
-            kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+            norm_emit<SF>(p, r, j, nb, codes, scales);
         }
     }
 }
@@ -1436,6 +1457,7 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
 // modulates, transforms and quantizes every block.
 constexpr int kNormRowSlot = 27;   // 8 D + 2 B/C + 1 (b4, c4, flag) + 8 (1 + gamma) + 8 beta
 
+template <bool SF>
 __global__ void __launch_bounds__(512, 1)
 norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
                     int64_t rows_per, float eps, const float *__restrict__ factors, int shared,
@@ -1581,7 +1603,7 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
                 load_factors(reinterpret_cast<const float4 *>(factors), shared, jb, g);
                 kq_direct_apply(p, g);
             }
-            kq_emit<KqOut::kCodes>(p, r * nb + jb, codes, scales, nullptr);
+            norm_emit<SF>(p, r, jb, nb, codes, scales);
         }
         __syncwarp();   // every lane is done with the buffer before it is refilled
     }
@@ -1643,7 +1665,7 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
     kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2,
-    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kKqAsync4, kKqAsync6, kNormRows, kNumKernels
+    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kKqAsync4, kKqAsync6, kNormRows, kNormKqSf, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1734,7 +1756,7 @@ int encode_act_map(const void *act, int64_t nblocks, CUtensorMap *map)
 
 std::atomic<int> g_smem_set[kNumKernels][kMaxDevices];
 constexpr size_t kNormRowsSmemMax = size_t(227) * 1024;
-std::atomic<int> g_norm_cfg[kMaxDevices][513];   // chosen single-pass norm configuration per row width
+std::atomic<int> g_norm_cfg[2][kMaxDevices][513];   // chosen single-pass norm configuration per row width
 
 // Dynamic shared memory above 48 KB needs an opt-in per kernel and device.
 int staged_prepare(KernelId id, const void *fn, int64_t *ctas_total)
@@ -2116,6 +2138,97 @@ int gemm_launch(const GemmArgs &g)
     return g.f32 ? gemm_launch_out<C, true>(g, amap, bmap, omap, grid) : gemm_launch_out<C, false>(g, amap, bmap, omap, grid);
 }
 
+template <bool SF>
+int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const float *beta, int64_t nsamples, float eps,
+                const float *factors, int shared, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
+                cudaStream_t stream)
+{
+    if (M < 0 || d <= 0 || d % kBlk != 0 || d / kBlk > 512)
+        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32, at most 16384 (M=%lld, d=%lld)",
+                    fn, (long long)M, (long long)d);
+    if (nsamples <= 0 || M % nsamples != 0)
+        return fail(KQ_ERR_SHAPE, "%s: M must be a multiple of nsamples > 0 (M=%lld, nsamples=%lld)", fn,
+                    (long long)M, (long long)nsamples);
+    if (M > 0 && M > INT64_MAX / d) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
+    if (!(eps >= 0.0f)) return fail(KQ_ERR_SHAPE, "%s: eps must be >= 0", fn);
+    if (M == 0) return ok();
+    if (!h_bf16 || !gamma || !beta || !factors || !out_codes || !out_scales)
+        return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
+    if (!aligned(h_bf16, 16) || !aligned(out_codes, 16) || !aligned(factors, 16) || !aligned(gamma, 16) ||
+        !aligned(beta, 16))
+        return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
+    const int nb = int(d / kBlk);
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    {
+        // single-pass kernel: the first (warps, row buffers) whose shared memory
+        // fits, chosen once per device and row width (cached: warps << 8 | nbuf
+        // << 4 | CTAs per SM; -1 = none fits)
+        int devc = 0;
+        cudaError_t e2 = cudaGetDevice(&devc);
+        if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e2));
+        const size_t tab = size_t(nb) * kNormRowSlot * 16, row = size_t(nb) * 64;
+        int packed = (devc >= 0 && devc < kMaxDevices) ? g_norm_cfg[SF][devc][nb].load(std::memory_order_acquire) : 0;
+        if (packed == 0) {
+            packed = -1;
+            e2 = cudaFuncSetAttribute(norm_kq_rows_kernel<SF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(kNormRowsSmemMax));
+            if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e2));
+            // fewer than 4 row buffers per CTA would leave the SM nearly idle: the
+            // fallback kernel is then faster
+            const int cfg[7][2] = {{16, 1}, {8, 2}, {12, 1}, {4, 2}, {8, 1}, {2, 2}, {4, 1}};
+            for (const auto &c : cfg) {
+                const size_t smem_r = tab + size_t(c[0]) * c[1] * row;
+                if (smem_r > kNormRowsSmemMax) continue;
+                int per_sm = 0;
+                e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_rows_kernel<SF>, 32 * c[0], smem_r);
+                if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e2));
+                if (per_sm < 1) continue;
+                packed = (c[0] << 8) | (c[1] << 4) | (per_sm > 15 ? 15 : per_sm);
+                break;
+            }
+            if (devc >= 0 && devc < kMaxDevices) g_norm_cfg[SF][devc][nb].store(packed, std::memory_order_release);
+        }
+        if (packed > 0) {
+            const int warps = packed >> 8, nbuf = (packed >> 4) & 15, per_sm = packed & 15;
+            const int64_t rows_per = M / nsamples;
+            int64_t cps = int64_t(sms) * per_sm / nsamples;
+            const int64_t most = rows_per / warps;          // at least one row per warp per CTA
+            if (cps > most) cps = most;
+            if (cps < 1) cps = 1;
+            if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
+            const size_t smem_r = tab + size_t(warps) * nbuf * row;
+            norm_kq_rows_kernel<SF><<<unsigned(cps * nsamples), 32 * warps, smem_r, stream>>>(
+                static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps, factors, shared ? 1 : 0,
+                reinterpret_cast<uint4 *>(out_codes), out_scales, nb, int(cps), nbuf);
+            return launch_check(fn);
+        }
+    }
+    const size_t smem = size_t(nb) * kNormSlot * sizeof(float);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (smem > 48 * 1024 && (dev < 0 || dev >= kMaxDevices || !g_smem_set[SF ? kNormKqSf : kNormKq][dev].load())) {
+        e = cudaFuncSetAttribute(norm_kq_kernel<SF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(size_t(512) * kNormSlot * sizeof(float)));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        if (dev >= 0 && dev < kMaxDevices) g_smem_set[SF ? kNormKqSf : kNormKq][dev].store(1);
+    }
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel<SF>, kThreads, smem);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+    if (per_sm < 1) per_sm = 1;
+    const int64_t warps_needed = M;
+    int64_t grid = int64_t(sms) * per_sm;
+    const int64_t need = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
+    if (grid > need) grid = need;
+    norm_kq_kernel<SF><<<unsigned(grid), kThreads, smem, stream>>>(
+        static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
+        reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb);
+    return launch_check(fn);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -2336,91 +2449,16 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta, 
                      const float *factors, int shared, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
                      cudaStream_t stream)
 {
-    const char *fn = "norm_kq_quantize";
-    if (M < 0 || d <= 0 || d % kBlk != 0 || d / kBlk > 512)
-        return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32, at most 16384 (M=%lld, d=%lld)",
-                    fn, (long long)M, (long long)d);
-    if (nsamples <= 0 || M % nsamples != 0)
-        return fail(KQ_ERR_SHAPE, "%s: M must be a multiple of nsamples > 0 (M=%lld, nsamples=%lld)", fn,
-                    (long long)M, (long long)nsamples);
-    if (M > 0 && M > INT64_MAX / d) return fail(KQ_ERR_SHAPE, "%s: size too large", fn);
-    if (!(eps >= 0.0f)) return fail(KQ_ERR_SHAPE, "%s: eps must be >= 0", fn);
-    if (M == 0) return ok();
-    if (!h_bf16 || !gamma || !beta || !factors || !out_codes || !out_scales)
-        return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
-    if (!aligned(h_bf16, 16) || !aligned(out_codes, 16) || !aligned(factors, 16) || !aligned(gamma, 16) ||
-        !aligned(beta, 16))
-        return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
-    const int nb = int(d / kBlk);
-    int sms = 0;
-    int rc = sm_count(&sms);
-    if (rc != KQ_OK) return rc;
-    {
-        // single-pass kernel: the first (warps, row buffers) whose shared memory
-        // fits, chosen once per device and row width (cached: warps << 8 | nbuf
-        // << 4 | CTAs per SM; -1 = none fits)
-        int devc = 0;
-        cudaError_t e2 = cudaGetDevice(&devc);
-        if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e2));
-        const size_t tab = size_t(nb) * kNormRowSlot * 16, row = size_t(nb) * 64;
-        int packed = (devc >= 0 && devc < kMaxDevices) ? g_norm_cfg[devc][nb].load(std::memory_order_acquire) : 0;
-        if (packed == 0) {
-            packed = -1;
-            e2 = cudaFuncSetAttribute(norm_kq_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(kNormRowsSmemMax));
-            if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e2));
-            // fewer than 4 row buffers per CTA would leave the SM nearly idle: the
-            // fallback kernel is then faster
-            const int cfg[7][2] = {{16, 1}, {8, 2}, {12, 1}, {4, 2}, {8, 1}, {2, 2}, {4, 1}};
-            for (const auto &c : cfg) {
-                const size_t smem_r = tab + size_t(c[0]) * c[1] * row;
-                if (smem_r > kNormRowsSmemMax) continue;
-                int per_sm = 0;
-                e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_rows_kernel, 32 * c[0], smem_r);
-                if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e2));
-                if (per_sm < 1) continue;
-                packed = (c[0] << 8) | (c[1] << 4) | (per_sm > 15 ? 15 : per_sm);
-                break;
-            }
-            if (devc >= 0 && devc < kMaxDevices) g_norm_cfg[devc][nb].store(packed, std::memory_order_release);
-        }
-        if (packed > 0) {
-            const int warps = packed >> 8, nbuf = (packed >> 4) & 15, per_sm = packed & 15;
-            const int64_t rows_per = M / nsamples;
-            int64_t cps = int64_t(sms) * per_sm / nsamples;
-            const int64_t most = rows_per / warps;          // at least one row per warp per CTA
-            if (cps > most) cps = most;
-            if (cps < 1) cps = 1;
-            if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
-            const size_t smem_r = tab + size_t(warps) * nbuf * row;
-            norm_kq_rows_kernel<<<unsigned(cps * nsamples), 32 * warps, smem_r, stream>>>(
-                static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps, factors, shared ? 1 : 0,
-                reinterpret_cast<uint4 *>(out_codes), out_scales, nb, int(cps), nbuf);
-            return launch_check(fn);
-        }
-    }
-    const size_t smem = size_t(nb) * kNormSlot * sizeof(float);
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (smem > 48 * 1024 && (dev < 0 || dev >= kMaxDevices || !g_smem_set[kNormKq][dev].load())) {
-        e = cudaFuncSetAttribute(norm_kq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(size_t(512) * kNormSlot * sizeof(float)));
-        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        if (dev >= 0 && dev < kMaxDevices) g_smem_set[kNormKq][dev].store(1);
-    }
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, norm_kq_kernel, kThreads, smem);
-    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
-    if (per_sm < 1) per_sm = 1;
-    const int64_t warps_needed = M;
-    int64_t grid = int64_t(sms) * per_sm;
-    const int64_t need = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
-    if (grid > need) grid = need;
-    norm_kq_kernel<<<unsigned(grid), kThreads, smem, stream>>>(
-        static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
-        reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb);
-    return launch_check(fn);
+    return norm_launch<false>("norm_kq_quantize", h_bf16, gamma, beta, nsamples, eps, factors, shared, out_codes,
+                              out_scales, M, d, stream);
+}
+
+int norm_kq_quantize_sf(const void *h_bf16, const float *gamma, const float *beta, int64_t nsamples, float eps,
+                        const float *factors, int shared, uint8_t *out_codes, uint8_t *out_sf, int64_t M, int64_t d,
+                        cudaStream_t stream)
+{
+    return norm_launch<true>("norm_kq_quantize_sf", h_bf16, gamma, beta, nsamples, eps, factors, shared, out_codes,
+                             out_sf, M, d, stream);
 }
 
 int64_t kq_sf_bytes(int64_t rows, int64_t d)
