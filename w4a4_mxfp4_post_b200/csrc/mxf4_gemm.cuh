@@ -47,8 +47,7 @@ namespace gemm {
 constexpr int kBM = 128;                                  // tile rows (MMA M)
 constexpr int kSfUnit = 512;                              // 128 rows x 4 blocks
 constexpr int kTmemCols = 512;                            // power of two >= 256 + scale columns
-constexpr uint32_t kAccCol = 0;                           // 256 fp32 accumulator columns
-constexpr uint32_t kSfCol = 256;                          // scale columns: 16 per stage and k-unit
+constexpr uint32_t kAccCol = 0;                           // fp32 accumulator(s), then the scale columns
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;             // 320
 constexpr int kStageOutBytes = 32 * 128 * 2;              // a warp's 32 rows x 128 bf16 columns
@@ -81,13 +80,19 @@ struct Cfg {
     static constexpr uint64_t kLayout = CB == 128 ? mma::kLayoutSw128 : mma::kLayoutSw64;
     static constexpr uint32_t kSbo = 8 * CB;              // 8-row swizzle atom
     static constexpr size_t kRing = size_t(ST) * kStageBytes;
+    // Two accumulators where they fit beside the scale columns (192-column
+    // tiles: 2 x 192 + scales <= 512): the MMAs of the next tile then start
+    // while the epilogue still drains the previous one.
+    static constexpr int kAccBufs = (2 * BN + ST * int(16 * (CB / 64)) <= kTmemCols) ? 2 : 1;
+    static constexpr uint32_t kSfCol = uint32_t(kAccBufs * BN);   // scale columns: 16 per stage and k-unit
     static constexpr size_t kSmem = kRing + (TMA_OUT ? size_t(kEpiWarps) * kStageOutBytes : 0) + 1024 +
-                                    (2 * ST + 4) * sizeof(uint64_t) + 16;
+                                    (2 * ST + 6) * sizeof(uint64_t) + 16;
     static_assert(CB == 64 || CB == 128, "chunk bytes");
     static_assert(BN == 256 || BN == 192, "tile columns");
     static_assert(kStageBytes % (8 * CB) == 0, "stages keep the alignment of the swizzle atom");
     static_assert(!TMA_OUT || kRing % 1024 == 0, "the output staging keeps the 1 KB alignment of its swizzle");
     static_assert(kSfCol + ST * kSfStageCols <= kTmemCols, "tensor memory columns");
+    static_assert(kSfCol % 4 == 0, "scale columns are 4-aligned");
     static_assert(kSmem <= kSmemMax, "shared memory");
 };
 
@@ -153,10 +158,11 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
     uint64_t *bars = reinterpret_cast<uint64_t *>(stage_out + (C::kTmaOut ? size_t(kEpiWarps) * kStageOutBytes : 0));
     uint64_t *full = bars;                    // [ST] stage landed (TMA / bulk tx)
     uint64_t *empty = bars + ST;              // [ST] MMAs reading the stage done (commit)
-    uint64_t *acc_full = bars + 2 * ST;       // accumulator holds a finished tile (commit)
-    uint64_t *acc_empty = acc_full + 1;       // accumulator read by the 8 epilogue warps
-    uint64_t *done = acc_full + 2;            // every MMA of this CTA completed (final commit)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 4);
+    constexpr int NA = C::kAccBufs;
+    uint64_t *acc_full = bars + 2 * ST;       // [2] accumulator b holds a finished tile (commit)
+    uint64_t *acc_empty = acc_full + 2;       // [2] accumulator b read by the 8 epilogue warps
+    uint64_t *done = acc_full + 4;            // every MMA of this CTA completed (final commit)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 6);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     const int MT = (M + kBM - 1) / kBM;
@@ -172,8 +178,10 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kEpiWarps);
+        }
         mbar_init(done, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -237,7 +245,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 // a tile starting mid-unit (192-column tiles): the MMA reads B's
                 // scales off = 0 or 2 columns (32-row groups) into the first unit
                 const uint32_t off = uint32_t(((t % NT) * kBN % 128) / 32);
-                if (it > 0 && !mbar_wait(acc_empty, (it - 1) & 1, budget)) {
+                const int ab = it % NA;               // accumulator of this tile
+                if (it >= NA && !mbar_wait(&acc_empty[ab], ((it / NA) - 1) & 1, budget)) {
                     atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
@@ -254,7 +263,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     const uint32_t b0 = a0 + C::kABytes;
                     const uint32_t sfa = b0 + C::kBBytes;
                     const uint32_t sfb = sfa + C::kSfaBytes;
-                    const uint32_t tsf = tmem_base + kSfCol + uint32_t(s) * C::kSfStageCols;   // + 16 u
+                    const uint32_t tsf = tmem_base + C::kSfCol + uint32_t(s) * C::kSfStageCols;   // + 16 u
                     // units past K or of a missing B row group are stale data:
                     // they reach only K steps not issued or output columns >= N
 #pragma unroll
@@ -270,13 +279,14 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                         const uint32_t u = j >> 1;
                         const uint64_t ad = mma::smem_desc(a0 + j * 32, C::kSbo, C::kLayout);
                         const uint64_t bd = mma::smem_desc(b0 + j * 32, C::kSbo, C::kLayout);
-                        umma_mxf4(tmem_base + kAccCol, ad, bd, idesc(C::kIdesc, sf_id), (tsf + 16 * u) | (sf_id << 30),
+                        umma_mxf4(tmem_base + kAccCol + uint32_t(ab * kBN), ad, bd, idesc(C::kIdesc, sf_id),
+                                  (tsf + 16 * u) | (sf_id << 30),
                                   (tsf + 16 * u + 8 + off) | (sf_id << 30), (c | j) != 0);
                     }
                     mma::umma_commit(&empty[s]);
                 }
                 if (!ok) break;
-                mma::umma_commit(acc_full);
+                mma::umma_commit(&acc_full[ab]);
             }
             // every MMA issued has completed before the tensor memory is freed
             mma::umma_commit(done);
@@ -289,14 +299,15 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
         int it = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
             const int mt = t / NT, nt = t % NT;
-            const bool ready = mbar_wait(acc_full, it & 1, budget);
+            const int ab = it % NA;
+            const bool ready = mbar_wait(&acc_full[ab], (it / NA) & 1, budget);
             if (!__all_sync(0xffffffffu, ready)) {   // tcgen05.ld below is warp-collective
                 if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                 break;
             }
             mma::tc_fence_after();
             constexpr int EC = C::kEpiCols;           // 128 or 96 columns per warp
-            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(h * EC);
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + kAccCol + uint32_t(ab * kBN + h * EC);
             const int row0 = mt * kBM + q * 32;
             const int col0 = nt * kBN + h * EC;
             if constexpr (F32OUT) {
@@ -306,7 +317,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 mma::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
                 const int row = row0 + lane;
                 if (row < M) {
                     float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + int64_t(row) * N + col0);
@@ -327,7 +338,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 }
                 mma::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty);
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);
                 if constexpr (kStaged) {
                     // the previous tile's stores have finished reading the staging buffer
                     if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
