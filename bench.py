@@ -51,7 +51,7 @@ KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.c
 # DRAM traffic per launch of the dominant kernel (KroQuant quantizer, d = 4608
 # layer), from one ncu capture, valid only for the kernel source it was taken
 # on (sha256 prefix of the .cu sources).  Updated after each capture.
-TRAFFIC = {"source_sha": "38c3c946accb4c0e", "bytes_per_launch": 80712448.0,
+TRAFFIC = {"source_sha": "3000e18ddd7d6ee5", "bytes_per_launch": 79977728.0,
            "capture": "ncu --set full, kq_packed_kernel, 8192x4608, dram__bytes_read.sum + dram__bytes_write.sum"}
 
 

@@ -68,3 +68,25 @@ def test_norm_kq_sf_layout_matches_row_major_path(cuda_device, M, d, ns):
     c2, sf = kq.norm_kq_quantize_sf(*args, eps=EPS, out_sf=sf0)
     np.testing.assert_array_equal(c2.cpu().numpy(), c.cpu().numpy())
     np.testing.assert_array_equal(sf.cpu().numpy(), oracle.scales_to_sf(s.cpu().numpy()))
+
+
+@pytest.mark.parametrize("M,d", [(256, 1152), (300, 4608)])
+def test_norm_kq_large_mean_takes_the_two_pass_variance(cuda_device, M, d):
+    """Rows whose mean is large against their spread (each row shifted by half
+    its root mean square, so mu^2 > E[x^2] / 64): the one-sweep variance
+    E[x^2] - mu^2 is not used there and the kernel takes the two-pass form; the
+    result meets the oracle criteria.  (A mean far above the spread, with the
+    spread near bf16's resolution, would be ill-conditioned for any fp32
+    LayerNorm: the mean's rounding is amplified by 1 / sigma.)"""
+    x = synth.bf16_bits_to_f32(synth.activation("pixart", M, d, seed=7)).astype(np.float64)
+    rms = np.sqrt((x * x).mean(axis=1, keepdims=True))
+    h = synth.bf16_bits_from_f32((x + 0.5 * rms).astype(np.float32))
+    hv = synth.bf16_bits_to_f32(h).astype(np.float64)
+    assert np.all(hv.mean(axis=1) ** 2 > (hv * hv).mean(axis=1) / 64)     # the two-pass branch
+    gamma, beta = synth.adaln(2, d, seed=d)
+    F = synth.factors(d // 32, seed=d)
+    c, s = kq.norm_kq_quantize(dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device),
+                               dev(F, cuda_device), eps=EPS)
+    ref = oracle.norm_kq(h, gamma, beta, EPS, F, want=("codes", "y", "absb"))
+    res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
+    assert res["ok"], res

@@ -1452,9 +1452,10 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
 // block b lands at b * 64 + 16 (p ^ ((b >> 1) & 3)), so the per-lane block
 // reads of the second sweep are free of bank conflicts), the next row in
 // flight while the current one is processed: the row is read from HBM once.
-// From shared memory a warp takes the mean (one sweep), the sum of squared
-// deviations from it (a second sweep: the two-pass variance), then normalises,
-// modulates, transforms and quantizes every block.
+// From shared memory a warp takes the sums of x and x^2 in one sweep (a
+// second sweep over (x - mu)^2 only where the mean is large against the root
+// mean square), then normalises, modulates, transforms and quantizes every
+// block.
 constexpr int kNormRowSlot = 27;   // 8 D + 2 B/C + 1 (b4, c4, flag) + 8 (1 + gamma) + 8 beta
 
 template <bool SF>
@@ -1527,37 +1528,59 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
         }
         __syncwarp();
         const uint4 *rb = wbuf + size_t(buf) * npieces;
-        // ---- statistics: mean, then the sum of squared deviations from it
+        // ---- statistics.  One sweep gives the sums of x and x^2; where the mean
+        // is small against the root mean square (mu^2 <= 2^-6 E[x^2]) the
+        // variance E[x^2] - mu^2 loses at most ~2 ulp to cancellation and is
+        // used directly, otherwise a second sweep sums (x - mu)^2 (the
+        // two-pass variance).  The choice is warp-uniform (reduced values).
         const uint4 *lp = rb + lslot;                             // this lane's pieces, 32 apart
-        float2 s2 = make_float2(0.0f, 0.0f);
-        for (int k = 0; k < nk; ++k) {
-            const uint4 w = lp[32 * k];
-            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.x), bf16_hi(w.x)));
-            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.y), bf16_hi(w.y)));
-            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.z), bf16_hi(w.z)));
-            s2 = __fadd2_rn(s2, make_float2(bf16_lo(w.w), bf16_hi(w.w)));
-        }
-        float sum = s2.x + s2.y;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        const float mu = sum / float(d);
-        const float2 nmu = make_float2(-mu, -mu);
-        float2 q2 = make_float2(0.0f, 0.0f);
+        float2 s2 = make_float2(0.0f, 0.0f), q2 = make_float2(0.0f, 0.0f);
         for (int k = 0; k < nk; ++k) {
             const uint4 w = lp[32 * k];
             float2 t;
-            t = __fadd2_rn(make_float2(bf16_lo(w.x), bf16_hi(w.x)), nmu);
+            t = make_float2(bf16_lo(w.x), bf16_hi(w.x));
+            s2 = __fadd2_rn(s2, t);
             q2 = __ffma2_rn(t, t, q2);
-            t = __fadd2_rn(make_float2(bf16_lo(w.y), bf16_hi(w.y)), nmu);
+            t = make_float2(bf16_lo(w.y), bf16_hi(w.y));
+            s2 = __fadd2_rn(s2, t);
             q2 = __ffma2_rn(t, t, q2);
-            t = __fadd2_rn(make_float2(bf16_lo(w.z), bf16_hi(w.z)), nmu);
+            t = make_float2(bf16_lo(w.z), bf16_hi(w.z));
+            s2 = __fadd2_rn(s2, t);
             q2 = __ffma2_rn(t, t, q2);
-            t = __fadd2_rn(make_float2(bf16_lo(w.w), bf16_hi(w.w)), nmu);
+            t = make_float2(bf16_lo(w.w), bf16_hi(w.w));
+            s2 = __fadd2_rn(s2, t);
             q2 = __ffma2_rn(t, t, q2);
         }
-        float m2 = q2.x + q2.y;
+        float sum = s2.x + s2.y, sq = q2.x + q2.y;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+        for (int off = 16; off > 0; off >>= 1) {
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float mu = sum / float(d);
+        const float2 nmu = make_float2(-mu, -mu);
+        const float ex2 = sq / float(d);
+        float m2;
+        if (mu * mu <= ex2 * (1.0f / 64.0f)) {
+            m2 = fmaxf(ex2 - mu * mu, 0.0f) * float(d);
+        } else {
+            q2 = make_float2(0.0f, 0.0f);
+            for (int k = 0; k < nk; ++k) {
+                const uint4 w = lp[32 * k];
+                float2 t;
+                t = __fadd2_rn(make_float2(bf16_lo(w.x), bf16_hi(w.x)), nmu);
+                q2 = __ffma2_rn(t, t, q2);
+                t = __fadd2_rn(make_float2(bf16_lo(w.y), bf16_hi(w.y)), nmu);
+                q2 = __ffma2_rn(t, t, q2);
+                t = __fadd2_rn(make_float2(bf16_lo(w.z), bf16_hi(w.z)), nmu);
+                q2 = __ffma2_rn(t, t, q2);
+                t = __fadd2_rn(make_float2(bf16_lo(w.w), bf16_hi(w.w)), nmu);
+                q2 = __ffma2_rn(t, t, q2);
+            }
+            m2 = q2.x + q2.y;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m2 += __shfl_xor_sync(0xffffffffu, m2, off);
+        }
         const float inv = 1.0f / sqrtf(m2 / float(d) + eps);
         const float2 iv = make_float2(inv, inv);
         // ---- normalise, modulate, transform, quantize
