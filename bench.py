@@ -795,6 +795,9 @@ def sweep_mode(args):
                     continue
                 gbs = BYTES_PER_ELEM * M * d / (r["mean_us"] * 1e-6) / 1e9
                 row[kind] = {"us": round(r["mean_us"], 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+            # a launch under 10 MB or 2 us measures launch latency and ramp, not the stream
+            row["launch_bound"] = bool(row["bytes"] < 10e6 or any(
+                isinstance(v, dict) and v.get("us", 1e9) < 2.0 for v in row.values()))
             del inp
             torch.cuda.empty_cache()
             rows.append(row)
