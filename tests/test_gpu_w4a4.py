@@ -218,3 +218,41 @@ def test_mxf4_gemm_full_size_sampled_rows(cuda_device, N, K):
     D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, rows=rows, want_absbound=True)
     got = out.index_select(0, torch.from_numpy(rows).to(cuda_device)).float().cpu().numpy()
     check_gemm(got, D, absd, K, True)
+
+
+def test_mxf4_gemm_extreme_scale_exponents(cuda_device):
+    """Scale bytes at both ends of E8M0: A at 2^127 (0xFE) and 2^126, B at
+    2^-127 (0x00) and 2^-126, so every product is of order one; the tensor
+    core must apply both exponents exactly (oracle bound as above)."""
+    import torch
+
+    M, N, K = 130, 136, 320
+    ca, _ = synth.mx_operand(M, K, 61)
+    cb, _ = synth.mx_operand(N, K, 62)
+    rng = np.random.default_rng(63)
+    sa = rng.choice(np.array([0xFE, 0xFD], np.uint8), size=(M, K // 32))
+    sb = rng.choice(np.array([0x00, 0x01], np.uint8), size=(N, K // 32))
+    D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+    out = kq.mxf4_gemm(dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
+                       dev(oracle.scales_to_sf(sb), cuda_device), out_dtype=torch.float32)
+    assert np.all(np.isfinite(D))
+    check_gemm(out.cpu().numpy(), D, absd, K, False)
+
+
+def test_mxf4_gemm_nan_scale_reaches_only_its_row(cuda_device):
+    """A scale byte 0xFF (E8M0 NaN) in one row of A makes exactly that output
+    row NaN (the header's stated behaviour); every other row is unaffected."""
+    import torch
+
+    M, N, K = 96, 64, 256
+    ca, sa = synth.mx_operand(M, K, 71)
+    cb, sb = synth.mx_operand(N, K, 72)
+    sa = sa.copy()
+    sa[5, 3] = 0xFF
+    D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+    out = kq.mxf4_gemm(dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
+                       dev(oracle.scales_to_sf(sb), cuda_device), out_dtype=torch.float32).cpu().numpy()
+    assert np.all(np.isnan(out[5])) and np.all(np.isnan(D[5]))
+    keep = np.arange(M) != 5
+    assert np.all(np.isfinite(out[keep]))
+    check_gemm(out[keep], D[keep], absd[keep], K, False)
