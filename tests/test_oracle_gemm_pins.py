@@ -146,3 +146,32 @@ def test_mx_quantize_f32_round_trip_error_bound():
     bound = np.where(v <= 6, 1.0, 2.0) * np.ldexp(1.0, e)
     assert np.all(np.abs(xr - x) <= bound)
     assert np.any(v > 6)            # the saturating branch is exercised
+
+
+def test_w4a4_chain_computes_x_wt_on_the_oracle():
+    """The chain the W4A4 consumer implements, on the oracle alone: with
+    Hadamard factors, (MXFP4(X T^T)) (MXFP4(W T^-1))^T approximates X W^T
+    better than plain MXFP4 on both operands, and dropping the fold (W left
+    untransformed) destroys it.  Pins that the fold pairs with the transform
+    (T^-1, not T or T^T) and that the product contracts the right indices."""
+    from w4a4_mxfp4_post_b200 import synth
+
+    M, N, d = 128, 96, 256
+    x = synth.activation("pixart", M, d, 3)
+    W = synth.weights(N, d, 3)
+    s = np.float32(1.0 / np.sqrt(2.0))
+    H = np.tile(np.array([[s, s], [s, -s]], np.float32), (d // 32, 5, 1, 1))
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ W.astype(np.float64).T
+    ca, sa = oracle.kq_quantize(x, H)
+
+    def rel(D):
+        return np.linalg.norm(D - ref) / np.linalg.norm(ref)
+
+    cb, sb = oracle.mx_quantize_f32(oracle.fold_weights(W, H))
+    folded = rel(oracle.mxf4_gemm(ca, sa, cb, sb))
+    cbu, sbu = oracle.mx_quantize_f32(W)
+    unfolded = rel(oracle.mxf4_gemm(ca, sa, cbu, sbu))
+    cam, sam = oracle.mx_quantize(x)
+    plain = rel(oracle.mxf4_gemm(cam, sam, cbu, sbu))
+    assert folded < plain < 0.5, (folded, plain)
+    assert unfolded > 0.9, unfolded
