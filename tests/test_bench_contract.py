@@ -1,0 +1,30 @@
+"""Host-side pieces of bench.py that need no GPU: the kernel-source hash that
+ties the recorded DRAM traffic to the code it was captured on."""
+import bench
+
+
+def _src():
+    with open(bench.KERNEL_SOURCES[0]) as fh:
+        return fh.read()
+
+
+def test_kernel_source_text_covers_the_kernel_and_its_launch_path():
+    t = bench.kernel_source_text(_src())
+    assert "kq_packed_kernel(const uint4" in t and "kq_fast_apply" in t and "mx_quantize_pairs" in t
+    for head in bench.LAUNCH_FUNCS:
+        assert head in t
+    assert "norm_kq_rows_kernel" not in t and "mxf4_gemm_kernel" not in t
+
+
+def test_hash_follows_the_kernel_not_unrelated_code():
+    src = _src()
+    base = bench.kernel_source_text(src)
+    # an edit inside the dominant kernel or its launch path changes the text
+    edited = src.replace("kq_fast_apply(p, st);", "kq_fast_apply(p, st); /* edit */", 1)
+    assert bench.kernel_source_text(edited) != base
+    launch = src.replace("Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)\n{",
+                         "Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)\n{ /* edit */", 1)
+    assert launch != src and bench.kernel_source_text(launch) != base
+    # an edit in an unrelated kernel later in the file does not
+    other = src.replace("norm_kq_rows_kernel(", "norm_kq_rows_kernel /* edit */ (", 1)
+    assert other != src and bench.kernel_source_text(other) == base
