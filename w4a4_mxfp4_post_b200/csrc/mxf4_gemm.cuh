@@ -11,34 +11,37 @@
 // element in the low nibble), with their E8M0 scales in the scale-factor
 // layout (SfPos in kroquant.cu).  D is bf16 or fp32, [M][N] row-major.
 //
-// One tcgen05 block-scaled MMA (kind::mxf4, block32) is M128 x N256 x K64: the
-// tensor core decodes E2M1 and applies the two E8M0 scales of every 32-block,
-// accumulating in fp32 in tensor memory.  The scale bytes reach tensor memory
-// by tcgen05.cp from shared memory (one 512-byte unit = 128 rows x 4 blocks
-// per copy, 32 lanes x 128 bits replicated to the four lane quarters).
+// One tcgen05 block-scaled MMA (kind::mxf4, block32) is M128 x BN x K64 (BN =
+// 256 or 192): the tensor core decodes E2M1 and applies the two E8M0 scales of
+// every 32-block, accumulating in fp32 in tensor memory.  The scale bytes reach
+// tensor memory by tcgen05.cp from shared memory (one 512-byte unit = 128 rows
+// x 4 blocks per copy, 32 lanes x 128 bits replicated to the four lane
+// quarters).
 //
-// A CTA owns one SM (persistent) and walks the 128 x 256 output tiles
+// A CTA owns one SM (persistent) and walks the 128 x BN output tiles
 // t = blockIdx.x, + gridDim.x, ...; a k-chunk is CB bytes of codes per row
 // (2 CB elements, one CB-byte swizzle atom; CB / 64 scale units per row
-// group), CB and the ring depth ST being compile-time choices (Cfg).
+// group), CB, the ring depth ST and BN being compile-time choices (Cfg).
 //   warp 0     producer: per chunk, TMA loads of the A box {CB x 128 rows}
-//              and the B box {CB x 256 rows} (CB-byte swizzle; rows and
-//              bytes past the matrix read as zero) and bulk copies of the
-//              chunk's scale units (A: its row group's, B: both row groups')
+//              and the B box {CB x BN rows} (CB-byte swizzle; rows and bytes
+//              past the matrix read as zero) and bulk copies of the chunk's
+//              scale units (A: its row group's, B: the tile's two row groups')
 //              into an ST-stage ring
 //   warp 1     allocates tensor memory; one thread copies a stage's scale
 //              units to that stage's own tensor-memory columns (so a copy
 //              never waits on MMAs still reading an older stage), issues the
-//              chunk's CB / 32 MMAs (only the K=64 steps below K) and commits the
-//              stage back to the producer; after a tile's last chunk it
-//              commits the accumulator
+//              chunk's CB / 32 MMAs (only the K=64 steps below K) and commits
+//              the stage back to the producer; after a tile's last chunk it
+//              commits the accumulator.  Where two accumulators fit beside the
+//              scale columns (BN = 192) tiles alternate between them.
 //   warps 2-9  epilogue: warp w reads accumulator lanes 32 (w % 4) .. +31 (tile
-//              rows) and columns 128 ((w - 2) / 4) .. +127 into registers and
-//              hands the accumulator back at once; then, while the MMAs of the
-//              next tile run, it stores its segment: with TMA_OUT (bf16) through
-//              the warp's 8 KB of shared memory (128-byte swizzle) and two TMA
-//              tensor stores of {64 columns x 32 rows} (rows and columns past D
-//              are clipped), otherwise with 16-byte stores from registers
+//              rows) and columns BN/2 ((w - 2) / 4) .. + BN/2 - 1 into
+//              registers and hands the accumulator back at once; then, while
+//              the MMAs of the next tile run, it stores its segment: with
+//              TMA_OUT (bf16) through the warp's 8 KB of shared memory and TMA
+//              tensor stores of {64 columns x 32 rows} (128-byte swizzle, BN =
+//              256) or {32 x 32} (64-byte swizzle, BN = 192), rows and columns
+//              past D clipped; otherwise with 16-byte stores from registers
 // Every mbarrier wait is bounded (g_wait_timeouts); every path drains the
 // copies in flight, waits for its MMAs and frees the tensor memory.
 
