@@ -59,6 +59,15 @@ def test_library_exports_every_declared_symbol(L):
         assert getattr(L, n) is not None
 
 
+def test_python_binding_mirrors_every_declared_entry_point():
+    """The binding is thin and complete: one Python function per C entry point, same name."""
+    import w4a4_mxfp4_post_b200 as kq
+
+    missing = [n for n in declared_functions() if not callable(getattr(kq, n, None))]
+    assert not missing, missing
+    assert set(declared_functions()) <= set(kq.__all__) | {"kq_last_error", "kq_abi_version"}
+
+
 def test_abi_version(L):
     assert L.kq_abi_version() == 1
 
