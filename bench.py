@@ -19,6 +19,20 @@ rank quantizes its own batch (weak scaling, no collective on the data path).
 
 `--impl reference` times the CPU oracle (oracle/, plain C) on the host cores on
 a bounded sample of the same workload and prints the same JSON line.
+
+Besides the step line, the JSON carries the roofline of the dominant launch
+(with the DRAM traffic of an ncu capture, valid for the kernel source it was
+taken on), the end-to-end figure through host buffers (H2D, quantize and D2H
+pipelined over three streams), the CPU-oracle baseline, the SM clocks sampled
+during the timed region and the number of kernel launches.
+
+Other modes (one JSON line each):
+    --mode kernel --kernel K --shape MxD     one quantizer or variant at one shape
+    --mode sweep [--kernels ...]             every shape of the sweep workload
+    --mode sqnr                              quantisation-error proxy (SQNR)
+    --mode gemm --shape MxNxK [--kernels v]  the W4A4 product, its tile configurations,
+                                             and the chains quantize -> product and
+                                             norm + quantize -> product
 """
 from __future__ import annotations
 
