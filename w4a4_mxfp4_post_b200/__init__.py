@@ -116,8 +116,16 @@ def kq_abi_version() -> int:
     return lib().kq_abi_version()
 
 
-def _call(name: str, *args) -> None:
-    rc = getattr(lib(), name)(*args)
+def _call(name: str, device, *args) -> None:
+    """Call entry point `name` with `device` (the tensors' device; None = the
+    current one) as the current CUDA device: the library launches on the
+    current device and caches its properties per device."""
+    fn = getattr(lib(), name)
+    if device is not None and device.index is not None and device.index != _torch().cuda.current_device():
+        with _torch().cuda.device(device):
+            rc = fn(*args)
+    else:
+        rc = fn(*args)
     if rc != KQ_OK:
         raise KroQuantError(name, rc, kq_last_error())
 
@@ -128,10 +136,14 @@ def _torch():
     return torch
 
 
-def _stream(stream):
+def _stream(stream, device):
+    """The raw handle of `stream`, default the current stream of `device`; a
+    torch stream must belong to `device`."""
     torch = _torch()
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif isinstance(stream, torch.cuda.Stream) and device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
@@ -190,7 +202,8 @@ def kq_quantize(act, factors, out_codes=None, out_scales=None, stream=None):
     M, d = _act(act)
     _factors(factors, d, False, act.device)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("kq_quantize", _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    _call("kq_quantize", act.device, _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -199,8 +212,8 @@ def kq_quantize_shared(act, factors, out_codes=None, out_scales=None, stream=Non
     M, d = _act(act)
     _factors(factors, d, True, act.device)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("kq_quantize_shared", _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d,
-          _stream(stream))
+    _call("kq_quantize_shared", act.device, _ptr(act), _ptr(factors), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -209,8 +222,8 @@ def kq_quantize_variant(variant, act, factors, shared=False, out_codes=None, out
     M, d = _act(act)
     _factors(factors, d, shared, act.device)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("kq_quantize_variant", int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes),
-          _ptr(out_scales), M, d, _stream(stream))
+    _call("kq_quantize_variant", act.device, int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes),
+          _ptr(out_scales), M, d, _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -220,7 +233,8 @@ def sq_quantize(act, mult, out_codes=None, out_scales=None, stream=None):
     M, d = _act(act)
     _need(mult, "mult", torch.float32, act.device, (d,))
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("sq_quantize", _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    _call("sq_quantize", act.device, _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -228,7 +242,7 @@ def mx_quantize(act, out_codes=None, out_scales=None, stream=None):
     """Plain MXFP4 baseline (no transform)."""
     M, d = _act(act)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("mx_quantize", _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    _call("mx_quantize", act.device, _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -241,8 +255,8 @@ def kq_quantize_lu(act, lu_params, shared=False, out_codes=None, out_scales=None
     if lu_params.numel() != n * 15:
         raise ValueError(f"lu_params must hold {n} x 5 x 3 floats, got {tuple(lu_params.shape)}")
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("kq_quantize_lu", _ptr(act), _ptr(lu_params), int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d,
-          _stream(stream))
+    _call("kq_quantize_lu", act.device, _ptr(act), _ptr(lu_params), int(bool(shared)), _ptr(out_codes),
+          _ptr(out_scales), M, d, _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -250,7 +264,8 @@ def fwht_quantize(act, H, out_codes=None, out_scales=None, stream=None):
     """Fixed-Hadamard (block size H) baseline quantizer."""
     M, d = _act(act)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("fwht_quantize", _ptr(act), int(H), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    _call("fwht_quantize", act.device, _ptr(act), int(H), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -265,8 +280,8 @@ def norm_kq_quantize(h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=
         raise ValueError("gamma and beta must be [nsamples, d]")
     _factors(factors, d, shared, h.device)
     out_codes, out_scales = _outs(h, out_codes, out_scales)
-    _call("norm_kq_quantize", _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps), _ptr(factors),
-          int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream))
+    _call("norm_kq_quantize", h.device, _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps),
+          _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream, h.device))
     return out_codes, out_scales
 
 
@@ -281,7 +296,8 @@ def kq_inverse_f32(y, factors, shared=False, out=None, stream=None):
     if out is None:
         out = torch.empty_like(y)
     _need(out, "out", torch.float32, y.device, (M, d))
-    _call("kq_inverse_f32", _ptr(y), _ptr(factors), int(bool(shared)), _ptr(out), M, d, _stream(stream))
+    _call("kq_inverse_f32", y.device, _ptr(y), _ptr(factors), int(bool(shared)), _ptr(out), M, d,
+          _stream(stream, y.device))
     return out
 
 
@@ -296,7 +312,7 @@ def mx_dequantize(codes, scales, out=None, stream=None):
     if out is None:
         out = torch.empty((M, d), dtype=torch.float32, device=codes.device)
     _need(out, "out", torch.float32, codes.device, (M, d))
-    _call("mx_dequantize", _ptr(codes), _ptr(scales), _ptr(out), M, d, _stream(stream))
+    _call("mx_dequantize", codes.device, _ptr(codes), _ptr(scales), _ptr(out), M, d, _stream(stream, codes.device))
     return out
 
 
@@ -306,8 +322,8 @@ def sq_quantize_variant(variant, act, mult, out_codes=None, out_scales=None, str
     M, d = _act(act)
     _need(mult, "mult", torch.float32, act.device, (d,))
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("sq_quantize_variant", int(variant), _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M, d,
-          _stream(stream))
+    _call("sq_quantize_variant", act.device, int(variant), _ptr(act), _ptr(mult), _ptr(out_codes), _ptr(out_scales), M,
+          d, _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -315,8 +331,8 @@ def mx_quantize_variant(variant, act, out_codes=None, out_scales=None, stream=No
     """The plain MXFP4 quantizer through a chosen kernel variant (0 = the default)."""
     M, d = _act(act)
     out_codes, out_scales = _outs(act, out_codes, out_scales)
-    _call("mx_quantize_variant", int(variant), _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d,
-          _stream(stream))
+    _call("mx_quantize_variant", act.device, int(variant), _ptr(act), _ptr(out_codes), _ptr(out_scales), M, d,
+          _stream(stream, act.device))
     return out_codes, out_scales
 
 
@@ -331,7 +347,7 @@ def kq_wait_timeouts(reset: bool = False) -> int:
 
 def kq_selftest_bounded_wait(stream=None) -> None:
     """Launch one staged CTA whose waits run out (no copies issued); see the C header."""
-    _call("kq_selftest_bounded_wait", _stream(stream))
+    _call("kq_selftest_bounded_wait", None, _stream(stream, None))
 
 
 def kq_fold_weights(W, factors, shared=False, out=None, stream=None):
@@ -345,7 +361,8 @@ def kq_fold_weights(W, factors, shared=False, out=None, stream=None):
     if out is None:
         out = torch.empty_like(W)
     _need(out, "out", torch.float32, W.device, (N, d))
-    _call("kq_fold_weights", _ptr(W), _ptr(factors), int(bool(shared)), _ptr(out), N, d, _stream(stream))
+    _call("kq_fold_weights", W.device, _ptr(W), _ptr(factors), int(bool(shared)), _ptr(out), N, d,
+          _stream(stream, W.device))
     return out
 
 
@@ -357,8 +374,8 @@ def kq_transform_f32_variant(variant, act, factors, shared=False, out=None, stre
     if out is None:
         out = torch.empty((M, d), dtype=torch.float32, device=act.device)
     _need(out, "out", torch.float32, act.device, (M, d))
-    _call("kq_transform_f32_variant", int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d,
-          _stream(stream))
+    _call("kq_transform_f32_variant", act.device, int(variant), _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out),
+          M, d, _stream(stream, act.device))
     return out
 
 
@@ -370,7 +387,8 @@ def kq_transform_f32(act, factors, shared=False, out=None, stream=None):
     if out is None:
         out = torch.empty((M, d), dtype=torch.float32, device=act.device)
     _need(out, "out", torch.float32, act.device, (M, d))
-    _call("kq_transform_f32", _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d, _stream(stream))
+    _call("kq_transform_f32", act.device, _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out), M, d,
+          _stream(stream, act.device))
     return out
 
 
@@ -400,8 +418,8 @@ def kq_quantize_sf(act, factors, shared=False, out_codes=None, out_sf=None, stre
         out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=act.device)
     _need(out_codes, "out_codes", torch.uint8, act.device, (M, d // 2))
     out_sf = _sf_out(out_sf, M, d, act.device)
-    _call("kq_quantize_sf", _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M, d,
-          _stream(stream))
+    _call("kq_quantize_sf", act.device, _ptr(act), _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M,
+          d, _stream(stream, act.device))
     return out_codes, out_sf
 
 
@@ -424,8 +442,8 @@ def mx_quantize_f32(x, sf_layout=False, out_codes=None, out_scales=None, stream=
         if out_scales is None:
             out_scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
         _need(out_scales, "out_scales", torch.uint8, x.device, (M, d // 32))
-    _call("mx_quantize_f32", _ptr(x), _ptr(out_codes), _ptr(out_scales),
-          KQ_SCALES_SF if sf_layout else KQ_SCALES_ROWMAJOR, M, d, _stream(stream))
+    _call("mx_quantize_f32", x.device, _ptr(x), _ptr(out_codes), _ptr(out_scales),
+          KQ_SCALES_SF if sf_layout else KQ_SCALES_ROWMAJOR, M, d, _stream(stream, x.device))
     return out_codes, out_scales
 
 
@@ -437,7 +455,7 @@ def mx_scales_to_sf(scales, out_sf=None, stream=None):
         raise ValueError("scales must be 2-D [M, d/32]")
     M, d = scales.shape[0], scales.shape[1] * 32
     out_sf = _sf_out(out_sf, M, d, scales.device)
-    _call("mx_scales_to_sf", _ptr(scales), _ptr(out_sf), M, d, _stream(stream))
+    _call("mx_scales_to_sf", scales.device, _ptr(scales), _ptr(out_sf), M, d, _stream(stream, scales.device))
     return out_sf
 
 
@@ -469,8 +487,8 @@ def mxf4_gemm_variant(variant, a_codes, a_sf, b_codes, b_sf, out=None, out_dtype
     if out.dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("out must be bfloat16 or float32")
     _need(out, "out", out.dtype, dev, (M, N))
-    _call("mxf4_gemm_variant", int(variant), _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
-          int(out.dtype == torch.float32), M, N, K, _stream(stream))
+    _call("mxf4_gemm_variant", dev, int(variant), _ptr(a_codes), _ptr(a_sf), _ptr(b_codes), _ptr(b_sf), _ptr(out),
+          int(out.dtype == torch.float32), M, N, K, _stream(stream, dev))
     return out
 
 
@@ -487,6 +505,6 @@ def norm_kq_quantize_sf(h, gamma, beta, factors, eps=1e-6, shared=False, out_cod
         out_codes = torch.empty((M, d // 2), dtype=torch.uint8, device=h.device)
     _need(out_codes, "out_codes", torch.uint8, h.device, (M, d // 2))
     out_sf = _sf_out(out_sf, M, d, h.device)
-    _call("norm_kq_quantize_sf", _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps), _ptr(factors),
-          int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M, d, _stream(stream))
+    _call("norm_kq_quantize_sf", h.device, _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps),
+          _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_sf), M, d, _stream(stream, h.device))
     return out_codes, out_sf
