@@ -46,8 +46,13 @@
  *     16 bytes; out_scales 1 byte.
  *   - Input with a non-finite value (inf/NaN) is outside the contract: such a
  *     block's outputs are unspecified (but written in bounds).
- *   - Calls on different streams that write the same output race; nothing else
- *     is shared between calls.
+ *   - Work runs on the calling thread's current CUDA device: every pointer and
+ *     `stream` must belong to it.  Device properties the launches need (SM
+ *     count, occupancy, shared-memory opt-ins, tile choices) are looked up
+ *     once per device and kept in thread-safe process-wide caches.
+ *   - Calls on different streams that write the same output race; besides
+ *     those caches and the bounded-wait counter (kq_wait_timeouts), nothing is
+ *     shared between calls.  Calls may come from several host threads.
  */
 #ifndef KROQUANT_H
 #define KROQUANT_H
