@@ -9,53 +9,65 @@
 // rounding); X is bf16 already, so each of the three products is exact in the
 // fp32 accumulator and Y_j = X_j K_hi^T + X_j K_mid^T + X_j K_lo^T.
 //
+// The three splits of a block are stacked along N (rows 0-31, 32-63 and
+// 64-95 of one K-major B matrix), so one M128 N96 K16 MMA per k-step computes
+// all three partial products of a block from one read of its A slice; the
+// epilogue adds them in fp32 as (hi + mid) + lo.
+//
 // A CTA owns one SM (1 CTA/SM, persistent) and walks a contiguous range of
-// tiles in group-major order: a tile is 128 rows x kNC block columns; the
+// tiles in group-major order: a tile is 128 rows x kNC = 2 block columns; the
 // tiles of one column group share the B operands, which are rebuilt only when
 // the group changes.
 //   warp 0     producer: builds the B operands of a column group (K_j split
 //              into 3 bf16 matrices, K-major, 64-byte swizzle) into one of
-//              two B buffers, and issues the TMA loads of the A tiles (two
-//              {64 cols x 128 rows} boxes, 128-byte swizzle) into a 4-stage ring
+//              two B buffers, and issues the TMA load of each A tile (one
+//              {64 cols x 128 rows} box, 128-byte swizzle) into an 8-stage ring
 //   warp 1     allocates the tensor memory; one thread issues the MMAs:
-//              2 k-steps x 3 splits x kNC block columns of M128 N32 K16 per
-//              tile (columns innermost) into one of two 128-column fp32
-//              accumulators
-//   warps 2-17 epilogue: tcgen05.ld of a row's 32 values of a block, amax,
-//              E8M0 byte, exact 2^-e scaling (packed FFMA with +0, so exact
-//              zeros come out +0 as in the other variants), E2M1.  Warp w reads
-//              TMEM lanes 32 (w % 4) .. +31 of block column (w - 2) / 4 and
-//              releases the accumulator at once; the codes of a tile are
-//              gathered in shared memory (double-buffered) and written by one
-//              TMA tensor store, the scales by one 4-byte store per row.
+//              2 k-steps x kNC block columns of M128 N96 K16 per tile into
+//              one of two accumulators (a 128-column slot per block column,
+//              96 columns used)
+//   warps 2-9  epilogue: tcgen05.ld of a row's 3 x 32 partial values of a
+//              block, their sum, amax, E8M0 byte, exact 2^-e scaling (packed
+//              FFMA with +0, so exact zeros come out +0 as in the other
+//              variants), E2M1.  Warp w reads TMEM lanes 32 (w % 4) .. +31 of
+//              block column (w - 2) / 4 and releases the accumulator at once;
+//              the codes of a tile are gathered in shared memory (double-
+//              buffered) and written by one TMA tensor store, the scales by
+//              one 2-byte store per row.
 // Every mbarrier wait is bounded (g_wait_timeouts); the tensor memory is
 // freed on every path.
 
 namespace mma {
 
-constexpr int kNC = 4;                                   // block columns per tile
+constexpr int kNC = 2;                                   // block columns per tile
 constexpr int kRows = 128;                               // tile rows (MMA M)
-constexpr int kAStages = 4;
+constexpr int kAStages = 8;
 constexpr int kABoxBytes = kRows * 128;                  // {64 cols x 128 rows} bf16 = 16 KB
-constexpr int kAStageBytes = 2 * kABoxBytes;             // kNC = 4 block columns: 32 KB
+constexpr int kAStageBytes = kABoxBytes;                 // kNC = 2 block columns: one box
 constexpr int kBMatBytes = 32 * 64;                      // one 32 x 32 bf16 matrix: 2 KB
-constexpr int kBSetBytes = kNC * 3 * kBMatBytes;         // 24 KB
-constexpr int kTmemCols = 2 * kNC * 32;                  // two accumulators of kNC x 32 columns
-constexpr int kEpiWarps = 16;                            // 4 lane quarters x kNC block columns
+constexpr int kBSetBytes = kNC * 3 * kBMatBytes;         // 12 KB
+constexpr int kMmaN = 96;                                // the three splits of a block
+constexpr int kAccCols = 128;                            // accumulator slot per block column (96 used)
+constexpr int kTmemCols = 2 * kNC * kAccCols;            // two accumulators: 512 columns
+constexpr int kEpiWarps = 4 * kNC;                       // 4 lane quarters x kNC block columns
 constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kThreads = 64 + kEpiThreads;               // 576
-constexpr int kCodesTileBytes = kRows * kNC * 16;        // 8 KB of codes per tile
-constexpr int kScalesTileBytes = kRows * kNC;            // 512 B of scales per tile
+constexpr int kThreads = 64 + kEpiThreads;               // 320
+constexpr int kCodesTileBytes = kRows * kNC * 16;        // 4 KB of codes per tile
+constexpr int kScalesTileBytes = kRows * kNC;            // 256 B of scales per tile
 constexpr size_t kSmemA = size_t(kAStages) * kAStageBytes;
 constexpr size_t kSmemB = 2 * size_t(kBSetBytes);
 constexpr size_t kSmemOut = 2 * size_t(kCodesTileBytes + kScalesTileBytes);
-constexpr size_t kSmemBars = 16 * sizeof(uint64_t) + 16;
+constexpr int kNumBars = 2 * kAStages + 8;               // A ring, accumulators, B sets
+constexpr size_t kSmemBars = kNumBars * sizeof(uint64_t) + 16;
 constexpr size_t kSmem = kSmemA + kSmemB + kSmemOut + kSmemBars + 1024;
+static_assert(kNC == 2, "one A box per tile and a 2-byte scale store per row");
+static_assert(kTmemCols <= 512, "tensor memory columns");
+static_assert(kSmemB % 1024 == 0 && kSmemA % 1024 == 0, "operand buffers keep the swizzle alignment");
 
 // Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
 // = 1), B bf16 (bits 10-12 = 1), A and B K-major (bits 15, 16 = 0),
 // N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(32 >> 3) << 17) |
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kMmaN >> 3) << 17) |
                             (uint32_t(kRows >> 4) << 24);
 
 // Shared-memory matrix descriptor: start address >> 4 (bits 0-13), leading
@@ -90,14 +102,15 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective),
+// without the wait: the caller issues several loads and then one
+// tcgen05.wait::ld before reading any of them.
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32])
 {
     uint32_t r[32];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -214,13 +227,13 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
     uint8_t *sB = base + kSmemA;
     uint8_t *sOut = sB + kSmemB;                               // [2] x (codes tile, scales tile)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sOut + kSmemOut);
-    uint64_t *full_a = bars;          // [kAStages] A tile landed (TMA tx)
-    uint64_t *empty_a = bars + 4;     // [kAStages] MMAs reading the stage done (commit)
-    uint64_t *tfull = bars + 8;       // [2] accumulator ready (commit)
-    uint64_t *tempty = bars + 10;     // [2] accumulator read by the epilogue warps
-    uint64_t *bfull = bars + 12;      // [2] B set built
-    uint64_t *bempty = bars + 14;     // [2] MMAs reading the B set done (commit)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    uint64_t *full_a = bars;                  // [kAStages] A tile landed (TMA tx)
+    uint64_t *empty_a = bars + kAStages;      // [kAStages] MMAs reading the stage done (commit)
+    uint64_t *tfull = bars + 2 * kAStages;    // [2] accumulator ready (commit)
+    uint64_t *tempty = tfull + 2;             // [2] accumulator read by the epilogue warps
+    uint64_t *bfull = tfull + 4;              // [2] B set built
+    uint64_t *bempty = tfull + 6;             // [2] MMAs reading the B set done (commit)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     const int64_t RT = (M + kRows - 1) / kRows;
@@ -286,7 +299,6 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
                     mbar_expect_tx(&full_a[s], kAStageBytes);
                     uint8_t *st = sA + size_t(s) * kAStageBytes;
                     tma_load_2d(st, &act_map, g * kNC * 32, int32_t(rt * kRows), &full_a[s]);
-                    tma_load_2d(st + kABoxBytes, &act_map, g * kNC * 32 + 64, int32_t(rt * kRows), &full_a[s]);
                     filled = k + 1;
                 }
             }
@@ -327,22 +339,18 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
                 tc_fence_after();
                 const uint32_t a0 = smem_addr(sA + size_t(s) * kAStageBytes);
                 const uint32_t b0 = smem_addr(sB + (bcount & 1) * kBSetBytes);
-                // Consecutive MMAs go to different accumulators (block column
-                // innermost): the six MMAs that accumulate into one column are
-                // kNC issues apart, so their latencies overlap instead of
-                // serialising.
+                // Block column innermost: the two MMAs that accumulate into
+                // one slot are kNC issues apart.  Block column jj's 32 A
+                // columns are bytes 64 jj .. 64 jj + 63 of the 128-byte rows;
+                // its B matrix is the 96 stacked split rows.
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
 #pragma unroll
-                    for (int sp = 0; sp < 3; ++sp) {
-#pragma unroll
-                        for (int jj = 0; jj < kNC; ++jj) {
-                            const uint32_t d = tmem_base + uint32_t(tb * kNC * 32 + jj * 32);
-                            const uint64_t ad =
-                                smem_desc(a0 + (jj >> 1) * kABoxBytes + (jj & 1) * 64 + kk * 32, 1024, kLayoutSw128);
-                            const uint64_t bd = smem_desc(b0 + (jj * 3 + sp) * kBMatBytes + kk * 32, 512, kLayoutSw64);
-                            umma_bf16(d, ad, bd, (sp | kk) != 0);
-                        }
+                    for (int jj = 0; jj < kNC; ++jj) {
+                        const uint32_t d = tmem_base + uint32_t(tb * kNC * kAccCols + jj * kAccCols);
+                        const uint64_t ad = smem_desc(a0 + jj * 64 + kk * 32, 1024, kLayoutSw128);
+                        const uint64_t bd = smem_desc(b0 + jj * 3 * kBMatBytes + kk * 32, 512, kLayoutSw64);
+                        umma_bf16(d, ad, bd, kk != 0);
                     }
                 }
                 umma_commit(&empty_a[s]);
@@ -376,12 +384,25 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
             const int rloc = q * 32 + lane;                 // row within the tile
             const int64_t row = rt * kRows + rloc;
             const int j = g * kNC + jj;
-            float v[32];
-            tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(tb * kNC * 32 + jj * 32), v);
+            // the three partial products (hi, mid, lo), then their fp32 sum
+            float v[32], u[32], w[32];
+            const uint32_t tcol = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(tb * kNC * kAccCols + jj * kAccCols);
+            tmem_ld32_nowait(tcol, v);
+            tmem_ld32_nowait(tcol + 32, u);
+            tmem_ld32_nowait(tcol + 64, w);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             // the accumulator has been read: hand it back to the MMA thread
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[tb]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float2 s = __fadd2_rn(__fadd2_rn(make_float2(v[2 * i], v[2 * i + 1]),
+                                                       make_float2(u[2 * i], u[2 * i + 1])),
+                                            make_float2(w[2 * i], w[2 * i + 1]));
+                v[2 * i] = s.x;
+                v[2 * i + 1] = s.y;
+            }
 
             if constexpr (OUT == KqOut::kF32) {
                 if (row < M && j < nb) {
@@ -425,14 +446,14 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
                 if (jj == 0 && row < M) {
-                    // this row's kNC scale bytes, one 4-byte store where the row layout allows it
+                    // this row's kNC = 2 scale bytes, one 2-byte store where the row layout allows it
                     const int nj = nb - g * kNC < kNC ? nb - g * kNC : kNC;
                     uint8_t *dst = scales + row * nb + int64_t(g) * kNC;
-                    const uint32_t w4 = *reinterpret_cast<const uint32_t *>(oscales + rloc * kNC);
-                    if (nj == kNC && (reinterpret_cast<uintptr_t>(dst) & 3) == 0) {
-                        *reinterpret_cast<uint32_t *>(dst) = w4;
+                    const uint8_t *src = oscales + rloc * kNC;
+                    if (nj == kNC && (reinterpret_cast<uintptr_t>(dst) & 1) == 0) {
+                        *reinterpret_cast<uint16_t *>(dst) = *reinterpret_cast<const uint16_t *>(src);
                     } else {
-                        for (int e = 0; e < nj; ++e) dst[e] = uint8_t(w4 >> (8 * e));
+                        for (int e = 0; e < nj; ++e) dst[e] = src[e];
                     }
                 }
             }
