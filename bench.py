@@ -33,6 +33,8 @@ Other modes (one JSON line each):
     --mode gemm --shape MxNxK [--kernels v]  the W4A4 product, its tile configurations,
                                              and the chains quantize -> product and
                                              norm + quantize -> product
+    --mode compare --kernels a,b --shapes MxD,...  several quantizers interleaved in one
+                                             process, --reps rounds (one line per timing)
 """
 from __future__ import annotations
 
@@ -841,6 +843,42 @@ def sweep_mode(args):
             json.dump({"peak": peak, "peak_source": src, "rows": rows}, fh, indent=1)
 
 
+def compare_mode(args):
+    """Several quantizers side by side at each shape of --shapes, in one process.
+
+    The kernels are timed in turn, and the whole round is repeated --reps
+    times, so clock and thermal drift fall on all of them alike.  Each
+    measurement is time_launches over RotatingInputs, as in kernel mode.
+    """
+    import torch
+
+    from w4a4_mxfp4_post_b200 import build
+
+    build.build()
+    dev = torch.device("cuda:0")
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2 ** 20))
+    peak, src = measured_peak()
+    stream = torch.cuda.Stream(device=dev)
+    kinds = args.kernels.split(",")
+    rows = []
+    for shape in args.shapes.split(","):
+        M, d = (int(t) for t in shape.lower().split("x"))
+        inp = RotatingInputs(M, d, dev, l2)
+        for rep in range(args.reps):
+            for kind in kinds:
+                r = time_launches(kind, inp, args.launches, args.warmup, stream)
+                gbs = BYTES_PER_ELEM * M * d / (r["mean_us"] * 1e-6) / 1e9
+                row = {"mode": "compare", "M": M, "d": d, "kernel": kind, "rep": rep, "us": round(r["mean_us"], 3),
+                       "gbs": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4)}
+                rows.append(row)
+                print(json.dumps(row), flush=True)
+        del inp
+        torch.cuda.empty_cache()
+    if args.json_out:
+        with open(args.json_out, "w") as fh:
+            json.dump({"peak": peak, "peak_source": src, "rows": rows}, fh, indent=1)
+
+
 def sqnr_mode(args):
     """Quantisation-error proxy: SQNR of the round trip x -> codes/scales -> x^ per method.
 
@@ -923,17 +961,21 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the cpu_baseline block")
     ap.add_argument("--ref-seconds", type=float, default=60.0, help="budget of the reference arm")
     ap.add_argument("--json-out", default="")
-    ap.add_argument("--mode", choices=["step", "kernel", "sweep", "sqnr", "gemm"], default="step",
+    ap.add_argument("--mode", choices=["step", "kernel", "sweep", "sqnr", "gemm", "compare"], default="step",
                     help="step: the benchmark line; kernel: one quantizer at --shape; sweep: all shapes; "
-                         "sqnr: quantisation-error proxy per method")
+                         "sqnr: quantisation-error proxy per method; gemm: the W4A4 product; "
+                         "compare: several quantizers interleaved at --shapes")
     ap.add_argument("--kernel", default="kq",
                     help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H> or norm_kq")
     ap.add_argument("--kernels", default="kq,sq,mx",
-                    help="sweep mode: comma-separated kernels; gemm mode: comma-separated tile configurations")
+                    help="sweep / compare mode: comma-separated kernels; gemm mode: comma-separated tile "
+                         "configurations")
     ap.add_argument("--shape", default="8192x12288", help="kernel mode: MxD; gemm mode: MxNxK")
     ap.add_argument("--budget-mb", type=int, default=0, help="kernel mode: total input rotation bytes")
     ap.add_argument("--no-graph", action="store_true", help="kernel mode: eager launches")
-    ap.add_argument("--launches", type=int, default=100, help="kernel / sweep mode: timed launches")
+    ap.add_argument("--launches", type=int, default=100, help="kernel / sweep / compare mode: timed launches")
+    ap.add_argument("--shapes", default="8192x4608,8192x1152", help="compare mode: comma-separated MxD")
+    ap.add_argument("--reps", type=int, default=3, help="compare mode: rounds over the kernels")
     args = ap.parse_args()
     if args.mode == "kernel":
         return kernel_mode(args)
@@ -943,6 +985,8 @@ def main():
         return sqnr_mode(args)
     if args.mode == "gemm":
         return gemm_mode(args)
+    if args.mode == "compare":
+        return compare_mode(args)
     if args.steps < 1 or args.warmup < 3:
         raise SystemExit("need --steps >= 1 and --warmup >= 3")
 

@@ -16,24 +16,26 @@
 //
 // A CTA owns one SM (1 CTA/SM, persistent) and walks a contiguous range of
 // tiles in group-major order: a tile is 128 rows x kNC = 2 block columns; the
-// tiles of one column group share the B operands, which are rebuilt only when
-// the group changes.
-//   warp 0     producer: builds the B operands of a column group (K_j split
-//              into 3 bf16 matrices, K-major, 64-byte swizzle) into one of
-//              two B buffers, and issues the TMA load of each A tile (one
-//              {64 cols x 128 rows} box, 128-byte swizzle) into an 8-stage ring
-//   warp 1     allocates the tensor memory; one thread issues the MMAs:
-//              2 k-steps x kNC block columns of M128 N96 K16 per tile into
-//              one of two accumulators (a 128-column slot per block column,
-//              96 columns used)
-//   warps 2-9  epilogue: tcgen05.ld of a row's 3 x 32 partial values of a
-//              block, their sum, amax, E8M0 byte, exact 2^-e scaling (packed
-//              FFMA with +0, so exact zeros come out +0 as in the other
-//              variants), E2M1.  Warp w reads TMEM lanes 32 (w % 4) .. +31 of
-//              block column (w - 2) / 4 and releases the accumulator at once;
-//              the codes of a tile are gathered in shared memory (double-
-//              buffered) and written by one TMA tensor store, the scales by
-//              one 2-byte store per row.
+// tiles of one column group share the B operands.
+//   warp 0      producer: the TMA load of each A tile (one {64 cols x 128
+//               rows} box, 128-byte swizzle) into an 8-stage ring
+//   warp 1      allocates the tensor memory; one thread issues the MMAs:
+//               2 k-steps x kNC block columns of M128 N96 K16 per tile into
+//               accumulator k % 2 (a 128-column slot per block column, 96
+//               columns used)
+//   warps 2-9   epilogue, two groups of four warps (one per TMEM lane quarter)
+//               taking alternate tiles, so each group owns one accumulator:
+//               a warp reads its 32 rows' 3 x 32 partial values of both block
+//               columns, sums them, releases the accumulator, and quantizes
+//               (amax, E8M0 byte, exact 2^-e scaling by a packed FFMA with +0,
+//               so exact zeros come out +0 as in the other variants, E2M1).
+//               It writes its 32 x 32 bytes of codes with its own TMA store
+//               (through a 1 KB staging buffer) and each row's two scale bytes
+//               with one 2-byte store.  No barrier joins the epilogue warps.
+//   warps 10-13 B builders: at each column-group change they build the group's
+//               B set (K_j split into 3 bf16 matrices, K-major, 64-byte
+//               swizzle), two of its eight parts per warp, into the B buffer
+//               the MMAs released, one set ahead of the MMAs.
 // Every mbarrier wait is bounded (g_wait_timeouts); the tensor memory is
 // freed on every path.
 
@@ -49,20 +51,21 @@ constexpr int kBSetBytes = kNC * 3 * kBMatBytes;         // 12 KB
 constexpr int kMmaN = 96;                                // the three splits of a block
 constexpr int kAccCols = 128;                            // accumulator slot per block column (96 used)
 constexpr int kTmemCols = 2 * kNC * kAccCols;            // two accumulators: 512 columns
-constexpr int kEpiWarps = 4 * kNC;                       // 4 lane quarters x kNC block columns
-constexpr int kEpiThreads = 32 * kEpiWarps;
-constexpr int kThreads = 64 + kEpiThreads;               // 320
-constexpr int kCodesTileBytes = kRows * kNC * 16;        // 4 KB of codes per tile
-constexpr int kScalesTileBytes = kRows * kNC;            // 256 B of scales per tile
+constexpr int kEpiWarps = 8;                             // two groups of 4 lane quarters
+constexpr int kBuildWarps = 4;                           // B builders, two of the 8 parts of a set each
+constexpr int kThreads = 64 + 32 * (kEpiWarps + kBuildWarps);   // 448
+constexpr int kStoreRows = 32;                           // codes store box: a warp's rows x kNC * 16 bytes
+constexpr int kWarpOutBytes = kStoreRows * kNC * 16;     // 1 KB of codes per warp and tile
 constexpr size_t kSmemA = size_t(kAStages) * kAStageBytes;
 constexpr size_t kSmemB = 2 * size_t(kBSetBytes);
-constexpr size_t kSmemOut = 2 * size_t(kCodesTileBytes + kScalesTileBytes);
+constexpr size_t kSmemOut = size_t(kEpiWarps) * kWarpOutBytes;
 constexpr int kNumBars = 2 * kAStages + 8;               // A ring, accumulators, B sets
 constexpr size_t kSmemBars = kNumBars * sizeof(uint64_t) + 16;
 constexpr size_t kSmem = kSmemA + kSmemB + kSmemOut + kSmemBars + 1024;
-static_assert(kNC == 2, "one A box per tile and a 2-byte scale store per row");
+static_assert(kNC == 2, "one A box per tile; a row's two scale bytes in one store");
 static_assert(kTmemCols <= 512, "tensor memory columns");
 static_assert(kSmemB % 1024 == 0 && kSmemA % 1024 == 0, "operand buffers keep the swizzle alignment");
+static_assert(kWarpOutBytes % 128 == 0, "TMA store sources stay 128-byte aligned");
 
 // Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
 // = 1), B bf16 (bits 10-12 = 1), A and B K-major (bits 15, 16 = 0),
@@ -130,62 +133,59 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Build the B operands of column group g into `dst` (warp-collective; lane n
-// writes row n of every matrix): for block column jj (j = g*kNC + jj) and
-// split s, matrix (jj, s) holds part s of K_j as 32 rows n x 32 columns l
-// (K-major, B[n][l] = K_j[n][l], since Y = X K^T), in the 64-byte swizzle
-// layout: row n at n*64, its 16-byte chunk c at chunk c ^ ((n >> 1) & 3).
-__device__ void build_b_operands(uint8_t *dst, const float4 *__restrict__ factors, int shared, int g, int nb,
-                                 int lane)
+// Part `part` = 4 jj + c of the B operands of column group g (warp-
+// collective; lane n writes row n): chunk c (columns l = 8c .. 8c+7) of row n
+// of the three split matrices of block column jj (j = g*kNC + jj).  Matrix
+// (jj, s) holds part s of K_j as 32 rows n x 32 columns l (K-major,
+// B[n][l] = K_j[n][l], since Y = X K^T), in the 64-byte swizzle layout: row n
+// at n*64, its 16-byte chunk c at chunk c ^ ((n >> 1) & 3).  The three
+// matrices of a block column are consecutive, so they form one 96-row
+// matrix in the same layout.
+__device__ void build_b_part(uint8_t *dst, const float4 *__restrict__ factors, int shared, int g, int nb, int lane,
+                             int part)
 {
+    const int jj = part >> 2, c = part & 3;
     const int n = lane;
     const int sw = (n >> 1) & 3;
-#pragma unroll 1
-    for (int jj = 0; jj < kNC; ++jj) {
-        const int j = g * kNC + jj;
-        float r[5][2];
-        if (j < nb) {
-            const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
+    const int j = g * kNC + jj;
+    float r[5][2];
+    if (j < nb) {
+        const float4 *fp = factors + (shared ? 0 : int64_t(j) * 5);
 #pragma unroll
-            for (int k = 0; k < 5; ++k) {
-                const float4 f = __ldg(fp + k);            // [g00, g01, g10, g11] of G_(k+1)
-                const int bn = (n >> (4 - k)) & 1;          // G_(k+1) acts on index bit 4-k
-                r[k][0] = bn ? f.z : f.x;
-                r[k][1] = bn ? f.w : f.y;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 5; ++k) r[k][0] = r[k][1] = 0.0f;
+        for (int k = 0; k < 5; ++k) {
+            const float4 f = __ldg(fp + k);            // [g00, g01, g10, g11] of G_(k+1)
+            const int bn = (n >> (4 - k)) & 1;          // G_(k+1) acts on index bit 4-k
+            r[k][0] = bn ? f.z : f.x;
+            r[k][1] = bn ? f.w : f.y;
         }
-        // one 16-byte chunk (8 columns l) of the row at a time
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float part[8];
+    } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int l = 8 * c + e;
-                const float a0 = ((l >> 4) & 1) ? r[0][1] : r[0][0];
-                const float a1 = ((l >> 3) & 1) ? r[1][1] : r[1][0];
-                const float a2 = ((l >> 2) & 1) ? r[2][1] : r[2][0];
-                const float a3 = ((l >> 1) & 1) ? r[3][1] : r[3][0];
-                const float a4 = (l & 1) ? r[4][1] : r[4][0];
-                part[e] = a0 * a1 * a2 * a3 * a4;
-            }
+        for (int k = 0; k < 5; ++k) r[k][0] = r[k][1] = 0.0f;
+    }
+    float part_v[8];
 #pragma unroll
-            for (int sp = 0; sp < 3; ++sp) {
-                // part sp of the split: round to bf16, carry the exact remainder on
-                uint32_t w[4];
+    for (int e = 0; e < 8; ++e) {
+        const int l = 8 * c + e;
+        const float a0 = ((l >> 4) & 1) ? r[0][1] : r[0][0];
+        const float a1 = ((l >> 3) & 1) ? r[1][1] : r[1][0];
+        const float a2 = ((l >> 2) & 1) ? r[2][1] : r[2][0];
+        const float a3 = ((l >> 1) & 1) ? r[3][1] : r[3][0];
+        const float a4 = (l & 1) ? r[4][1] : r[4][0];
+        part_v[e] = a0 * a1 * a2 * a3 * a4;
+    }
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const __nv_bfloat16 ha = __float2bfloat16_rn(part[e]), hb = __float2bfloat16_rn(part[e + 1]);
-                    part[e] -= __bfloat162float(ha);
-                    part[e + 1] -= __bfloat162float(hb);
-                    w[e / 2] = uint32_t(__bfloat16_as_ushort(ha)) | (uint32_t(__bfloat16_as_ushort(hb)) << 16);
-                }
-                *reinterpret_cast<uint4 *>(dst + (jj * 3 + sp) * kBMatBytes + n * 64 + 16 * (c ^ sw)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-            }
+    for (int sp = 0; sp < 3; ++sp) {
+        // part sp of the split: round to bf16, carry the exact remainder on
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const __nv_bfloat16 ha = __float2bfloat16_rn(part_v[e]), hb = __float2bfloat16_rn(part_v[e + 1]);
+            part_v[e] -= __bfloat162float(ha);
+            part_v[e + 1] -= __bfloat162float(hb);
+            w[e / 2] = uint32_t(__bfloat16_as_ushort(ha)) | (uint32_t(__bfloat16_as_ushort(hb)) << 16);
         }
+        *reinterpret_cast<uint4 *>(dst + (jj * 3 + sp) * kBMatBytes + n * 64 + 16 * (c ^ sw)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -197,22 +197,43 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int32_t x, 
                  : "memory");
 }
 
-// Named barrier among the epilogue warps only (id 1; id 0 is __syncthreads).
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
-
-// AND of `pred` over all epilogue threads (barrier id 2): makes a give-up
-// decision uniform across the epilogue warps, which share named barriers.
-__device__ __forceinline__ bool epi_all(bool pred)
+// Sum of the three partial products of one block column at TMEM address
+// `tcol` (this warp's lane quarter): (hi + mid) + lo in fp32.
+__device__ __forceinline__ void load_block_sum(uint32_t tcol, float (&y)[32])
 {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\t"
-                 "setp.ne.b32 p, %1, 0;\n\t"
-                 "bar.red.and.pred q, 2, %2, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r)
-                 : "r"(uint32_t(pred)), "n"(kEpiThreads)
-                 : "memory");
-    return r != 0;
+    float u[32], w[32];
+    tmem_ld32_nowait(tcol, y);
+    tmem_ld32_nowait(tcol + 32, u);
+    tmem_ld32_nowait(tcol + 64, w);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 s = __fadd2_rn(__fadd2_rn(make_float2(y[2 * i], y[2 * i + 1]), make_float2(u[2 * i], u[2 * i + 1])),
+                                    make_float2(w[2 * i], w[2 * i + 1]));
+        y[2 * i] = s.x;
+        y[2 * i + 1] = s.y;
+    }
+}
+
+// MXFP4 of one block's 32 transformed values (amax, E8M0 byte, exact 2^-e
+// scaling by a packed FFMA with +0, E2M1).
+__device__ __forceinline__ void quantize_block32(float (&v)[32], uint4 &cw, uint32_t &sb)
+{
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = max3_abs(amax, v[2 * i], v[2 * i + 1]);
+    sb = e8m0_byte(amax);
+    const float sc = inv_scale(sb);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 pr = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), make_float2(sc, sc), plus_zero2());
+        v[2 * i] = pr.x;
+        v[2 * i + 1] = pr.y;
+    }
+    cw.x = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    cw.y = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+    cw.z = cvt_e2m1x8(v[16], v[17], v[18], v[19], v[20], v[21], v[22], v[23]);
+    cw.w = cvt_e2m1x8(v[24], v[25], v[26], v[27], v[28], v[29], v[30], v[31]);
 }
 
 template <KqOut OUT>
@@ -225,13 +246,13 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
     uint8_t *sB = base + kSmemA;
-    uint8_t *sOut = sB + kSmemB;                               // [2] x (codes tile, scales tile)
+    uint8_t *sOut = sB + kSmemB;                               // [kEpiWarps] x a warp's codes (32 rows x 32 bytes)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sOut + kSmemOut);
     uint64_t *full_a = bars;                  // [kAStages] A tile landed (TMA tx)
     uint64_t *empty_a = bars + kAStages;      // [kAStages] MMAs reading the stage done (commit)
     uint64_t *tfull = bars + 2 * kAStages;    // [2] accumulator ready (commit)
-    uint64_t *tempty = tfull + 2;             // [2] accumulator read by the epilogue warps
-    uint64_t *bfull = tfull + 4;              // [2] B set built
+    uint64_t *tempty = tfull + 2;             // [2] accumulator read by its epilogue group
+    uint64_t *bfull = tfull + 4;              // [2] B set built (the builder warps)
     uint64_t *bempty = tfull + 6;             // [2] MMAs reading the B set done (commit)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -249,8 +270,8 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
-            mbar_init(&bfull[b], 1);
+            mbar_init(&tempty[b], 4);
+            mbar_init(&bfull[b], kBuildWarps);
             mbar_init(&bempty[b], 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -267,44 +288,23 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer: B sets and A tiles
-        int last_g = -1, buse = -1, k = 0, filled = 0;
-        bool ok = true;
-        for (int64_t t = t_begin; t < t_end && ok; ++t, ++k) {
-            const int g = int(t / RT);
-            const int64_t rt = t % RT;
-            if (g != last_g) {
-                ++buse;
-                const int bb = buse & 1;
-                // every lane waits (each acquires the release of the old B set);
-                // the give-up decision is made warp-uniform
-                const bool freed = buse < 2 || mbar_wait(&bempty[bb], ((buse >> 1) - 1) & 1, budget);
-                if (!__all_sync(0xffffffffu, freed)) {
-                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
-                    ok = false;
-                    break;
-                }
-                build_b_operands(sB + bb * kBSetBytes, factors, shared, g, nb, lane);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bfull[bb]);
-                last_g = g;
-            }
-            if (lane == 0) {
+        // ---------------- producer: A tiles (one thread)
+        if (lane == 0) {
+            int filled = 0;
+            int k = 0;
+            for (int64_t t = t_begin; t < t_end; ++t, ++k) {
+                const int g = int(t / RT);
+                const int64_t rt = t % RT;
                 const int s = k % kAStages;
                 if (k >= kAStages && !mbar_wait(&empty_a[s], ((k / kAStages) - 1) & 1, budget)) {
                     atomicAdd(&g_wait_timeouts, 1);
-                    ok = false;
-                } else {
-                    mbar_expect_tx(&full_a[s], kAStageBytes);
-                    uint8_t *st = sA + size_t(s) * kAStageBytes;
-                    tma_load_2d(st, &act_map, g * kNC * 32, int32_t(rt * kRows), &full_a[s]);
-                    filled = k + 1;
+                    break;
                 }
+                mbar_expect_tx(&full_a[s], kAStageBytes);
+                tma_load_2d(sA + size_t(s) * kAStageBytes, &act_map, g * kNC * 32, int32_t(rt * kRows), &full_a[s]);
+                filled = k + 1;
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        }
-        if (lane == 0) {   // drain: the copies issued have landed before the CTA may exit
+            // drain: the copies issued have landed before the CTA may exit
             for (int kk = (filled > kAStages ? filled - kAStages : 0); kk < filled; ++kk)
                 if (!mbar_wait(&full_a[kk % kAStages], (kk / kAStages) & 1, budget)) {
                     atomicAdd(&g_wait_timeouts, 1);
@@ -361,105 +361,110 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
             if (issued > 0 && !mbar_wait(&tfull[(issued - 1) & 1], ((issued - 1) >> 1) & 1, budget))
                 atomicAdd(&g_wait_timeouts, 1);
         }
-    } else {
-        // ---------------- epilogue warps: warp w reads TMEM lane quarter w % 4
-        // (tile rows 32q .. 32q+31) of block column (w - 2) / 4
+    } else if (warp < 2 + kEpiWarps) {
+        // ---------------- epilogue: group gr takes the tiles k with k % 2 == gr
+        // (accumulator gr); warp w reads TMEM lane quarter w % 4 (tile rows
+        // 32q .. 32q+31), both block columns
         const int q = warp & 3;
-        const int jj = (warp - 2) >> 2;
-        const int et = threadIdx.x - 64;                  // 0 .. kEpiThreads-1
-        const bool store_leader = (et == 0);
+        const int gr = (warp - 2) >> 2;
+        uint8_t *stg = sOut + size_t(warp - 2) * kWarpOutBytes;
         int k = 0;
         for (int64_t t = t_begin; t < t_end; ++t, ++k) {
-            const int g = int(t / RT);
-            const int64_t rt = t % RT;
-            const int tb = k & 1;
-            const bool ready = mbar_wait(&tfull[tb], (k >> 1) & 1, budget);
-            // uniform over the epilogue: tcgen05.ld is warp-collective and the
-            // epilogue warps meet at named barriers below
-            if (!epi_all(ready)) {
+            if ((k & 1) != gr) continue;
+            const int use = k >> 1;
+            const bool ready = mbar_wait(&tfull[gr], use & 1, budget);
+            if (!__all_sync(0xffffffffu, ready)) {   // tcgen05.ld below is warp-collective
                 if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                 break;
             }
             tc_fence_after();
-            const int rloc = q * 32 + lane;                 // row within the tile
-            const int64_t row = rt * kRows + rloc;
-            const int j = g * kNC + jj;
-            // the three partial products (hi, mid, lo), then their fp32 sum
-            float v[32], u[32], w[32];
-            const uint32_t tcol = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(tb * kNC * kAccCols + jj * kAccCols);
-            tmem_ld32_nowait(tcol, v);
-            tmem_ld32_nowait(tcol + 32, u);
-            tmem_ld32_nowait(tcol + 64, w);
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            // the accumulator has been read: hand it back to the MMA thread
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[tb]);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float2 s = __fadd2_rn(__fadd2_rn(make_float2(v[2 * i], v[2 * i + 1]),
-                                                       make_float2(u[2 * i], u[2 * i + 1])),
-                                            make_float2(w[2 * i], w[2 * i + 1]));
-                v[2 * i] = s.x;
-                v[2 * i + 1] = s.y;
-            }
-
+            const int g = int(t / RT);
+            const int64_t rt = t % RT;
+            const int64_t row0 = rt * kRows + q * 32;
+            const int64_t row = row0 + lane;
+            const int j0 = g * kNC;
+            const uint32_t tcol = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(gr * kNC * kAccCols);
+            float y[32];
             if constexpr (OUT == KqOut::kF32) {
-                if (row < M && j < nb) {
-                    // the fp32 transform itself (+0: exact zeros come out +0)
-                    float4 *yo = y_out + (row * nb + j) * 8;
+#pragma unroll 1
+                for (int jj = 0; jj < kNC; ++jj) {
+                    load_block_sum(tcol + jj * kAccCols, y);
+                    if (row < M && j0 + jj < nb) {
+                        // the fp32 transform itself (+0: exact zeros come out +0)
+                        float4 *yo = y_out + (row * nb + j0 + jj) * 8;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        yo[i] = make_float4(v[4 * i] + 0.0f, v[4 * i + 1] + 0.0f, v[4 * i + 2] + 0.0f,
-                                            v[4 * i + 3] + 0.0f);
+                        for (int i = 0; i < 8; ++i)
+                            yo[i] = make_float4(y[4 * i] + 0.0f, y[4 * i + 1] + 0.0f, y[4 * i + 2] + 0.0f,
+                                                y[4 * i + 3] + 0.0f);
+                    }
                 }
+                // both block columns have been read: hand the accumulator back
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[gr]);
             } else {
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) amax = max3_abs(amax, v[2 * i], v[2 * i + 1]);
-                const uint32_t sb = e8m0_byte(amax);
-                const float sc = inv_scale(sb);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 pr = __ffma2_rn(make_float2(v[2 * i], v[2 * i + 1]), make_float2(sc, sc), plus_zero2());
-                    v[2 * i] = pr.x;
-                    v[2 * i + 1] = pr.y;
-                }
-                uint4 cw;
-                cw.x = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
-                cw.y = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
-                cw.z = cvt_e2m1x8(v[16], v[17], v[18], v[19], v[20], v[21], v[22], v[23]);
-                cw.w = cvt_e2m1x8(v[24], v[25], v[26], v[27], v[28], v[29], v[30], v[31]);
-                // staging buffer k & 1: the tile store that read it two tiles ago must be done
-                uint8_t *ocodes = sOut + (k & 1) * (kCodesTileBytes + kScalesTileBytes);
-                uint8_t *oscales = ocodes + kCodesTileBytes;
-                if (store_leader) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                epi_sync();
-                // codes tile = rows x 64 bytes (the box of the codes tensor map, no swizzle)
-                *reinterpret_cast<uint4 *>(ocodes + rloc * (kNC * 16) + jj * 16) = cw;
-                oscales[rloc * kNC + jj] = uint8_t(sb);
+                uint4 cw0, cw1;
+                uint32_t sb0, sb1;
+                load_block_sum(tcol, y);
+                quantize_block32(y, cw0, sb0);
+                load_block_sum(tcol + kAccCols, y);
+                // both block columns have been read: hand the accumulator back
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[gr]);
+                quantize_block32(y, cw1, sb1);
+                // this warp's codes: 32 rows x 32 bytes through its staging
+                // buffer (the previous store has finished reading it) and one
+                // TMA store; rows past M and columns past d/2 are clipped
+                if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                __syncwarp();
+                *reinterpret_cast<uint4 *>(stg + lane * 32) = cw0;
+                *reinterpret_cast<uint4 *>(stg + lane * 32 + 16) = cw1;
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                epi_sync();
-                if (store_leader) {
-                    // rows beyond M and columns beyond d/2 are clipped by the tensor map
-                    tma_store_2d(&codes_map, g * kNC * 16, int32_t(rt * kRows), ocodes);
+                __syncwarp();
+                if (lane == 0 && row0 < M) {
+                    tma_store_2d(&codes_map, j0 * 16, int32_t(row0), stg);
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
-                if (jj == 0 && row < M) {
-                    // this row's kNC = 2 scale bytes, one 2-byte store where the row layout allows it
-                    const int nj = nb - g * kNC < kNC ? nb - g * kNC : kNC;
-                    uint8_t *dst = scales + row * nb + int64_t(g) * kNC;
-                    const uint8_t *src = oscales + rloc * kNC;
-                    if (nj == kNC && (reinterpret_cast<uintptr_t>(dst) & 1) == 0) {
-                        *reinterpret_cast<uint16_t *>(dst) = *reinterpret_cast<const uint16_t *>(src);
+                // the row's two scale bytes, one 2-byte store where the layout allows it
+                if (row < M) {
+                    uint8_t *dst = scales + row * nb + j0;
+                    if (j0 + 1 < nb && (reinterpret_cast<uintptr_t>(dst) & 1) == 0) {
+                        *reinterpret_cast<uint16_t *>(dst) = uint16_t(sb0 | (sb1 << 8));
                     } else {
-                        for (int e = 0; e < nj; ++e) dst[e] = src[e];
+                        dst[0] = uint8_t(sb0);
+                        if (j0 + 1 < nb) dst[1] = uint8_t(sb1);
                     }
                 }
             }
         }
         if constexpr (OUT == KqOut::kCodes) {
-            if (store_leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        }
+    } else {
+        // ---------------- B builders: warp bw builds parts 2 bw and 2 bw + 1 of
+        // each column group's B set, one set ahead of the MMAs where the
+        // second buffer is free
+        const int bw = warp - 2 - kEpiWarps;
+        int last_g = -1, buse = -1;
+        for (int64_t t = t_begin; t < t_end; ++t) {
+            const int g = int(t / RT);
+            if (g == last_g) continue;
+            ++buse;
+            const int bb = buse & 1;
+            // every lane waits (each acquires the release of the old B set);
+            // the give-up decision is made warp-uniform
+            const bool freed = buse < 2 || mbar_wait(&bempty[bb], ((buse >> 1) - 1) & 1, budget);
+            if (!__all_sync(0xffffffffu, freed)) {
+                if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
+                break;
+            }
+            build_b_part(sB + bb * kBSetBytes, factors, shared, g, nb, lane, 2 * bw);
+            build_b_part(sB + bb * kBSetBytes, factors, shared, g, nb, lane, 2 * bw + 1);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bfull[bb]);
+            last_g = g;
         }
     }
 

@@ -1849,8 +1849,8 @@ int encode_act_map_rows(const void *act, int64_t M, int64_t d, CUtensorMap *map)
     return KQ_OK;
 }
 
-// The codes as the [M][d/2] uint8 matrix, boxes of {kNC*16 bytes x 128 rows}
-// (one tile of the tcgen05 variant), no swizzle.
+// The codes as the [M][d/2] uint8 matrix, boxes of {kNC*16 bytes x 32 rows}
+// (one epilogue warp's rows of a tile of the tcgen05 variant), no swizzle.
 int encode_codes_map(void *codes, int64_t M, int64_t d, CUtensorMap *map)
 {
     EncodeTiledFn enc;
@@ -1858,7 +1858,7 @@ int encode_codes_map(void *codes, int64_t M, int64_t d, CUtensorMap *map)
     if (rc != KQ_OK) return rc;
     const cuuint64_t dims[2] = {cuuint64_t(d / 2), cuuint64_t(M)};
     const cuuint64_t strides[1] = {cuuint64_t(d / 2)};
-    const cuuint32_t box[2] = {cuuint32_t(mma::kNC * 16), cuuint32_t(mma::kRows)};
+    const cuuint32_t box[2] = {cuuint32_t(mma::kNC * 16), cuuint32_t(mma::kStoreRows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
