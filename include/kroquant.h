@@ -256,13 +256,16 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
  *      register prefetch,
  *   3  the arithmetic of 2 on input staged through shared memory by TMA,
  *   4  the block transform on the tcgen05 tensor cores: Y_j = X_j K_j^T with
- *      K_j expanded in fp32 and split into three bf16 parts (each product
- *      exact in the fp32 accumulator), TMA-fed, accumulators in tensor memory,
+ *      K_j expanded in fp32 and split into three bf16 parts stacked along N
+ *      (one MMA per block and k-step; bf16 x bf16 products are exact), the
+ *      three fp32 partial results summed by the epilogue; TMA-fed,
+ *      accumulators in tensor memory,
  *   5  the arithmetic of 2 with the diagonal part of the factors in shared
  *      memory (fewer registers, more resident warps, no prefetch),
  *   6  the arithmetic of 2 with a two-deep register prefetch,
- *   7  the arithmetic of 2 with the input prefetched by cp.async into a
- *      per-thread shared-memory ring, 3 blocks in flight per thread,
+ *   7  the arithmetic of 2 with the input prefetched by cp.async (coalesced
+ *      512-byte copies per warp) into a per-warp shared-memory ring, 3 blocks
+ *      in flight per thread,
  *   8  as 7 with 5 blocks in flight.
  * Other values return KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
