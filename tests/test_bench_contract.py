@@ -28,3 +28,14 @@ def test_hash_follows_the_kernel_not_unrelated_code():
     # an edit in an unrelated kernel later in the file does not
     other = src.replace("norm_kq_rows_kernel(", "norm_kq_rows_kernel /* edit */ (", 1)
     assert other != src and bench.kernel_source_text(other) == base
+
+
+def test_every_mode_is_offered_on_the_command_line():
+    import subprocess
+    import sys
+
+    out = subprocess.run([sys.executable, bench.__file__, "--help"], capture_output=True, text=True, check=True).stdout
+    for mode in ("step", "kernel", "sweep", "sqnr", "gemm", "compare"):
+        assert mode in out
+    for flag in ("--shapes", "--reps", "--kernels", "--launches"):
+        assert flag in out
