@@ -17,7 +17,7 @@ def data():
 
 def test_identical_outputs_pass():
     c, s, y, ab = data()
-    r = pc.check_kq(c, s, c, s, y, ab)
+    r = pc.check_kq(c, s, c, s, y, ab, pool=False)
     assert r["ok"] and r["code_mismatch"] == 0
 
 
@@ -29,7 +29,7 @@ def test_planted_code_flip_fails():
     far = np.abs(v[:, :, None] - pc.BOUNDARIES[None, None, :]).min(axis=2) > 0.1
     r_, i_ = np.argwhere(far)[0]
     bad[r_, i_ // 2] ^= (1 << (4 * (i_ % 2)))
-    r = pc.check_kq(bad, s, c, s, y, ab)
+    r = pc.check_kq(bad, s, c, s, y, ab, pool=False)
     assert not r["ok"] and r["code_mismatch_nonexempt"] == 1
 
 
@@ -37,8 +37,8 @@ def test_planted_scale_change_fails():
     c, s, y, ab = data()
     bad = s.copy()
     bad[3, 1] += 1
-    r = pc.check_kq(c, bad, c, s, y, ab)
-    assert not r["ok"] and r["scale_mismatch_unflagged"] == 1
+    r = pc.check_kq(c, bad, c, s, y, ab, pool=False)
+    assert not r["ok"] and r["scale_mismatch_unflagged"] == 1 and r["scale_mismatch"] == 1
 
 
 def test_near_boundary_flip_is_exempt():
@@ -52,8 +52,10 @@ def test_near_boundary_flip_is_exempt():
     y, ab = oracle.kq_transform(xb, F, want_absbound=True)
     other = c.copy()
     other[0, 0] = (other[0, 0] & 0x0F) | (5 << 4)
-    r = pc.check_kq(other, s, c, s, y, ab)
+    r = pc.check_kq(other, s, c, s, y, ab, pool=False)
     assert r["ok"] and r["code_mismatch_exempt"] == 1
+    # exactly on the boundary: inside the boundary-relative window too
+    assert r["code_mismatch_exempt_outside_rel"] == 0
 
 
 def test_exact_checker():
@@ -70,3 +72,59 @@ def test_transform_check():
     y2 = y.copy()
     y2[1, 5] += np.float32(3e-5) * np.float32(ab[1, 5])
     assert pc.check_transform(y2, y, ab)["bad"] == 1
+
+
+def test_flagged_scale_mismatch_counts_against_the_pooled_rate():
+    # amax exactly 4 = 2^2: the block is flagged (a tolerance-sized error could
+    # take either exponent); its mismatch passes the case but enters the pool
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0] = 4.0
+    xb = synth.bf16_bits_from_f32(x)
+    F = np.tile(np.eye(2, dtype=np.float32), (1, 5, 1, 1))
+    c, s = oracle.kq_quantize(xb, F)
+    y, ab = oracle.kq_transform(xb, F, want_absbound=True)
+    bad = s.copy()
+    bad[0, 0] -= 1
+    r = pc.check_kq(c, bad, c, s, y, ab, pool=False)
+    # allowed per case, counted against the pooled rate
+    assert r["flagged_blocks"] == 1 and r["scale_mismatch_flagged"] == 1 and r["ok"]
+    assert not pc.pooled_verdict({"cases": 1, "codes": 32, "blocks": 1, "code_mismatch_exempt": 0,
+                                  "code_mismatch_exempt_outside_rel": 0, "flagged_blocks": 1,
+                                  "scale_mismatch_flagged": 1})["ok"]
+
+
+def test_sign_of_zero_flip_is_exempt_but_outside_the_relative_window():
+    # y_1 = x_0 - x_1 cancels exactly under the factor [[1, 1], [1, -1]] on
+    # the lowest index bit: the oracle codes +0; a -0 (0x8) is within the
+    # |K||x| window of the zero boundary but not within 1e-5 of a boundary b > 0
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0] = 3.0
+    x[0, 1] = 3.0
+    xb = synth.bf16_bits_from_f32(x)
+    F = np.tile(np.eye(2, dtype=np.float32), (1, 5, 1, 1))
+    F[0, 4] = np.array([[1.0, 1.0], [1.0, -1.0]], np.float32)
+    c, s = oracle.kq_quantize(xb, F)
+    y, ab = oracle.kq_transform(xb, F, want_absbound=True)
+    assert y[0, 1] == 0.0 and (c[0, 0] >> 4) == 0
+    other = c.copy()
+    other[0, 0] |= 0x80
+    r = pc.check_kq(other, s, c, s, y, ab, pool=False)
+    assert r["ok"] and r["code_mismatch_exempt"] == 1 and r["code_mismatch_exempt_outside_rel"] == 1
+
+
+def test_pooled_rate():
+    # one exempt mismatch per 1e6 codes passes, more fails; the rate is over
+    # every code of every pooled case
+    ok = pc.pooled_verdict({"cases": 2, "codes": 2_000_000, "blocks": 62_500, "code_mismatch_exempt": 2,
+                            "code_mismatch_exempt_outside_rel": 0, "flagged_blocks": 0})
+    assert ok["ok"] and ok["exempt_rate"] == 1e-6
+    bad = pc.pooled_verdict({"cases": 2, "codes": 2_000_000, "blocks": 62_500, "code_mismatch_exempt": 3,
+                             "code_mismatch_exempt_outside_rel": 0, "flagged_blocks": 0})
+    assert not bad["ok"]
+
+
+def test_unpooled_checks_leave_the_pool_alone():
+    before = dict(pc.POOL)
+    c, s, y, ab = data()
+    pc.check_kq(c, s, c, s, y, ab, pool=False)
+    assert pc.POOL == before
