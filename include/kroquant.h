@@ -260,14 +260,15 @@ int kq_transform_f32(const void *act_bf16, const float *factors, int shared,
  *      (one MMA per block and k-step; bf16 x bf16 products are exact), the
  *      three fp32 partial results summed by the epilogue; TMA-fed,
  *      accumulators in tensor memory,
- *   5  the arithmetic of 2 with the diagonal part of the factors in shared
- *      memory (fewer registers, more resident warps, no prefetch),
- *   6  the arithmetic of 2 with a two-deep register prefetch,
- *   7  the arithmetic of 2 with the input prefetched by cp.async (coalesced
- *      512-byte copies per warp) into a per-warp shared-memory ring, 3 blocks
- *      in flight per thread,
- *   8  as 7 with 5 blocks in flight.
- * Other values return KQ_ERR_VARIANT. */
+ *   9  the operations of 2 on two rows of a column at once (every stage a
+ *      packed f32x2 FMA), input staged through shared memory by TMA, one
+ *      CTA per SM; shapes whose block-column count does not fit its grid
+ *      rule (and the fp32 export) run 2.
+ * Variants 2, 3 and 9 give identical results.  Every variant emits a block
+ * whose transformed values are not finite as the scale byte 0xFF with zero
+ * codes; a unit-diagonal block that overflows only in its intermediates is
+ * recomputed in the direct form.  Other values (5-8 were retired) return
+ * KQ_ERR_VARIANT. */
 int kq_quantize_variant(int variant, const void *act_bf16, const float *factors,
                         int shared, uint8_t *out_codes, uint8_t *out_scales,
                         int64_t M, int64_t d, cudaStream_t stream);
@@ -291,9 +292,14 @@ int mx_quantize_variant(int variant, const void *act_bf16,
  * about a second of clock cycles, adds 1 to a device counter per giving-up
  * thread, drains its copies in flight and returns, so the context stays
  * usable.  kq_wait_timeouts copies the counter to *count (synchronising the
- * device) and zeroes it if reset != 0.  kq_selftest_bounded_wait launches one
- * staged CTA whose producer issues no copies, so its waits run out after about
- * a millisecond; it reads and writes no memory other than the counter. */
+ * device) and zeroes it if reset != 0.  The counter is one device-global int
+ * of the library, shared by every call on that device: calls that overlap on
+ * the GPU (several streams or threads) add to the same count, and a reset
+ * clears theirs too.  kq_selftest_bounded_wait launches one staged CTA whose
+ * producer issues no copies, so its waits run out after about a millisecond;
+ * its operand is a fixed 80 KB device array of the library (1280 blocks of
+ * 64 bytes, shared by all its calls), and it reads and writes no memory other
+ * than that array and the counter (in fact only the counter). */
 int kq_wait_timeouts(int *count, int reset);
 int kq_selftest_bounded_wait(cudaStream_t stream);
 

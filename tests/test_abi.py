@@ -124,7 +124,9 @@ def test_alignment_errors(L):
 
 
 def test_variant_errors_before_cuda(L):
-    assert L.kq_quantize_variant(9, P(16), P(16), 0, P(16), P(16), 4, 64, None) == -5
+    assert L.kq_quantize_variant(10, P(16), P(16), 0, P(16), P(16), 4, 64, None) == -5
+    for retired in (5, 6, 7, 8):
+        assert L.kq_quantize_variant(retired, P(16), P(16), 0, P(16), P(16), 4, 64, None) == -5
     assert L.sq_quantize_variant(5, P(16), P(16), P(16), P(16), 4, 64, None) == -5
     assert L.mx_quantize_variant(-1, P(16), P(16), P(16), 4, 64, None) == -5
     assert "variant" in err(L)

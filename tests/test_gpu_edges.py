@@ -171,7 +171,7 @@ def test_variants_agree_with_oracle(cuda_device):
     cr, sr = oracle.kq_quantize(x, F)
     yr, ab = oracle.kq_transform(x, F, want_absbound=True)
     tried = 0
-    for v in range(8):
+    for v in range(10):
         try:
             c, s = kq.kq_quantize_variant(v, xd, Fd)
         except kq.KroQuantError as e:
@@ -183,7 +183,11 @@ def test_variants_agree_with_oracle(cuda_device):
     assert tried >= 1
 
 
-VARIANT_SHAPES = [(1, 32), (37, 64), (129, 5600), (257, 2240), (1000, 1152), (300, 12288)]
+# ragged final stage, odd block counts, a single block; 4099 x 1152 gives the
+# two-block ring kernel an odd number of chunks per CTA, 129 x 5600 (175
+# block columns) a shape its grid rule hands to variant 2
+VARIANT_SHAPES = [(1, 32), (37, 64), (129, 5600), (257, 2240), (1000, 1152), (300, 12288), (4099, 1152)]
+RING = (9,)
 
 
 @pytest.mark.parametrize("M,d", VARIANT_SHAPES, ids=[f"{M}x{d}" for M, d in VARIANT_SHAPES])
@@ -203,24 +207,24 @@ def test_baseline_variants_bit_exact(cuda_device, M, d):
 
 @pytest.mark.parametrize("M,d", VARIANT_SHAPES, ids=[f"{M}x{d}" for M, d in VARIANT_SHAPES])
 def test_kq_variants_sharing_arithmetic_are_identical(cuda_device, M, d):
-    """Variants 2, 3, 5, 6, 7 and 8 share the arithmetic, so their outputs are identical."""
+    """Variants 2, 3 and 9 share the arithmetic, so their outputs are identical."""
     x = synth.activation("pixart", M, d, seed=M * 3 + d)
     F = synth.factors(d // 32, seed=d + 1)
     xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
     c2, s2 = kq.kq_quantize_variant(2, xd, Fd)
-    for v in (3, 5, 6, 7, 8):
+    for v in (3,) + RING:
         cv, sv = kq.kq_quantize_variant(v, xd, Fd)
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
     F1 = synth.factors(1, seed=d, shared=True)
     c2, s2 = kq.kq_quantize_variant(2, xd, dev_f32(F1, cuda_device), shared=True)
-    for v in (3, 5, 6, 7, 8):
+    for v in (3,) + RING:
         cv, sv = kq.kq_quantize_variant(v, xd, dev_f32(F1, cuda_device), shared=True)
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
     # a column that falls back to the direct form (swap factor) alongside split ones
     F2 = F.copy()
     F2[0, 2] = np.array([[0, 1], [1, 0]], np.float32)
     c2, s2 = kq.kq_quantize_variant(2, xd, dev_f32(F2, cuda_device))
-    for v in (3, 5, 6, 7, 8):
+    for v in (3,) + RING:
         cv, sv = kq.kq_quantize_variant(v, xd, dev_f32(F2, cuda_device))
         assert bool((c2 == cv).all()) and bool((s2 == sv).all()), v
 
@@ -236,8 +240,17 @@ def test_bounded_wait_gives_up_and_context_stays_usable(cuda_device):
     assert kq.kq_wait_timeouts(reset=True) > 0
     M, d = 64, 128
     x = synth.activation("tiny", M, d, 0)
-    c, s = kq.mx_quantize(dev_bf16(x, cuda_device))
+    xd = dev_bf16(x, cuda_device)
+    c, s = kq.mx_quantize(xd)
     assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *oracle.mx_quantize(x))["ok"]
+    # the staged kernels themselves (shared-memory opt-in, barrier set-up and
+    # TMA ring of the kernel whose waits just ran out) still work
+    c, s = kq.mx_quantize_variant(2, xd)
+    assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *oracle.mx_quantize(x))["ok"]
+    m = synth.sq_multipliers(x)
+    c, s = kq.sq_quantize(xd, dev_f32(m, cuda_device))            # default: the staged kernel
+    assert pc.check_exact(c.cpu().numpy(), s.cpu().numpy(), *oracle.sq_quantize(x, m))["ok"]
+    torch.cuda.synchronize()
     assert kq.kq_wait_timeouts() == 0
 
 
@@ -304,3 +317,60 @@ def test_extreme_magnitudes(cuda_device):
     cm, sm = oracle.mx_quantize(x)
     np.testing.assert_array_equal(s.cpu().numpy(), sm)
     np.testing.assert_array_equal(c.cpu().numpy(), cm)
+
+
+KQ_VARIANTS = (0, 1, 2, 3, 4) + RING
+
+
+def test_unit_split_limits_near_the_top_of_the_range(cuda_device):
+    """Factors at the limits of the unit-diagonal split (|b| = |c| = 16,
+    diagonals 1/16) on inputs near 2^115: the split's intermediates U x grow
+    by up to 17^5 and overflow fp32 there, while the transform itself (row
+    sums of |K| = 1.0625^5) stays finite, so every variant must still match
+    the oracle.  Column 1 has a factor beyond the split (|b| = 20) and runs
+    the direct form."""
+    M, d = 300, 128
+    G = np.array([[1 / 16, 1.0], [1.0, 1 / 16]], np.float32)
+    F = np.tile(G, (d // 32, 5, 1, 1))
+    F[1, 2] = np.array([[1 / 20, 1.0], [1.0, 1 / 16]], np.float32)
+    rng = np.random.default_rng(11)
+    x = bf16(rng.standard_normal((M, d)).astype(np.float32) * np.float32(2.0 ** 115))
+    cr, sr = oracle.kq_quantize(x, F)
+    yr, ab = oracle.kq_transform(x, F, want_absbound=True)
+    assert np.isfinite(yr).all() and int(sr.max()) < 0xFF
+    xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
+    for v in KQ_VARIANTS:
+        c, s = kq.kq_quantize_variant(v, xd, Fd)
+        res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), cr, sr, yr, ab)
+        assert res["ok"], (v, res)
+    # the fp32 transform export and the LU form take the same path
+    y = kq.kq_transform_f32(xd, Fd).cpu().numpy()
+    assert pc.check_transform(y, yr, ab)["bad"] == 0
+    assert kq.kq_wait_timeouts() == 0
+
+
+def test_transform_overflow_gives_the_nan_scale(cuda_device):
+    """Where the transform of a finite block exceeds fp32 (here the unnormalised
+    Hadamard factor [[1, 1], [1, -1]], row sums 2^5, on inputs near 2^126), the
+    oracle writes the E8M0 NaN byte 0xFF and zero codes; so does every variant.
+    Other blocks are unaffected."""
+    M, d = 96, 256
+    H = np.array([[1.0, 1.0], [1.0, -1.0]], np.float32)
+    F = np.tile(H, (d // 32, 5, 1, 1))
+    rng = np.random.default_rng(12)
+    vals = rng.standard_normal((M, d)).astype(np.float32)
+    vals[::3] *= np.float32(2.0 ** 126)          # every third row overflows
+    x = bf16(vals)
+    cr, sr = oracle.kq_quantize(x, F)
+    assert (sr[::3] == 0xFF).all() and (cr[::3] == 0).all() and (sr[1::3] < 0xFF).all()
+    xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
+    for v in KQ_VARIANTS:
+        c, s = kq.kq_quantize_variant(v, xd, Fd)
+        c, s = c.cpu().numpy(), s.cpu().numpy()
+        np.testing.assert_array_equal(s[::3], sr[::3], err_msg=f"variant {v}")
+        np.testing.assert_array_equal(c[::3], cr[::3], err_msg=f"variant {v}")
+        keep = np.ones(M, bool)
+        keep[::3] = False
+        yr, ab = oracle.kq_transform(x[keep], F, want_absbound=True)
+        res = pc.check_kq(c[keep], s[keep], cr[keep], sr[keep], yr, ab)
+        assert res["ok"], (v, res)

@@ -9,7 +9,7 @@ from w4a4_mxfp4_post_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-MMA = 4
+MMAS = (4,)
 
 
 def dev_bf16(bits, device):
@@ -29,8 +29,9 @@ SHAPES = [(1, 32), (128, 128), (3, 96), (130, 160), (37, 64), (129, 5600), (257,
           (300, 12288), (8192, 4608)]
 
 
+@pytest.mark.parametrize("MMA", MMAS)
 @pytest.mark.parametrize("M,d", SHAPES, ids=[f"{M}x{d}" for M, d in SHAPES])
-def test_mma_variant_matches_oracle(cuda_device, M, d):
+def test_mma_variant_matches_oracle(cuda_device, M, d, MMA):
     x = synth.activation("pixart", M, d, seed=M * 5 + d)
     F = synth.factors(d // 32, seed=d + 2)
     xd, Fd = dev_bf16(x, cuda_device), dev_f32(F, cuda_device)
@@ -46,7 +47,8 @@ def test_mma_variant_matches_oracle(cuda_device, M, d):
     assert res["ok"], res
 
 
-def test_mma_variant_shared_factors(cuda_device):
+@pytest.mark.parametrize("MMA", MMAS)
+def test_mma_variant_shared_factors(cuda_device, MMA):
     M, d = 300, 2240
     x = synth.activation("sana", M, d, 2)
     F1 = synth.factors(1, 2, shared=True)
@@ -58,7 +60,8 @@ def test_mma_variant_shared_factors(cuda_device):
     assert res["ok"], res
 
 
-def test_mma_variant_hand_worked_blocks(cuda_device):
+@pytest.mark.parametrize("MMA", MMAS)
+def test_mma_variant_hand_worked_blocks(cuda_device, MMA):
     import os
 
     from conftest import GOLDEN, parse_blocks

@@ -216,12 +216,16 @@ __device__ __forceinline__ void load_block_sum(uint32_t tcol, float (&y)[32])
 }
 
 // MXFP4 of one block's 32 transformed values (amax, E8M0 byte, exact 2^-e
-// scaling by a packed FFMA with +0, E2M1).
+// scaling by a packed FFMA with +0, E2M1); a block that is not finite gets
+// the E8M0 NaN byte 0xFF and zero codes.
 __device__ __forceinline__ void quantize_block32(float (&v)[32], uint4 &cw, uint32_t &sb)
 {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = max3_abs(amax, v[2 * i], v[2 * i + 1]);
+    const float amax = amax32<true>([&](int i) { return v[i]; });
+    if (!(amax <= 3.40282347e38f)) {
+        cw = make_uint4(0u, 0u, 0u, 0u);
+        sb = 0xFFu;
+        return;
+    }
     sb = e8m0_byte(amax);
     const float sc = inv_scale(sb);
 #pragma unroll

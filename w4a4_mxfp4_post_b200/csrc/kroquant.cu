@@ -135,13 +135,57 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
     return r;
 }
 
+// max(|a|, |b|, |c|) in one instruction (three-input max, sm_100).
+__device__ __forceinline__ float max3_abs(float a, float b, float c)
+{
+    float r;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// max(|a|, |b|, |c|), NaN if any input is NaN (three-input max, sm_100).
+__device__ __forceinline__ float max3_abs_nan(float a, float b, float c)
+{
+    float r;
+    asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <bool NAN_>
+__device__ __forceinline__ float max3_mag(float a, float b, float c)
+{
+    return NAN_ ? max3_abs_nan(a, b, c) : max3_abs(a, b, c);
+}
+
+// max |v(i)| over i < 32 as a tree of three-input maxes (depth 4), not a
+// chain of 16 dependent ones: the block amax is on every quantizer's
+// critical path, and inline-asm maxes are never reassociated by the
+// compiler.  NAN_ selects the NaN-propagating form.
+template <bool NAN_, class V>
+__device__ __forceinline__ float amax32(V v)
+{
+    float m[11];
+#pragma unroll
+    for (int k = 0; k < 10; ++k) m[k] = max3_mag<NAN_>(v(3 * k), v(3 * k + 1), v(3 * k + 2));
+    m[10] = max3_mag<NAN_>(v(30), v(31), 0.0f);
+    const float n0 = max3_mag<NAN_>(m[0], m[1], m[2]);
+    const float n1 = max3_mag<NAN_>(m[3], m[4], m[5]);
+    const float n2 = max3_mag<NAN_>(m[6], m[7], m[8]);
+    const float n3 = max3_mag<NAN_>(m[9], m[10], 0.0f);
+    return max3_mag<NAN_>(max3_mag<NAN_>(n0, n1, n2), n3, 0.0f);
+}
+
 // The MXFP4 block quantizer on 32 fp32 values: amax, E8M0 byte, scaling by
-// the exact power of two 2^-e, E2M1 rounding, packing.
+// the exact power of two 2^-e, E2M1 rounding, packing.  A block with a value
+// that is not finite gets the E8M0 NaN byte 0xFF and zero codes.
 __device__ __forceinline__ void mx_quantize_block(const float (&v)[32], uint4 &codes, uint32_t &sbyte)
 {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kBlk; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float amax = amax32<true>([&](int i) { return v[i]; });
+    if (!(amax <= 3.40282347e38f)) {
+        codes = make_uint4(0u, 0u, 0u, 0u);
+        sbyte = 0xFFu;
+        return;
+    }
     const uint32_t sb = e8m0_byte(amax);
     const float s = inv_scale(sb);
     uint32_t w[4];
@@ -275,22 +319,11 @@ __device__ __forceinline__ void unpack_pairs(const uint4 (&raw)[4], float2 (&p)[
     }
 }
 
-// max(|a|, |b|, |c|) in one instruction (three-input max, sm_100).
-__device__ __forceinline__ float max3_abs(float a, float b, float c)
+// The rest of the MXFP4 block quantizer on the pair layout once the amax is
+// known: E8M0 byte from its exponent field, exact scaling by 2^-e, E2M1
+// round-to-nearest-even with saturation, packing.
+__device__ __forceinline__ void mx_finish_pairs(float2 (&p)[16], float amax, uint4 &codes, uint32_t &sbyte)
 {
-    float r;
-    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// MXFP4 block quantizer on the pair layout (same arithmetic as
-// mx_quantize_block: amax, E8M0 byte from its exponent field, exact scaling
-// by 2^-e, E2M1 round-to-nearest-even with saturation, packing).
-__device__ __forceinline__ void mx_quantize_pairs(float2 (&p)[16], uint4 &codes, uint32_t &sbyte)
-{
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = max3_abs(amax, p[i].x, p[i].y);
     const uint32_t sb = e8m0_byte(amax);
     const float s = inv_scale(sb);
     const float2 ss = make_float2(s, s);
@@ -301,6 +334,21 @@ __device__ __forceinline__ void mx_quantize_pairs(float2 (&p)[16], uint4 &codes,
     codes.z = cvt_e2m1x8(p[0].y, p[1].y, p[2].y, p[3].y, p[4].y, p[5].y, p[6].y, p[7].y);
     codes.w = cvt_e2m1x8(p[8].y, p[9].y, p[10].y, p[11].y, p[12].y, p[13].y, p[14].y, p[15].y);
     sbyte = sb;
+}
+
+// MXFP4 block quantizer on the pair layout (same arithmetic as
+// mx_quantize_block: amax, E8M0 byte from its exponent field, exact scaling
+// by 2^-e, E2M1 round-to-nearest-even with saturation, packing).
+__device__ __forceinline__ void mx_quantize_pairs(float2 (&p)[16], uint4 &codes, uint32_t &sbyte)
+{
+    const float amax = amax32<false>([&](int i) { return (i & 1) ? p[i >> 1].y : p[i >> 1].x; });
+    mx_finish_pairs(p, amax, codes, sbyte);
+}
+
+// Block amax on the pair layout, NaN if any value is NaN.
+__device__ __forceinline__ float pair_amax_nan(const float2 (&p)[16])
+{
+    return amax32<true>([&](int i) { return (i & 1) ? p[i >> 1].y : p[i >> 1].x; });
 }
 
 // Stage on in-block index bit b < 4 (pair-index distance S = 2^b) in unit-
@@ -427,14 +475,22 @@ __device__ __forceinline__ void kq_direct_apply(float2 (&p)[16], const float4 (&
     }
 }
 
+// Output of one transformed block: its MXFP4 codes and scale from the block
+// amax (NaN-propagating; a non-finite block gets 0xFF and zero codes), or the
+// fp32 values themselves.
 template <KqOut OUT>
-__device__ __forceinline__ void kq_emit(float2 (&p)[16], int64_t gi, uint4 *__restrict__ codes,
+__device__ __forceinline__ void kq_emit(float2 (&p)[16], float amax, int64_t gi, uint4 *__restrict__ codes,
                                         uint8_t *__restrict__ scales, float4 *__restrict__ y_out)
 {
     if constexpr (OUT == KqOut::kCodes) {
         uint4 c;
         uint32_t sb;
-        mx_quantize_pairs(p, c, sb);
+        if (amax <= 3.40282347e38f) {
+            mx_finish_pairs(p, amax, c, sb);
+        } else {
+            c = make_uint4(0u, 0u, 0u, 0u);
+            sb = 0xFFu;
+        }
         codes[gi] = c;
         scales[gi] = uint8_t(sb);
     } else {
@@ -481,12 +537,17 @@ __device__ __forceinline__ int64_t sf_offset(const SfPos &s)
 }
 
 // Codes as kq_emit; the scale byte at its scale-factor-layout offset.
-__device__ __forceinline__ void kq_emit_sf(float2 (&p)[16], int64_t gi, uint4 *__restrict__ codes,
+__device__ __forceinline__ void kq_emit_sf(float2 (&p)[16], float amax, int64_t gi, uint4 *__restrict__ codes,
                                            uint8_t *__restrict__ sf, SfPos &sp)
 {
     uint4 c;
     uint32_t sb;
-    mx_quantize_pairs(p, c, sb);
+    if (amax <= 3.40282347e38f) {
+        mx_finish_pairs(p, amax, c, sb);
+    } else {
+        c = make_uint4(0u, 0u, 0u, 0u);
+        sb = 0xFFu;
+    }
     codes[gi] = c;
     const int64_t off = sf_offset(sp);
     sf[off] = uint8_t(sb);
@@ -515,6 +576,51 @@ __device__ __forceinline__ void load_lu(const float *__restrict__ lu, int shared
     }
 }
 
+// The unit-diagonal form's intermediates (U x) can exceed the block's final
+// values by up to 17^5 (|b|, |c| <= 16 per stage), so a finite block can
+// overflow there while the direct form and the oracle stay finite.  The
+// unit-diagonal loops only note that a block's amax came out non-finite
+// (the NaN-propagating amax) and emit it as a non-finite block; after its
+// loop, a thread that noted one walks its blocks start, start + stride, ...
+// again and rewrites every block whose unit-diagonal amax is not finite with
+// the direct form's result (0xFF and zero codes where that is not finite
+// either).  Only inputs within 2^21 of the top of the fp32 range get here,
+// and the loops keep no registers for it.
+template <KqOut OUT, bool LU, bool SF>
+__device__ __noinline__ void kq_redo_overflow(const uint4 *__restrict__ act, const float *__restrict__ params,
+                                              int shared, int64_t start, int64_t stride, int64_t nblocks, int nb,
+                                              uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
+                                              float4 *__restrict__ y_out)
+{
+    const int j = int(start % nb);
+    float4 g[5];
+    if constexpr (LU)
+        load_lu(params, shared, j, g);
+    else
+        load_factors(reinterpret_cast<const float4 *>(params), shared, j, g);
+    KqFast st;
+    kq_fast_setup(g, st);
+    SfPos sp{};
+    if constexpr (SF) sp = sf_pos(start, stride, nb);
+    for (int64_t gi = start; gi < nblocks; gi += stride) {
+        uint4 raw[4];
+        load_block_nc(act, gi, raw);
+        float2 p[16];
+        unpack_pairs(raw, p);
+        kq_fast_apply(p, st);
+        if (pair_amax_nan(p) <= 3.40282347e38f) {
+            if constexpr (SF) sp.row += sp.rstep;
+            continue;
+        }
+        unpack_pairs(raw, p);
+        kq_direct_apply(p, g);
+        if constexpr (SF)
+            kq_emit_sf(p, pair_amax_nan(p), gi, codes, scales, sp);
+        else
+            kq_emit<OUT>(p, pair_amax_nan(p), gi, codes, scales, y_out);
+    }
+}
+
 // KroQuant quantizer, packed butterfly (variant 2).
 //
 // Each 2x2 factor is split as G = [[g00, g01], [g10, g11]]
@@ -540,17 +646,20 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
     if (t >= T || t >= nblocks) return;
     SfPos sp{};
     if constexpr (SF) sp = sf_pos(t, T, nb);
-    float4 g[5];
-    if constexpr (LU)
-        load_lu(params, shared, int(t % nb), g);
-    else
-        load_factors(reinterpret_cast<const float4 *>(params), shared, int(t % nb), g);
-    KqFast st;
-    const bool fast = kq_fast_setup(g, st);
-
+    // the first block's load goes out before the column set-up, so the two
+    // latencies (activation from HBM, factors from L2) overlap
     int64_t gi = t;
     uint4 raw[4];
     load_block_nc(act, gi, raw);
+    const int j = int(t % nb);
+    float4 g[5];
+    if constexpr (LU)
+        load_lu(params, shared, j, g);
+    else
+        load_factors(reinterpret_cast<const float4 *>(params), shared, j, g);
+    KqFast st;
+    const bool fast = kq_fast_setup(g, st);
+    bool overflow = false;
     if (fast) {
         for (;;) {
             const int64_t gn = gi + T;
@@ -559,10 +668,12 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
             float2 p[16];
             unpack_pairs(raw, p);
             kq_fast_apply(p, st);
+            const float amax = pair_amax_nan(p);
+            overflow |= !(amax <= 3.40282347e38f);
             if constexpr (SF)
-                kq_emit_sf(p, gi, codes, scales, sp);
+                kq_emit_sf(p, amax, gi, codes, scales, sp);
             else
-                kq_emit<OUT>(p, gi, codes, scales, y_out);
+                kq_emit<OUT>(p, amax, gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
@@ -577,15 +688,16 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
             unpack_pairs(raw, p);
             kq_direct_apply(p, g);
             if constexpr (SF)
-                kq_emit_sf(p, gi, codes, scales, sp);
+                kq_emit_sf(p, pair_amax_nan(p), gi, codes, scales, sp);
             else
-                kq_emit<OUT>(p, gi, codes, scales, y_out);
+                kq_emit<OUT>(p, pair_amax_nan(p), gi, codes, scales, y_out);
             if (gn >= nblocks) break;
 #pragma unroll
             for (int q = 0; q < 4; ++q) raw[q] = nxt[q];
             gi = gn;
         }
     }
+    if (overflow) kq_redo_overflow<OUT, LU, SF>(act, params, shared, t, T, nblocks, nb, codes, scales, y_out);
 }
 
 // Fixed-Hadamard baseline (the transform the pages compare the on-the-fly
@@ -652,198 +764,6 @@ fwht_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *_
             scales[gi] = uint8_t(sb);
         }
     }
-}
-
-// KroQuant quantizer, lean (variant 5): the arithmetic of variant 2 with the
-// column coefficients (the 32 values of D and the 10 off-diagonal
-// coefficients) kept in shared memory instead of registers, and no register
-// prefetch.  A thread's coefficients sit in its own 176-byte slot (11 x 16 B:
-// an odd number of 16-byte units, so the 8 lanes of a 16-byte shared-load
-// phase hit 8 distinct bank groups) and are re-read every block (11 shared
-// loads).  64 registers per thread instead of 108, so 4 CTAs (32 warps) per
-// SM hide the memory latency without a prefetch.
-constexpr int kLeanSlotFloats = 44;   // 32 D values + 12 pad (176 bytes)
-
-__global__ void __launch_bounds__(kThreads, 4)
-kq_lean_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
-               uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
-{
-    __shared__ __align__(16) float dslot[kThreads * kLeanSlotFloats];
-    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    const bool active = t < T && t < nblocks;
-    const int j = active ? int(t % nb) : 0;
-    float *slot = dslot + threadIdx.x * kLeanSlotFloats;
-    bool fast;
-    {
-        float4 g[5];
-        load_factors(factors, shared, j, g);
-        KqFast st;
-        fast = kq_fast_setup(g, st);
-        float2 *myd = reinterpret_cast<float2 *>(slot);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) myd[i] = st.DP[i];
-        float4 *cq = reinterpret_cast<float4 *>(slot + 32);
-        cq[0] = make_float4(st.B[0], st.C[0], st.B[1], st.C[1]);
-        cq[1] = make_float4(st.B[2], st.C[2], st.B[3], st.C[3]);
-        cq[2] = make_float4(st.b4, st.c4, 0.0f, 0.0f);
-    }
-    if (!active) return;
-    const float4 *dq = reinterpret_cast<const float4 *>(slot);
-    for (int64_t gi = t; gi < nblocks; gi += T) {
-        uint4 raw[4];
-        load_block_nc(act, gi, raw);
-        float2 p[16];
-        unpack_pairs(raw, p);
-        if (fast) {
-            const float4 c01 = dq[8], c23 = dq[9], c4q = dq[10];
-            const float b4 = c4q.x, c4 = c4q.y;
-            unit_stage2<1>(p, bcast(c01.x), bcast(c01.y));
-            unit_stage2<2>(p, bcast(c01.z), bcast(c01.w));
-            unit_stage2<4>(p, bcast(c23.x), bcast(c23.y));
-            unit_stage2<8>(p, bcast(c23.z), bcast(c23.w));
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 dd = dq[q];   // (D_2q, D_2q+16, D_2q+1, D_2q+17)
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int i = 2 * q + h2;
-                    const float lo = p[i].x, hi = p[i].y;
-                    const float2 dp = h2 ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y);
-                    p[i] = __ffma2_rn(make_float2(fmaf(b4, hi, lo), fmaf(c4, lo, hi)), dp, plus_zero2());
-                }
-            }
-        } else {   // rare: the factors are reloaded (L1) rather than kept live
-            float4 g[5];
-            load_factors(factors, shared, j, g);
-            kq_direct_apply(p, g);
-        }
-        kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
-    }
-}
-
-// KroQuant quantizer, variant 6: the arithmetic of variant 2 with a two-deep
-// register prefetch (three 64-byte blocks per thread in flight), for more
-// memory-level parallelism at the same 2 CTAs per SM.
-__global__ void __launch_bounds__(kThreads, 2)
-kq_packed2_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
-                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
-{
-    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    if (t >= T || t >= nblocks) return;
-    const int j = int(t % nb);
-    KqFast st;
-    bool fast;
-    {
-        float4 g[5];
-        load_factors(factors, shared, j, g);
-        fast = kq_fast_setup(g, st);
-    }
-    int64_t gi = t;
-    uint4 r0[4], r1[4];
-    load_block_nc(act, gi, r0);
-    if (gi + T < nblocks) load_block_nc(act, gi + T, r1);
-    for (;;) {
-        const int64_t g2 = gi + 2 * T;
-        uint4 r2[4];
-        if (g2 < nblocks) load_block_nc(act, g2, r2);
-        float2 p[16];
-        unpack_pairs(r0, p);
-        if (fast) {
-            kq_fast_apply(p, st);
-        } else {   // rare: the factors are reloaded (L1) rather than kept live
-            float4 g[5];
-            load_factors(factors, shared, j, g);
-            kq_direct_apply(p, g);
-        }
-        kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
-        if (gi + T >= nblocks) break;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            r0[q] = r1[q];
-            r1[q] = r2[q];
-        }
-        gi += T;
-    }
-}
-
-// KroQuant quantizer, variants 7 and 8: the arithmetic of variant 2, with the
-// input prefetched by cp.async into a per-warp ring in shared memory (D steps,
-// D - 1 of them in flight): the copies hold no registers, so the memory-level
-// parallelism does not cost occupancy.  At every step a warp's 32 threads own
-// 32 consecutive blocks (2 KB); the warp copies them cooperatively, each
-// cp.async instruction covering 512 contiguous bytes, into its ring slot with
-// the 16-byte piece p of block b at b * 64 + 16 (p ^ ((b >> 1) & 3)), so the
-// per-thread reads of a block are free of bank conflicts.  The loop is
-// warp-uniform (a warp's first thread has the most steps); a thread without a
-// block at a step only helps copy and synchronise.
-__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *g)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
-kq_async_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
-                uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
-{
-    extern __shared__ uint4 ring[];   // [warp][D][128 pieces of 16 bytes]
-    const int lane = threadIdx.x & 31;
-    const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    const int64_t t0 = t - lane;                          // the warp's first thread
-    const bool live = t < T && t < nblocks;
-    const int j = live ? int(t % nb) : 0;
-    KqFast st;
-    bool fast = false;
-    if (live) {
-        float4 g[5];
-        load_factors(factors, shared, j, g);
-        fast = kq_fast_setup(g, st);
-    }
-    uint4 *wring = ring + size_t(threadIdx.x >> 5) * D * 128;
-    const uint32_t wbase = static_cast<uint32_t>(__cvta_generic_to_shared(wring));
-    const int64_t nsteps = (t0 < T && t0 < nblocks) ? (nblocks - t0 + T - 1) / T : 0;   // warp-uniform
-    auto issue = [&](int64_t i, int slot) {
-        const int64_t b0 = t0 + i * T;                    // the warp's first block at step i
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int c = q * 32 + lane;                  // piece c of the warp's 2 KB
-            const int b = c >> 2, pc = c & 3;
-            if (t0 + b < T && b0 + b < nblocks)
-                cp_async16(wbase + uint32_t(slot * 2048 + b * 64 + ((pc ^ ((b >> 1) & 3)) << 4)), act + (b0 + b) * 4 + pc);
-        }
-    };
-#pragma unroll
-    for (int s = 0; s < D - 1; ++s) {
-        if (s < nsteps) issue(s, s);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    }
-    int slot = 0;
-    for (int64_t i = 0; i < nsteps; ++i) {
-        // one group per step (possibly empty): step i + D - 1 into the slot read at step i - 1
-        if (i + D - 1 < nsteps) issue(i + D - 1, slot == 0 ? D - 1 : slot - 1);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group %0;" ::"n"(D - 1) : "memory");   // step i has landed (own copies)
-        __syncwarp();                                                       // ... and the other lanes'
-        const int64_t gi = t + i * T;
-        if (live && gi < nblocks) {
-            uint4 raw[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) raw[q] = wring[slot * 128 + lane * 4 + (q ^ ((lane >> 1) & 3))];
-            float2 p[16];
-            unpack_pairs(raw, p);
-            if (fast) {
-                kq_fast_apply(p, st);
-            } else {   // rare: the factors are reloaded (L1) rather than kept live
-                float4 g[5];
-                load_factors(factors, shared, j, g);
-                kq_direct_apply(p, g);
-            }
-            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
-        }
-        __syncwarp();   // every lane has read the slot before it is refilled
-        slot = slot == D - 1 ? 0 : slot + 1;
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // SmoothQuant quantizer on the pair layout: y = fp32(x * m) per channel (one
@@ -940,7 +860,14 @@ constexpr int kStagedThreads = kConsumers + 32;        // + one producer warp
 constexpr size_t kStagedSmem = size_t(kStages) * kStageBytes + 1024 + 2 * kStages * sizeof(uint64_t);
 
 __device__ int g_wait_timeouts;
-__device__ __align__(256) uint8_t g_selftest_dummy[256];
+
+// Operand of kq_selftest_bounded_wait: its tensor map covers kSelftestBlocks
+// rows of 64 bytes, and the same array stands in for the codes (16 B per
+// block) and scales (1 B per block) outputs, so it spans the whole map even
+// though that launch issues no copies and writes nothing.
+constexpr int64_t kSelftestBlocks = int64_t(kStageRows) * (kStages + 1);
+__device__ __align__(256) uint8_t g_selftest_dummy[kSelftestBlocks * 64];
+static_assert(sizeof(g_selftest_dummy) >= kSelftestBlocks * 64, "selftest map and outputs stay inside the array");
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -1085,7 +1012,8 @@ __device__ __forceinline__ bool staged_consume(const StagedRing &r, int64_t nchu
 // The grid is a multiple of nb / gcd(nb, kStageRows), so gridDim.x *
 // kStageRows is a multiple of nb and a thread's column j never changes.
 __global__ void __launch_bounds__(kStagedThreads, 2)
-kq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const float4 *__restrict__ factors, int shared,
+kq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const uint4 *__restrict__ act,
+                 const float4 *__restrict__ factors, int shared,
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb,
                  long long budget, int issue_copies)
 {
@@ -1100,18 +1028,25 @@ kq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const float4 *__re
     load_factors(factors, shared, j, g);
     KqFast st;
     if (kq_fast_setup(g, st)) {
+        bool overflow = false;
         staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
             float2 p[16];
             unpack_pairs(raw, p);
             kq_fast_apply(p, st);
-            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+            const float amax = pair_amax_nan(p);
+            overflow |= !(amax <= 3.40282347e38f);
+            kq_emit<KqOut::kCodes>(p, amax, gi, codes, scales, nullptr);
         });
+        if (overflow)
+            kq_redo_overflow<KqOut::kCodes, false, false>(
+                act, reinterpret_cast<const float *>(factors), shared, int64_t(blockIdx.x) * kStageRows + threadIdx.x,
+                int64_t(gridDim.x) * kStageRows, nblocks, nb, codes, scales, nullptr);
     } else {
         staged_consume(r, nchunks, nblocks, budget, [&](const uint4 (&raw)[4], int64_t gi) {
             float2 p[16];
             unpack_pairs(raw, p);
             kq_direct_apply(p, g);
-            kq_emit<KqOut::kCodes>(p, gi, codes, scales, nullptr);
+            kq_emit<KqOut::kCodes>(p, pair_amax_nan(p), gi, codes, scales, nullptr);
         });
     }
 }
@@ -1269,6 +1204,13 @@ sf_relayout_kernel(const uint8_t *__restrict__ scales, uint8_t *__restrict__ sf,
     }
 }
 
+// 16-byte global -> shared copy through L2 only (cp.async, no register staging).
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void *g)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+
+
 // The quantizer fused with the normalisation that produces its input (KroQuant
 // abstract: normalisation layers force the transform online).  For every token
 // row h of a bf16 activation: LayerNorm without affine (mean, biased
@@ -1322,7 +1264,7 @@ __device__ __forceinline__ void norm_emit(float2 (&p)[16], int64_t r, int j, int
         scales[off] = uint8_t(sb);
         if ((nb & 1) && j == nb - 1) scales[off + 1] = 0;
     } else {
-        kq_emit<KqOut::kCodes>(p, r * nb + j, codes, scales, nullptr);
+        kq_emit<KqOut::kCodes>(p, pair_amax_nan(p), r * nb + j, codes, scales, nullptr);
     }
 }
 
@@ -1634,6 +1576,7 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 }
 
 #include "kq_mma.cuh"
+#include "kq_ring.cuh"
 #include "mxf4_gemm.cuh"
 
 // ---------------------------------------------------------------------------
@@ -1687,8 +1630,8 @@ Geometry pinned_geometry(int64_t M, int64_t nb, int64_t target_threads)
 // per SM (occupancy query, cached per device and kernel).
 enum KernelId {
     kKqDirect, kKqDirectF32, kKqPacked, kKqPackedF32, kSqPacked, kMxPacked, kFold,
-    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq, kKqLean, kKqPacked2,
-    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kKqAsync4, kKqAsync6, kNormRows, kNormKqSf, kNumKernels
+    kKqStaged, kSqStaged, kMxStaged, kKqMma, kKqMmaF32, kKqLu, kFwht, kInverse, kDequant, kNormKq,
+    kKqPackedSf, kMxF32, kMxF32Sf, kSfRelayout, kNormRows, kNormKqSf, kKqRing, kNumKernels
 };
 std::atomic<int> g_ctas_per_sm[kNumKernels][kMaxDevices];
 
@@ -1761,14 +1704,14 @@ int encode_fn(EncodeTiledFn *out)
 
 // The activation as a [nblocks][32] bf16 matrix, boxes of kStageRows rows,
 // 64-byte swizzle (the row is exactly one 64-byte swizzle span).
-int encode_act_map(const void *act, int64_t nblocks, CUtensorMap *map)
+int encode_act_map(const void *act, int64_t nblocks, CUtensorMap *map, int box_rows = kStageRows)
 {
     EncodeTiledFn enc;
     int rc = encode_fn(&enc);
     if (rc != KQ_OK) return rc;
     const cuuint64_t dims[2] = {32, cuuint64_t(nblocks)};
     const cuuint64_t strides[1] = {64};
-    const cuuint32_t box[2] = {32, cuuint32_t(kStageRows)};
+    const cuuint32_t box[2] = {32, cuuint32_t(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(act), dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1941,28 +1884,6 @@ constexpr long long kWaitBudget = 1LL << 31;
 // Largest block count the staged path takes (row coordinates are int32).
 constexpr int64_t kStagedMaxBlocks = (int64_t(1) << 31) - kStageRows;
 
-// As launch_pinned, for a kernel with dynamic shared memory (the occupancy
-// query then accounts for it).
-template <typename Kernel>
-int launch_pinned_smem(const char *fn, KernelId id, Kernel kernel, size_t smem, int64_t M, int64_t nb, Geometry *geo)
-{
-    int sms = 0;
-    int rc = sm_count(&sms);
-    if (rc != KQ_OK) return rc;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    int c = (dev >= 0 && dev < kMaxDevices) ? g_ctas_per_sm[id][dev].load(std::memory_order_relaxed) : 0;
-    if (c <= 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c, reinterpret_cast<const void *>(kernel), kThreads, smem);
-        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "%s: occupancy query: %s", fn, cudaGetErrorString(e));
-        if (c < 1) c = 1;
-        if (dev >= 0 && dev < kMaxDevices) g_ctas_per_sm[id][dev].store(c, std::memory_order_relaxed);
-    }
-    *geo = pinned_geometry(M, nb, int64_t(sms) * c * kThreads);
-    return KQ_OK;
-}
-
 template <typename Kernel>
 int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t nb, Geometry *geo)
 {
@@ -1974,12 +1895,54 @@ int launch_pinned(const char *fn, KernelId id, Kernel kernel, int64_t M, int64_t
     return KQ_OK;
 }
 
+// Grid of the two-block ring kernel (variant 9): one CTA per SM, G a
+// multiple of q = nb / gcd(nb, P) so that G * P is a multiple of nb and a
+// thread's column never changes (any G with shared factors), at most the SM
+// count and no more than the chunks need.  0 where no such G fits.
+unsigned ring_grid(int64_t nchunks, int64_t nb, int shared, int P, int sms)
+{
+    const int64_t q = shared ? 1 : nb / gcd64(nb, P);
+    if (q > sms) return 0;
+    int64_t G = (sms / q) * q;
+    const int64_t need = ((nchunks + q - 1) / q) * q;
+    if (G > need) G = need;
+    return unsigned(G);
+}
+
+// Launch of the ring kernel with P consumers; *launched = false (and KQ_OK)
+// where its grid rule or its int32 row coordinates rule the shape out, and
+// the caller then runs variant 2.
+template <int P>
+int ring_launch(const char *fn, KernelId id, const void *act, const float *factors, int shared, uint8_t *codes,
+                uint8_t *scales, int64_t nblocks, int64_t nb, cudaStream_t stream, bool *launched)
+{
+    using C = ring::Cfg<P>;
+    *launched = false;
+    if (nblocks > int64_t(INT32_MAX) - 2 * P) return KQ_OK;
+    int sms = 0;
+    int rc = sm_count(&sms);
+    if (rc != KQ_OK) return rc;
+    const int64_t nchunks = (nblocks + P - 1) / P;
+    const unsigned grid = ring_grid(nchunks, nb, shared, P, sms);
+    if (grid == 0) return KQ_OK;
+    auto k = ring::kq_ring_kernel<P>;
+    if ((rc = smem_prepare(id, reinterpret_cast<const void *>(k), C::kSmem)) != KQ_OK) return rc;
+    CUtensorMap map;
+    if ((rc = encode_act_map(act, nblocks, &map, C::kBoxRows)) != KQ_OK) return rc;
+    k<<<grid, C::kThreads, C::kSmem, stream>>>(map, static_cast<const uint4 *>(act), factors, shared,
+                                               reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb),
+                                               kWaitBudget);
+    *launched = true;
+    return launch_check(fn);
+}
+
 // Kernel variants of the KroQuant quantizer: 1 = one block per thread, direct
 // 2x2 stages; 2 = packed pairs with the unit-diagonal split, register
 // prefetch; 3 = the arithmetic of 2 on TMA-staged input; 4 = the transform
-// as tcgen05 MMAs on K split into three bf16 parts.  0 = the default,
-// the fastest on the benchmark shapes (2: the staged input does not help a
-// kernel whose limit is its instruction stream; see the profiles).
+// as tcgen05 MMAs on K split into three bf16 parts; 9 = the operations of 2
+// on two rows per thread from a TMA ring.  0 = the default, the fastest on
+// the benchmark shapes (2: every form shares the FMA-pipe floor of seven
+// lane operations per element, and 2 hides its latency best).
 constexpr int kDefaultVariant = 2;
 
 int kq_launch(const char *fn, int variant, const void *act, const float *factors, int shared,
@@ -1990,44 +1953,15 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
     if (rc == 1) return ok();
     if (rc != KQ_OK) return rc;
     if (variant == 0) variant = kDefaultVariant;
-    if (variant < 1 || variant > 8)
+    if (variant < 1 || variant > 9 || (variant >= 5 && variant <= 8))
         return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
-    if ((variant == 7 || variant == 8) && !f32) {
-        const int64_t nb7 = d / kBlk;
-        const int depth = variant == 7 ? 4 : 6;
-        auto k = variant == 7 ? kq_async_kernel<4> : kq_async_kernel<6>;
-        const KernelId id = variant == 7 ? kKqAsync4 : kKqAsync6;
-        const size_t smem = size_t(depth) * kThreads * 64;   // per warp depth x 2 KB
-        if ((rc = smem_prepare(id, reinterpret_cast<const void *>(k), smem)) != KQ_OK) return rc;
-        Geometry geo;
-        if ((rc = launch_pinned_smem(fn, id, k, smem, M, nb7, &geo)) != KQ_OK) return rc;
-        k<<<geo.grid, kThreads, smem, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
-                                                shared, reinterpret_cast<uint4 *>(codes), scales, M * nb7, int(nb7), geo.T);
-        return launch_check(fn);
+    if (variant == 9 && !f32) {
+        const int64_t nb9 = d / kBlk;
+        bool launched = false;
+        rc = ring_launch<256>(fn, kKqRing, act, factors, shared, codes, scales, M * nb9, nb9, stream, &launched);
+        if (rc != KQ_OK || launched) return rc;
     }
-    if (variant == 7 || variant == 8) variant = 2;   // the fp32 export: the same arithmetic in variant 2
-    if (variant == 6 && !f32) {
-        const int64_t nb6 = d / kBlk;
-        Geometry geo;
-        auto k = kq_packed2_kernel;
-        if ((rc = launch_pinned(fn, kKqPacked2, k, M, nb6, &geo)) != KQ_OK) return rc;
-        k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
-                                             shared, reinterpret_cast<uint4 *>(codes), scales, M * nb6, int(nb6),
-                                             geo.T);
-        return launch_check(fn);
-    }
-    if (variant == 6) variant = 2;
-    if (variant == 5 && !f32) {
-        const int64_t nb5 = d / kBlk;
-        Geometry geo;
-        auto k = kq_lean_kernel;
-        if ((rc = launch_pinned(fn, kKqLean, k, M, nb5, &geo)) != KQ_OK) return rc;
-        k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act), reinterpret_cast<const float4 *>(factors),
-                                             shared, reinterpret_cast<uint4 *>(codes), scales, M * nb5, int(nb5),
-                                             geo.T);
-        return launch_check(fn);
-    }
-    if (variant == 5) variant = 2;   // the fp32 export: the same arithmetic in variant 2
+    if (variant == 9) variant = 2;   // the fp32 export, or a shape the ring's grid rule excludes
     if (variant == 4 && M < (int64_t(1) << 31)) {
         const int64_t nb4 = d / kBlk;
         CUtensorMap map;
@@ -2068,7 +2002,7 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
         if ((rc = staged_prepare(kKqStaged, reinterpret_cast<const void *>(kq_staged_kernel), &resident)) != KQ_OK)
             return rc;
         kq_staged_kernel<<<staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream>>>(
-            map, f, shared, reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb), kWaitBudget, 1);
+            map, a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb), kWaitBudget, 1);
     } else if (variant == 1) {
         if (f32) {
             auto k = kq_butterfly_kernel<KqOut::kF32>;
@@ -2609,7 +2543,7 @@ int kq_selftest_bounded_wait(cudaStream_t stream)
     void *dummy = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&dummy, g_selftest_dummy);
     if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "kq_selftest_bounded_wait: %s", cudaGetErrorString(e));
-    const int64_t nblocks = int64_t(kStageRows) * (kStages + 1);
+    const int64_t nblocks = kSelftestBlocks;
     CUtensorMap map;
     int rc = encode_act_map(dummy, nblocks, &map);
     if (rc != KQ_OK) return rc;
