@@ -3,28 +3,35 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one pass of the whole hot path over one batch: the KroQuant
-quantizer, the SmoothQuant quantizer and the plain MXFP4 quantizer, each on
-both PixArt-Sigma layer inputs (M = 8192 tokens x d = 1152 and d = 4608, bf16,
-seeded synthetic activations).  The headline value is the KroQuant quantizer's
-algorithmic HBM throughput, 2.53125 bytes per element (2 B bf16 in, 0.5 B
-codes, 1/32 B scale) over the summed duration of its launches.
+A step is one pass of the whole hot path over one batch of each DiT-shaped
+workload: the KroQuant quantizer, the SmoothQuant quantizer and the plain
+MXFP4 quantizer, each on every layer input of PixArt-Sigma (M = 8192 tokens x
+d = 1152 and 4608), SANA (2048 x 2240 and 5600, one shared factor set) and
+FLUX (4608 x 3072 and 12288), bf16, seeded synthetic activations: 18 launches.
+The headline value is the KroQuant quantizer's algorithmic HBM throughput,
+2.53125 bytes per element (2 B bf16 in, 0.5 B codes, 1/32 B scale) over the
+summed duration of its six launches; the same for SmoothQuant and plain MXFP4,
+per workload and per layer, is reported beside it.
 
 Timing: inputs resident in HBM and rotated over per-layer input sets so that
 a set is read again only after >= 3x the L2 of other input; per (quantizer,
-layer) a CUDA graph of 200 back-to-back launches; a round replays the six
-graphs in step order; CUDA events on the launching stream sit between graph
-replays; barrier + synchronize on both sides; max over ranks.  Multi-GPU: every
-rank quantizes its own batch (weak scaling, no collective on the data path).
+layer) a CUDA graph of min(K, 200) back-to-back launches; a round replays the
+18 graphs in step order; CUDA events on the launching stream sit between
+graph replays.  The clocks are spun up by untimed rounds that end right
+before the timed region (the nvidia-smi sampler is started before them), and
+the bounded-wait counter of the library must read 0 after the timed region.
+Barrier + synchronize on both sides; max over ranks.  Multi-GPU: every rank
+quantizes its own batch (weak scaling, no collective on the data path).
 
 `--impl reference` times the CPU oracle (oracle/, plain C) on the host cores on
 a bounded sample of the same workload and prints the same JSON line.
 
 Besides the step line, the JSON carries the roofline of the dominant launch
-(with the DRAM traffic of an ncu capture, valid for the kernel source it was
-taken on), the end-to-end figure through host buffers (H2D, quantize and D2H
-pipelined over three streams), the CPU-oracle baseline, the SM clocks sampled
-during the timed region and the number of kernel launches.
+(the KroQuant quantizer on the largest layer, FLUX d = 12288, with the DRAM
+traffic of an ncu capture, valid for the kernel source it was taken on), the
+end-to-end figure through host buffers (H2D, quantize and D2H pipelined over
+three streams), the CPU-oracle baseline, the SM clocks sampled during the
+timed region and the number of kernel launches.
 
 Other modes (one JSON line each):
     --mode kernel --kernel K --shape MxD     one quantizer or variant at one shape
@@ -57,19 +64,20 @@ if ROOT not in sys.path:
 
 METRIC = "KroQuant quantizer HBM GB/s (bf16→MXFP4+E8M0) and % of B200 peak vs SQ"
 BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 32.0
-WORKLOAD = "pixart"
+WORKLOADS = ("pixart", "sana", "flux")
+WORKLOAD_NAMES = {"pixart": "PixArt-Sigma", "sana": "SANA", "flux": "FLUX"}
 GRAPH_STEPS = 200          # launches per captured graph
 E2E_CHUNKS = 4             # row chunks per layer in the end-to-end (host buffer) pipeline
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0
 KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.cu")]
 
-# DRAM traffic per launch of the dominant kernel (KroQuant quantizer, d = 4608
-# layer), from one ncu capture, valid only for the kernel source it was taken
+# DRAM traffic per launch of the dominant kernel (KroQuant quantizer on the
+# largest layer, FLUX 4608 x 12288), from one ncu capture, valid only for the kernel source it was taken
 # on (sha256 prefix of kernel_source_text: the kernel, its helpers and its
 # launch path).  Updated after each capture.
-TRAFFIC = {"source_sha": "e7f650230a4d9a4a", "bytes_per_launch": 79977728.0,
-           "capture": "ncu --set full, kq_packed_kernel, 8192x4608, dram__bytes_read.sum + dram__bytes_write.sum"}
+TRAFFIC = {"source_sha": "2f5b27cf4f68040f", "bytes_per_launch": 127422976.0,
+           "capture": "ncu --set full, kq_packed_kernel, 4608x12288, dram__bytes_read.sum + dram__bytes_write.sum"}
 
 
 # The code that determines the dominant kernel (KroQuant variant 2): the
@@ -217,18 +225,30 @@ def barrier(pg):
 
 # ----------------------------------------------------------------------------- inputs
 def workload_inputs(seed_offset: int = 0, world: int = 1, rank: int = 0):
-    """Layer inputs of the workload: the whole batch (world == 1), or rank's rows of it."""
+    """Layer inputs of every benchmark workload: the whole batch (world == 1), or rank's rows of it."""
     from w4a4_mxfp4_post_b200 import shard, synth
 
     layers = []
-    for (M, d, model, shared, seed) in synth.workload_layers(WORKLOAD):
-        rows = shard.row_range(M, world, rank) if world > 1 else None
-        x = synth.activation(model, M, d, seed + seed_offset, rows=rows)
-        M = x.shape[0]
-        F = synth.factors(d // 32, seed + seed_offset, shared=shared)
-        m = synth.sq_multipliers(x)
-        layers.append({"M": M, "d": d, "x": x, "F": F, "m": m, "shared": shared})
+    for wl in WORKLOADS:
+        for (M, d, model, shared, seed) in synth.workload_layers(wl):
+            rows = shard.row_range(M, world, rank) if world > 1 else None
+            x = synth.activation(model, M, d, seed + seed_offset, rows=rows)
+            M = x.shape[0]
+            F = synth.factors(d // 32, seed + seed_offset, shared=shared)
+            m = synth.sq_multipliers(x)
+            layers.append({"workload": wl, "M": M, "d": d, "x": x, "F": F, "m": m, "shared": shared})
     return layers
+
+
+def workload_text():
+    from w4a4_mxfp4_post_b200 import synth
+
+    parts = []
+    for wl in WORKLOADS:
+        w = synth.WORKLOADS[wl]
+        parts.append(f"{WORKLOAD_NAMES[wl]} M={w['M']} x d in {{{', '.join(str(d) for d in w['ds'])}}}"
+                     + (" (one shared factor set)" if w["factors"] == "shared" else ""))
+    return "DiT layer inputs: " + "; ".join(parts) + "; bf16 -> MXFP4 (E2M1 codes + E8M0 scales)"
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
@@ -309,9 +329,10 @@ def gpu_arm(args, rank, local, world, pg):
 
     quantizers = ("kq", "sq", "mx")
     n_layers = len(layers)
-    pairs = [(q, li) for q in quantizers for li in range(n_layers)]
+    pairs = [(q, li) for li in range(n_layers) for q in quantizers]
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
+    kq.kq_wait_timeouts(reset=True)
     # warm-up steps (eager)
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -320,7 +341,7 @@ def gpu_arm(args, rank, local, world, pg):
     stream.synchronize()
 
     # One CUDA graph per (quantizer, layer) holding S back-to-back launches;
-    # a round replays the six graphs in step order, so K steps = K/S rounds
+    # a round replays the 18 graphs in step order, so K steps = K/S rounds
     # (the last round shorter).  Events sit only between graph replays.
     K = args.steps
     S = min(GRAPH_STEPS, K)
@@ -338,24 +359,24 @@ def gpu_arm(args, rank, local, world, pg):
     for g in list(graphs.values()) + list(tails.values()):
         g.replay()
     stream.synchronize()
-    # more untimed rounds until the SM and HBM clocks have left their idle states
-    t_end = time.perf_counter() + SPINUP_S
-    with torch.cuda.stream(stream):
-        while time.perf_counter() < t_end:
-            for pl in pairs:
-                graphs[pl].replay()
-            stream.synchronize()
 
     rounds = [graphs] * full + ([tails] if tail else [])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(pairs) + 1)] for _ in rounds]
     uuid = getattr(props, "uuid", None)
     gpu_id = f"GPU-{uuid}" if uuid is not None else str(local)
     clocks = ClockSampler(gpu_id) if rank == 0 else None
-    barrier(pg)
-    torch.cuda.synchronize(dev)
     if clocks:
         clocks.start()
-        time.sleep(0.3)
+    barrier(pg)
+    # untimed rounds until the SM and HBM clocks have left their idle states;
+    # they run right up to the timed region, so no launch of it starts cold
+    t_end = time.perf_counter() + SPINUP_S
+    with torch.cuda.stream(stream):
+        while time.perf_counter() < t_end:
+            for pl in pairs:
+                graphs[pl].replay()
+            stream.synchronize()
+    barrier(pg)
     with torch.cuda.stream(stream):
         for r, gs in enumerate(rounds):
             evs[r][0].record(stream)
@@ -365,30 +386,50 @@ def gpu_arm(args, rank, local, world, pg):
     torch.cuda.synchronize(dev)
     barrier(pg)
     clk = clocks.stop() if clocks else None
+    timeouts = kq.kq_wait_timeouts(reset=True)
+    if timeouts:
+        raise SystemExit(f"{timeouts} bounded waits of the library gave up during the benchmark: "
+                         "its launches did not finish their work, the timing is void")
 
     total_ms = evs[0][0].elapsed_time(evs[-1][-1])
     per = {q: [0.0] * n_layers for q in quantizers}
     for r in range(len(rounds)):
         for k, (q, li) in enumerate(pairs):
             per[q][li] += evs[r][k].elapsed_time(evs[r][k + 1])
-    us = {q: [1e3 * v / K for v in per[q]] for q in per}      # mean us per launch, gaps in the graph included
+    us_local = {q: [1e3 * v / K for v in per[q]] for q in per}   # mean us per launch, gaps in the graph included
 
-    # kernel-only quantizer throughput from the per-launch means
+    # max over ranks of every per-launch mean and of the step time
+    flat = [total_ms] + [us_local[q][li] for q in quantizers for li in range(n_layers)]
+    vals = allreduce_max(pg, flat, dev)
+    total_ms_max = vals[0]
+    us = {q: vals[1 + qi * n_layers: 1 + (qi + 1) * n_layers] for qi, q in enumerate(quantizers)}
     elems = [L["M"] * L["d"] for L in layers]
     qbytes = sum(BYTES_PER_ELEM * e for e in elems)
-    q_time_us = {name: sum(us[name]) for name in us}
-    vals = allreduce_max(pg, [total_ms] + [q_time_us[n] for n in ("kq", "sq", "mx")] + us["kq"], dev)
-    total_ms_max = vals[0]
-    qt = dict(zip(("kq", "sq", "mx"), vals[1:4]))
-    kq_us_max = vals[4:]
     all_bytes = allreduce_sum(pg, [qbytes], dev)[0]          # units all ranks processed per step
-    gbs = {n: all_bytes / (qt[n] * 1e-6) / 1e9 for n in qt}
+    qt = {q: sum(us[q]) for q in quantizers}
+    gbs = {q: all_bytes / (qt[q] * 1e-6) / 1e9 for q in quantizers}
+    peak, peak_src = measured_peak()
+
+    def rate(nbytes, t_us):
+        g = nbytes / (t_us * 1e-6) / 1e9
+        return {"gbs": round(g, 1), "frac_of_peak": round(g / peak, 4)}
+
+    per_workload = {}
+    for wl in WORKLOADS:
+        idx = [li for li, L in enumerate(layers) if L["workload"] == wl]
+        wb = sum(BYTES_PER_ELEM * elems[li] for li in idx)
+        entry = {"layers": {f"{layers[li]['M']}x{layers[li]['d']}": {
+            q: {"us": round(us[q][li], 3), **rate(BYTES_PER_ELEM * elems[li], us[q][li])} for q in quantizers}
+            for li in idx}}
+        for q in quantizers:
+            entry[q] = rate(wb, sum(us[q][li] for li in idx))
+        entry["kq_time_vs_sq"] = round(sum(us["kq"][li] for li in idx) / sum(us["sq"][li] for li in idx), 4)
+        per_workload[WORKLOAD_NAMES[wl]] = entry
 
     # dominant kernel: the KroQuant launch on the largest layer
     dom = int(np.argmax(elems))
     dom_bytes = BYTES_PER_ELEM * elems[dom]
-    peak, peak_src = measured_peak()
-    achieved = dom_bytes / (kq_us_max[dom] * 1e-6) / 1e9
+    achieved = dom_bytes / (us["kq"][dom] * 1e-6) / 1e9
     sha = source_sha()
     traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["source_sha"] == sha else None
 
@@ -407,31 +448,34 @@ def gpu_arm(args, rank, local, world, pg):
         "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": "f32",
-        "data": "synthetic (seeded PixArt-Sigma-shaped activations with per-channel outliers; no trained weights)",
+        "data": "synthetic (seeded DiT-shaped activations with per-channel outliers; no trained weights)",
         "config": {
-            "workload": "PixArt-Sigma layer inputs: M=8192 tokens x d in {1152, 4608}, bf16 -> MXFP4 (E2M1 codes + "
-                        "E8M0 scales), per-block Kronecker factors",
-            "M": layers[0]["M"], "d": [L["d"] for L in layers], "quantizers_per_step": ["kq", "sq", "mx"],
+            "workload": workload_text(),
+            "layers": [f"{L['M']}x{L['d']}" for L in layers],
+            "quantizers_per_step": list(quantizers),
             "l2": f"inputs larger than L2: per layer {[ls['n'] for ls in layer_sets]} rotating input sets "
                   f"({resident / 2**20:.0f} MiB resident, L2 {l2 / 2**20:.0f} MiB); a set is reused only after "
                   ">= 3x L2 of other input",
-            "timing": f"per (quantizer, layer) a CUDA graph of {S} back-to-back launches; a step's six graphs "
-                      "replayed in order; CUDA events between replays on the launching stream",
+            "timing": f"per (quantizer, layer) a CUDA graph of {S} back-to-back launches; a step's 18 graphs "
+                      "replayed in order; CUDA events between replays on the launching stream; untimed "
+                      f"spin-up rounds ({SPINUP_S} s) end right before the timed region",
             "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'row shards of one batch'}"
                            ", no collective on the data path)",
         },
         "kernels": {
-            n: {"gbs": round(gbs[n], 1), "frac_of_peak": round(gbs[n] / peak, 4),
-                "frac_of_8tbs_spec": round(gbs[n] / SPEC_HBM_GBS, 4),
-                "us_per_launch": {str(L["d"]): round(v, 3) for L, v in zip(layers, us[n])}}
-            for n in ("kq", "sq", "mx")
+            q: {"gbs": round(gbs[q], 1), "frac_of_peak": round(gbs[q] / peak, 4),
+                "frac_of_8tbs_spec": round(gbs[q] / SPEC_HBM_GBS, 4)}
+            for q in quantizers
         },
+        "workloads": per_workload,
         "kq_time_vs_sq": round(qt["kq"] / qt["sq"], 4),
-        "roofline": {"bound": "hbm", "kernel": f"kq_quantize d={layers[dom]['d']}", "achieved": round(achieved, 1),
-                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+        "roofline": {"bound": "hbm", "kernel": f"kq_quantize {layers[dom]['M']}x{layers[dom]['d']}",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src},
         "e2e": e2e,
         "gpu_launches": K * len(pairs),
+        "wait_timeouts": timeouts,
         "clocks": clk,
         "kernel_source_sha": sha,
     }
@@ -520,7 +564,7 @@ def e2e_kq(args, layers, dev, stream, kq, pg, world):
 def cpu_baseline_block(layers, seconds):
     r = time_oracle(layers, seconds)
     return {"value": round(r["kq_gbs"], 4), "unit": "GB/s", "cores": r["threads"], "kind": "oracle",
-            "sample": f"{r['passes']} full passes of the workload (KQ, SQ, MX on both layers), "
+            "sample": f"{r['passes']} full passes of the workload (KQ, SQ, MX on all six layers), "
                       f"{r['t_all']:.1f} s of oracle time; value = KQ bytes / KQ time"}
 
 
@@ -538,7 +582,7 @@ def reference_arm(args, rank, world):
     probe = time_oracle(layers, 0.0, rows_per_pass=64)
     per_row = (time.perf_counter() - t0) / 64
     budget = args.ref_seconds
-    rows = int(max(1, min(layers[0]["M"], budget / max(1, args.steps + args.warmup) / per_row)))
+    rows = int(max(1, min(max(L["M"] for L in layers), budget / max(1, args.steps + args.warmup) / per_row)))
     for _ in range(args.warmup):
         time_oracle(layers, 0.0, rows_per_pass=rows)
     t_kq = 0.0
@@ -555,8 +599,7 @@ def reference_arm(args, rank, world):
         "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * t_all / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": "PixArt-Sigma layer inputs: M=8192 tokens x d in {1152, 4608}, bf16 -> MXFP4",
-                   "sample_rows_per_layer_per_step": rows},
+        "config": {"workload": workload_text(), "sample_rows_per_layer_per_step": rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"{rows} rows of each layer per step (KQ, SQ, MX), {args.steps} steps"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
