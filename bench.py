@@ -674,6 +674,9 @@ def time_launches(kind, inp, launches, warmup, stream, graph=True):
             kq.mx_quantize(inp.xs[k], inp.cs[k], inp.ss[k], stream=stream)
         elif kind == "norm_kq":
             kq.norm_kq_quantize(inp.xs[k], inp.gamma, inp.beta, inp.F, 1e-6, False, inp.cs[k], inp.ss[k], stream=stream)
+        elif kind.startswith("norm_kq_v"):
+            kq.norm_kq_quantize_variant(int(kind[9:]), inp.xs[k], inp.gamma, inp.beta, inp.F, 1e-6, False, inp.cs[k],
+                                        inp.ss[k], stream=stream)
         elif kind == "kq_lu":
             kq.kq_quantize_lu(inp.xs[k], inp.P, False, inp.cs[k], inp.ss[k], stream=stream)
         elif kind.startswith("fwht"):
@@ -1009,7 +1012,8 @@ def main():
                          "sqnr: quantisation-error proxy per method; gemm: the W4A4 product; "
                          "compare: several quantizers interleaved at --shapes")
     ap.add_argument("--kernel", default="kq",
-                    help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H> or norm_kq")
+                    help="kernel mode: kq, sq, mx, kq_v<variant>, sq_v<n>, mx_v<n>, kq_lu, fwht<H>, norm_kq or "
+                         "norm_kq_v<n>")
     ap.add_argument("--kernels", default="kq,sq,mx",
                     help="sweep / compare mode: comma-separated kernels; gemm mode: comma-separated tile "
                          "configurations")

@@ -127,6 +127,21 @@ int norm_kq_quantize(const void *h_bf16, const float *gamma, const float *beta,
                      uint8_t *out_codes, uint8_t *out_scales,
                      int64_t M, int64_t d, cudaStream_t stream);
 
+/* Test export: norm_kq_quantize through a chosen kernel (the same result up
+ * to the rounding of the row statistics, within the transform tolerance):
+ *   0  the default (3 from 192 block columns up, else 1 where it fits, else 2),
+ *   1  one warp per row, rows streamed once into shared-memory row buffers
+ *      beside a per-column coefficient table (falls to 2 where none fits),
+ *   2  one warp per row, the row read twice (statistics, then transform),
+ *   3  one CTA per row, one thread per block column: coefficients in
+ *      registers, rows streamed once through a per-thread cp.async ring,
+ *      row statistics by a CTA reduction.
+ * Other values return KQ_ERR_VARIANT. */
+int norm_kq_quantize_variant(int variant, const void *h_bf16, const float *gamma, const float *beta,
+                             int64_t nsamples, float eps, const float *factors, int shared,
+                             uint8_t *out_codes, uint8_t *out_scales,
+                             int64_t M, int64_t d, cudaStream_t stream);
+
 /* Fixed-Hadamard baseline (the pages' comparison point for the on-the-fly
  * kernel, a fast Walsh-Hadamard transform): y = H_H x / sqrt(H) on every H
  * consecutive channels of a row, H_H the Sylvester Hadamard matrix, H a

@@ -154,6 +154,9 @@ def test_norm_inverse_dequant_argument_errors(L):
     assert L.norm_kq_quantize(P(16), None, P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 64, None) == -1
     assert L.norm_kq_quantize(P(16), P(8), P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 64, None) == -3
     assert L.norm_kq_quantize(P(16), P(16), P(16), 1, f(-1.0), P(16), 0, P(16), P(16), 4, 64, None) == -2
+    # the variant export: same checks, then the variant number
+    assert L.norm_kq_quantize_variant(1, P(16), P(16), P(16), 2, f(1e-6), P(16), 0, P(16), P(16), 5, 64, None) == -2
+    assert L.norm_kq_quantize_variant(9, P(16), P(16), P(16), 1, f(1e-6), P(16), 0, P(16), P(16), 4, 64, None) == -5
     assert L.kq_inverse_f32(P(16), P(16), 0, None, 4, 64, None) == -1
     assert L.kq_inverse_f32(P(16), P(16), 0, P(16), 4, 40, None) == -2
     assert L.mx_dequantize(P(16), P(16), P(8), 4, 64, None) == -3

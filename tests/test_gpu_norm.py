@@ -10,6 +10,7 @@ from w4a4_mxfp4_post_b200 import synth
 pytestmark = pytest.mark.gpu
 
 EPS = 1e-6
+NORM_VARIANTS = (0, 1, 2, 3)
 
 
 def dev(a, device):
@@ -34,11 +35,13 @@ def test_norm_kq_matches_oracle(cuda_device, M, d, ns, shared):
     h = synth.activation("pixart", M, d, seed=M + d)
     gamma, beta = synth.adaln(ns, d, seed=d)
     F = synth.factors(d // 32, seed=d, shared=shared)
-    c, s = kq.norm_kq_quantize(dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device),
-                               dev(F, cuda_device), eps=EPS, shared=shared)
     ref = oracle.norm_kq(h, gamma, beta, EPS, F, shared=shared, want=("codes", "y", "absb"))
-    res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
-    assert res["ok"], res
+    args = (dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device), dev(F, cuda_device))
+    # the default and each of the three kernels (row buffers, row re-read, one CTA per row)
+    for v in NORM_VARIANTS:
+        c, s = kq.norm_kq_quantize_variant(v, *args, eps=EPS, shared=shared)
+        res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
+        assert res["ok"], (v, res)
 
 
 def test_norm_kq_shape_errors(cuda_device):
@@ -70,7 +73,7 @@ def test_norm_kq_sf_layout_matches_row_major_path(cuda_device, M, d, ns):
     np.testing.assert_array_equal(sf.cpu().numpy(), oracle.scales_to_sf(s.cpu().numpy()))
 
 
-@pytest.mark.parametrize("M,d", [(256, 1152), (300, 4608)])
+@pytest.mark.parametrize("M,d", [(256, 1152), (300, 4608), (64, 12288)])
 def test_norm_kq_large_mean_takes_the_two_pass_variance(cuda_device, M, d):
     """Rows whose mean is large against their spread (each row shifted by half
     its root mean square, so mu^2 > E[x^2] / 64): the one-sweep variance
@@ -85,8 +88,18 @@ def test_norm_kq_large_mean_takes_the_two_pass_variance(cuda_device, M, d):
     assert np.all(hv.mean(axis=1) ** 2 > (hv * hv).mean(axis=1) / 64)     # the two-pass branch
     gamma, beta = synth.adaln(2, d, seed=d)
     F = synth.factors(d // 32, seed=d)
-    c, s = kq.norm_kq_quantize(dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device),
-                               dev(F, cuda_device), eps=EPS)
     ref = oracle.norm_kq(h, gamma, beta, EPS, F, want=("codes", "y", "absb"))
-    res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
-    assert res["ok"], res
+    args = (dev_bf16(h, cuda_device), dev(gamma, cuda_device), dev(beta, cuda_device), dev(F, cuda_device))
+    for v in NORM_VARIANTS:
+        c, s = kq.norm_kq_quantize_variant(v, *args, eps=EPS)
+        res = pc.check_kq(c.cpu().numpy(), s.cpu().numpy(), ref["codes"], ref["scales"], ref["y"], ref["absb"])
+        assert res["ok"], (v, res)
+
+
+def test_norm_kq_variant_errors(cuda_device):
+    h = dev_bf16(synth.activation("pixart", 4, 64, 1), cuda_device)
+    g = dev(np.zeros((1, 64), np.float32), cuda_device)
+    F = dev(synth.factors(2, 1), cuda_device)
+    with pytest.raises(kq.KroQuantError) as ei:
+        kq.norm_kq_quantize_variant(4, h, g, g.clone(), F)
+    assert ei.value.status == kq.KQ_ERR_VARIANT

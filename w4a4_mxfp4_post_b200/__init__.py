@@ -33,7 +33,7 @@ __all__ = [
     "sq_quantize_variant", "mx_quantize_variant", "kq_wait_timeouts", "kq_selftest_bounded_wait",
     "kq_transform_f32_variant", "kq_quantize_lu", "fwht_quantize", "kq_inverse_f32", "mx_dequantize", "norm_kq_quantize",
     "KQ_SCALES_ROWMAJOR", "KQ_SCALES_SF", "kq_sf_bytes", "kq_quantize_sf", "mx_quantize_f32", "mx_scales_to_sf",
-    "mxf4_gemm", "mxf4_gemm_variant", "norm_kq_quantize_sf",
+    "mxf4_gemm", "mxf4_gemm_variant", "norm_kq_quantize_sf", "norm_kq_quantize_variant",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkroquant.so")
@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
         L.norm_kq_quantize.restype = ctypes.c_int
         L.norm_kq_quantize_sf.argtypes = L.norm_kq_quantize.argtypes
         L.norm_kq_quantize_sf.restype = ctypes.c_int
+        L.norm_kq_quantize_variant.argtypes = [ctypes.c_int] + L.norm_kq_quantize.argtypes
+        L.norm_kq_quantize_variant.restype = ctypes.c_int
         L.kq_sf_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
         L.kq_sf_bytes.restype = ctypes.c_int64
         _lib = L
@@ -272,6 +274,12 @@ def fwht_quantize(act, H, out_codes=None, out_scales=None, stream=None):
 def norm_kq_quantize(h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=None, out_scales=None,
                      stream=None):
     """LayerNorm + AdaLN modulation (gamma, beta: [nsamples, d]) fused with kq_quantize."""
+    return norm_kq_quantize_variant(0, h, gamma, beta, factors, eps, shared, out_codes, out_scales, stream)
+
+
+def norm_kq_quantize_variant(variant, h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=None,
+                             out_scales=None, stream=None):
+    """norm_kq_quantize through a chosen kernel (0 = the default)."""
     torch = _torch()
     M, d = _act(h)
     _need(gamma, "gamma", torch.float32, h.device)
@@ -280,8 +288,12 @@ def norm_kq_quantize(h, gamma, beta, factors, eps=1e-6, shared=False, out_codes=
         raise ValueError("gamma and beta must be [nsamples, d]")
     _factors(factors, d, shared, h.device)
     out_codes, out_scales = _outs(h, out_codes, out_scales)
-    _call("norm_kq_quantize", h.device, _ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps),
-          _ptr(factors), int(bool(shared)), _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream, h.device))
+    args = (_ptr(h), _ptr(gamma), _ptr(beta), int(gamma.shape[0]), float(eps), _ptr(factors), int(bool(shared)),
+            _ptr(out_codes), _ptr(out_scales), M, d, _stream(stream, h.device))
+    if variant == 0:
+        _call("norm_kq_quantize", h.device, *args)
+    else:
+        _call("norm_kq_quantize_variant", h.device, int(variant), *args)
     return out_codes, out_scales
 
 

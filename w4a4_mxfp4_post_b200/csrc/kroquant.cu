@@ -1579,6 +1579,228 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 #include "kq_ring.cuh"
 #include "mxf4_gemm.cuh"
 
+// Third form of the fused normalisation + quantizer, for long rows (where the
+// per-column table and whole-row buffers of the single-pass kernel do not
+// fit, or fit for too few warps): a CTA takes two rows of its sample at a
+// time, thread t owning block column t (blockDim = nb rounded up to a warp),
+// and holds the two rows' blocks as register pairs p[i] = (row a x_i, row b
+// x_i), as the two-row ring quantizer does: every stage of the transform and
+// every step of the normalisation is one packed f32x2 instruction for both
+// rows, and the two rows are independent chains.  A thread's column never
+// changes, so its transform coefficients sit in registers, and its sample's
+// 1 + gamma and beta in a shared-memory table laid out [q][t] (float4 q of
+// thread t), conflict-free for a warp.  Each thread streams its own 64-byte
+// block of every row through a DEPTH-row cp.async ring in shared memory (a
+// CTA's copies of a row are contiguous; the 16-byte piece p of thread t lands
+// at t * 64 + 16 (p ^ ((t >> 1) & 3)), so the reads back are conflict-free),
+// DEPTH - 2 rows ahead of the pair it transforms: each row is read from HBM
+// once, without a register prefetch.  The row statistics are a CTA reduction:
+// per warp a shuffle reduction of both rows' sums, per CTA the warps' partial
+// sums in a shared array double-buffered by step parity, so one barrier per
+// two rows suffices (a second one only on the two-pass branch).  Per element:
+// x / sigma - mu / sigma (one FMA), times 1 + gamma plus beta, the unit-
+// diagonal transform, MXFP4 -- the other two kernels' arithmetic except that
+// the normalisation is one FMA instead of a subtraction and a product.
+template <bool SF>
+__device__ __forceinline__ void norm_store(uint4 c, uint32_t sb, int64_t r, int j, int nb, uint4 *__restrict__ codes,
+                                           uint8_t *__restrict__ scales)
+{
+    codes[r * nb + j] = c;
+    if constexpr (SF) {
+        const int64_t off = (r >> 7) * (int64_t((nb + 3) >> 2) * 512) + (r & 31) * 16 + ((r >> 5) & 3) * 4 +
+                            int64_t(j >> 2) * 512 + (j & 3);
+        scales[off] = uint8_t(sb);
+        if ((nb & 1) && j == nb - 1) scales[off + 1] = 0;
+    } else {
+        scales[r * nb + j] = uint8_t(sb);
+    }
+}
+
+template <bool SF, int DEPTH, int kMaxThreads>
+__global__ void __launch_bounds__(kMaxThreads, 1)
+norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, const float *__restrict__ beta,
+                    int64_t rows_per, float eps, const float *__restrict__ factors, int shared,
+                    uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int nb, int cps)
+{
+    static_assert(DEPTH % 2 == 0 && DEPTH >= 2, "the ring holds whole pairs of rows");
+    extern __shared__ float4 smc[];
+    const int nt = int(blockDim.x);                                        // threads = nb rounded up to 32
+    const int t = int(threadIdx.x), wid = t >> 5, lane = t & 31, nw = nt >> 5;
+    float4 *gtab = smc;                                                    // [8][nt] (1 + gamma)
+    float4 *btab = smc + 8 * nt;                                           // [8][nt] beta
+    uint4 *ring = reinterpret_cast<uint4 *>(smc + 16 * nt);                // [DEPTH][nt * 4]
+    float4 *red = reinterpret_cast<float4 *>(ring + DEPTH * nt * 4);       // [2][nw] (sums, squares) of a, b
+    float2 *red2 = reinterpret_cast<float2 *>(red + 2 * nw);               // [2][nw] (x - mu)^2 sums of a, b
+    const int64_t smp = blockIdx.x / cps;
+    const int part = int(blockIdx.x % cps);
+    const int64_t r0 = smp * rows_per + rows_per * part / cps;
+    const int64_t r1 = smp * rows_per + rows_per * (part + 1) / cps;
+    const int d = nb * kBlk;
+    const bool active = t < nb;
+    const int j = active ? t : 0;
+
+    // this thread's copies of row r into ring slot `slot` (16-byte pieces, swizzled)
+    const uint32_t rbase = static_cast<uint32_t>(__cvta_generic_to_shared(ring)) + uint32_t(t) * 64;
+    const int sw = (t >> 1) & 3;
+    auto issue = [&](int64_t r, int slot) {
+        if (active && r < r1) {
+            const uint4 *src = h + (r * nb + t) * 4;
+            const uint32_t dst = rbase + uint32_t(slot) * uint32_t(nt) * 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cp_async16(dst + 16 * (q ^ sw), src + q);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // the first rows go out before the set-up
+#pragma unroll
+    for (int k = 0; k < DEPTH; ++k) issue(r0 + k, k);
+
+    ring::Coef st;
+    bool fast = true;
+    {
+        float4 g[5];
+        load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
+        fast = ring::coef_setup(g, st);
+        const float4 *gp = reinterpret_cast<const float4 *>(gamma + smp * d + int64_t(j) * kBlk);
+        const float4 *bp = reinterpret_cast<const float4 *>(beta + smp * d + int64_t(j) * kBlk);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 ga = active ? __ldg(gp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            gtab[q * nt + t] = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
+            btab[q * nt + t] = active ? __ldg(bp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    int step = 0;
+    for (int64_t ra = r0; ra < r1; ra += 2, ++step) {
+        const int64_t rb = ra + 1;
+        const bool two = rb < r1;
+        const int sa = int((ra - r0) % DEPTH), sb = sa + 1;
+        // rows ra and rb have landed (DEPTH - 2 younger groups may be in flight)
+        asm volatile("cp.async.wait_group %0;" ::"n"(DEPTH - 2) : "memory");
+        uint4 xa[4], xb[4];
+        const uint4 *pa = ring + size_t(sa) * nt * 4 + size_t(t) * 4;
+        const uint4 *pb = ring + size_t(sb) * nt * 4 + size_t(t) * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            xa[q] = active ? pa[q ^ sw] : make_uint4(0u, 0u, 0u, 0u);
+            xb[q] = (active && two) ? pb[q ^ sw] : make_uint4(0u, 0u, 0u, 0u);
+        }
+        // the slots are read: refill them with the rows DEPTH ahead
+        issue(ra + DEPTH, sa);
+        issue(rb + DEPTH, sb);
+        float2 p[32];
+        ring::unpack_rows(xa, xb, p);
+        // ---- statistics of both rows (one sweep of sums; the two-pass variance
+        // where the mean is large against the root mean square, as the row kernel)
+        // four partial sums each, so the additions are four short chains
+        float2 sa4[4], qa4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            sa4[k] = p[k];
+            qa4[k] = __fmul2_rn(p[k], p[k]);
+        }
+#pragma unroll
+        for (int k = 4; k < 32; ++k) {
+            sa4[k & 3] = __fadd2_rn(sa4[k & 3], p[k]);
+            qa4[k & 3] = __ffma2_rn(p[k], p[k], qa4[k & 3]);
+        }
+        float2 s2 = __fadd2_rn(__fadd2_rn(sa4[0], sa4[1]), __fadd2_rn(sa4[2], sa4[3]));
+        float2 q2 = __fadd2_rn(__fadd2_rn(qa4[0], qa4[1]), __fadd2_rn(qa4[2], qa4[3]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            s2.x += __shfl_xor_sync(0xffffffffu, s2.x, off);
+            s2.y += __shfl_xor_sync(0xffffffffu, s2.y, off);
+            q2.x += __shfl_xor_sync(0xffffffffu, q2.x, off);
+            q2.y += __shfl_xor_sync(0xffffffffu, q2.y, off);
+        }
+        const int par = step & 1;
+        if (lane == 0) red[par * nw + wid] = make_float4(s2.x, s2.y, q2.x, q2.y);
+        __syncthreads();
+        float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < nw; ++w) {
+            const float4 v = red[par * nw + w];
+            tot.x += v.x;
+            tot.y += v.y;
+            tot.z += v.z;
+            tot.w += v.w;
+        }
+        const float2 mu = make_float2(tot.x / float(d), tot.y / float(d));
+        const float2 ex2 = make_float2(tot.z / float(d), tot.w / float(d));
+        const float2 nmu = make_float2(-mu.x, -mu.y);
+        float2 m2;
+        // uniform over the CTA: the same totals everywhere
+        if (mu.x * mu.x <= ex2.x * (1.0f / 64.0f) && mu.y * mu.y <= ex2.y * (1.0f / 64.0f)) {
+            m2 = make_float2(fmaxf(ex2.x - mu.x * mu.x, 0.0f) * float(d), fmaxf(ex2.y - mu.y * mu.y, 0.0f) * float(d));
+        } else {
+            float2 c2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float2 tt = __fadd2_rn(p[k], nmu);
+                c2 = __ffma2_rn(tt, tt, c2);
+            }
+            if (!active) c2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                c2.x += __shfl_xor_sync(0xffffffffu, c2.x, off);
+                c2.y += __shfl_xor_sync(0xffffffffu, c2.y, off);
+            }
+            if (lane == 0) red2[par * nw + wid] = c2;
+            __syncthreads();
+            float2 two_pass = make_float2(0.f, 0.f);
+            for (int w = 0; w < nw; ++w) {
+                const float2 v = red2[par * nw + w];
+                two_pass.x += v.x;
+                two_pass.y += v.y;
+            }
+            // each row keeps the one-sweep value where its own mean allows it
+            m2.x = mu.x * mu.x <= ex2.x * (1.0f / 64.0f) ? fmaxf(ex2.x - mu.x * mu.x, 0.0f) * float(d) : two_pass.x;
+            m2.y = mu.y * mu.y <= ex2.y * (1.0f / 64.0f) ? fmaxf(ex2.y - mu.y * mu.y, 0.0f) * float(d) : two_pass.y;
+        }
+        if (!active) continue;
+        const float2 iv = make_float2(1.0f / sqrtf(m2.x / float(d) + eps), 1.0f / sqrtf(m2.y / float(d) + eps));
+        // ---- normalise, modulate (both rows): x / sigma - mu / sigma as one
+        // FMA (the product x / sigma is exact inside it, so the result differs
+        // from (x - mu) / sigma by one rounding of mu / sigma), then times
+        // 1 + gamma plus beta; transform, quantize
+        const float2 off = make_float2(-mu.x * iv.x, -mu.y * iv.y);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 ga = gtab[q * nt + t], ba = btab[q * nt + t];
+            const float gg[4] = {ga.x, ga.y, ga.z, ga.w}, bb[4] = {ba.x, ba.y, ba.z, ba.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * q + e;
+                const float2 tt = __ffma2_rn(p[i], iv, off);
+                p[i] = __ffma2_rn(tt, make_float2(gg[e], gg[e]), make_float2(bb[e], bb[e]));
+            }
+        }
+        if (fast) {
+            ring::fast_apply(p, st);
+        } else {   // rare: the raw factors, from L1
+            float4 g[5];
+            load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
+            ring::direct_apply(p, g);
+        }
+        float a0, a1;
+        ring::amax_rows(p, a0, a1);
+        uint4 c0, c1;
+        uint32_t b0, b1;
+        ring::finish_rows(p, a0, a1, c0, c1, b0, b1);
+        if (!(a0 <= 3.40282347e38f)) {
+            c0 = make_uint4(0u, 0u, 0u, 0u);
+            b0 = 0xFFu;
+        }
+        if (!(a1 <= 3.40282347e38f)) {
+            c1 = make_uint4(0u, 0u, 0u, 0u);
+            b1 = 0xFFu;
+        }
+        norm_store<SF>(c0, b0, ra, t, nb, codes, scales);
+        if (two) norm_store<SF>(c1, b1, rb, t, nb, codes, scales);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // launch geometry
 // ---------------------------------------------------------------------------
@@ -2095,10 +2317,45 @@ int gemm_launch(const GemmArgs &g)
     return g.f32 ? gemm_launch_out<C, true>(g, amap, bmap, omap, grid) : gemm_launch_out<C, false>(g, amap, bmap, omap, grid);
 }
 
+// Shared memory of the long-row kernel: the (1 + gamma, beta) table, the
+// row ring and the reduction arrays.
+size_t cols_smem(int nt, int depth) { return size_t(16) * nt * 16 + size_t(depth) * nt * 64 + size_t(nt / 32) * 48; }
+
+template <bool SF, int DEPTH, int MAXT>
+int cols_launch(const char *fn, const void *h_bf16, const float *gamma, const float *beta, int64_t nsamples,
+                float eps, const float *factors, int shared, uint8_t *out_codes, uint8_t *out_scales, int64_t M,
+                int nb, int sms, cudaStream_t stream)
+{
+    const int nt = (nb + 31) / 32 * 32;
+    const size_t smem = cols_smem(nt, DEPTH);
+    auto k = norm_kq_cols_kernel<SF, DEPTH, MAXT>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, nt, smem);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+    if (per_sm < 1) return fail(KQ_ERR_CUDA, "%s: the long-row kernel does not fit on this device", fn);
+    const int64_t rows_per = M / nsamples;
+    int64_t cps = int64_t(sms) * per_sm / nsamples;
+    if (cps > rows_per) cps = rows_per;
+    if (cps < 1) cps = 1;
+    if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
+    k<<<unsigned(cps * nsamples), nt, smem, stream>>>(static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps,
+                                                      factors, shared ? 1 : 0, reinterpret_cast<uint4 *>(out_codes),
+                                                      out_scales, nb, int(cps));
+    return launch_check(fn);
+}
+
+// Kernels of the fused normalisation: 1 = the single-pass row kernel (where
+// a configuration fits), 2 = the warp-per-row kernel that re-reads the row,
+// 3 = the long-row kernel; 0 = the default: 3 from kColsMinBlocks block
+// columns up (d >= 6144), else 1 where it fits, else 2.
+constexpr int kColsMinBlocks = 192;
+
 template <bool SF>
 int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const float *beta, int64_t nsamples, float eps,
                 const float *factors, int shared, uint8_t *out_codes, uint8_t *out_scales, int64_t M, int64_t d,
-                cudaStream_t stream)
+                cudaStream_t stream, int variant = 0)
 {
     if (M < 0 || d <= 0 || d % kBlk != 0 || d / kBlk > 512)
         return fail(KQ_ERR_SHAPE, "%s: need M >= 0 and d a positive multiple of 32, at most 16384 (M=%lld, d=%lld)",
@@ -2114,11 +2371,23 @@ int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const fl
     if (!aligned(h_bf16, 16) || !aligned(out_codes, 16) || !aligned(factors, 16) || !aligned(gamma, 16) ||
         !aligned(beta, 16))
         return fail(KQ_ERR_ALIGN, "%s: h, out_codes, factors, gamma and beta must be 16-byte aligned", fn);
+    if (variant < 0 || variant > 3)
+        return fail(KQ_ERR_VARIANT, "%s: variant %d is not available in this build", fn, variant);
     const int nb = int(d / kBlk);
     int sms = 0;
     int rc = sm_count(&sms);
     if (rc != KQ_OK) return rc;
-    {
+    if (variant == 0) variant = nb >= kColsMinBlocks ? 3 : 1;
+    if (variant == 3) {
+        // up to 384 threads (d <= 12288): a 4-row ring (two pairs) and up to 168
+        // registers; wider rows: 512 threads, a 2-row ring, 128 registers
+        if (nb <= 384)
+            return cols_launch<SF, 4, 384>(fn, h_bf16, gamma, beta, nsamples, eps, factors, shared, out_codes,
+                                           out_scales, M, nb, sms, stream);
+        return cols_launch<SF, 2, 512>(fn, h_bf16, gamma, beta, nsamples, eps, factors, shared, out_codes, out_scales,
+                                       M, nb, sms, stream);
+    }
+    if (variant == 1) {
         // single-pass kernel: the first (warps, row buffers) whose shared memory
         // fits, chosen once per device and row width (cached: warps << 8 | nbuf
         // << 4 | CTAs per SM; -1 = none fits)
@@ -2416,6 +2685,14 @@ int norm_kq_quantize_sf(const void *h_bf16, const float *gamma, const float *bet
 {
     return norm_launch<true>("norm_kq_quantize_sf", h_bf16, gamma, beta, nsamples, eps, factors, shared, out_codes,
                              out_sf, M, d, stream);
+}
+
+int norm_kq_quantize_variant(int variant, const void *h_bf16, const float *gamma, const float *beta,
+                             int64_t nsamples, float eps, const float *factors, int shared, uint8_t *out_codes,
+                             uint8_t *out_scales, int64_t M, int64_t d, cudaStream_t stream)
+{
+    return norm_launch<false>("norm_kq_quantize_variant", h_bf16, gamma, beta, nsamples, eps, factors, shared,
+                              out_codes, out_scales, M, d, stream, variant);
 }
 
 int64_t kq_sf_bytes(int64_t rows, int64_t d)
