@@ -145,3 +145,42 @@ def check_exact(codes_gpu, scales_gpu, codes_ref, scales_ref):
     }
     res["ok"] = res["scale_mismatch"] == 0 and res["code_byte_mismatch"] == 0
     return res
+
+
+# -- the W4A4 product ---------------------------------------------------------------
+# Each product of two MXFP4 values is exact (two significant bits times a power
+# of two), so the product differs from the oracle's double sum only by the fp32
+# accumulation: per element at most K * 2^-23 * sum_k |a_k b_k| (any order,
+# truncating adds included), plus bf16's rounding of the output (2^-8 of the
+# value).  That worst case grows with K; accumulation errors of random sign
+# grow with sqrt(K), so the fp32 results must also meet a statistical bound:
+# the root mean square over all elements of err / sum_k |a_k b_k| at most
+# GEMM_RMS_FACTOR * sqrt(K) * 2^-24.  A systematic mistake that the per-element
+# bound could miss (a dropped or repeated K-block, whose contribution is a
+# near-cancelling partial sum) moves this statistic by orders of magnitude.
+GEMM_RMS_FACTOR = 8.0
+
+
+def gemm_bound(K, D, absd, bf16_out):
+    acc = K * 2.0 ** -23 * absd
+    return acc + (2.0 ** -8 * (np.abs(D) + acc) if bf16_out else 0.0)
+
+
+def check_gemm(Dg, D, absd, K, bf16_out):
+    """Per-element worst-case bound; for fp32 output also the rms statistic.
+
+    Returns {"bad": elements over the bound, "worst": max err / bound,
+    "rms_rel": rms of err / absd (fp32 only), "rms_bound": its bound, "ok"}."""
+    err = np.abs(np.asarray(Dg, np.float64) - D)
+    bound = gemm_bound(K, D, absd, bf16_out)
+    bad = int(np.count_nonzero(err > bound))
+    res = {"bad": bad, "worst": float(np.max(err / np.maximum(bound, 1e-300))) if err.size else 0.0}
+    ok = bad == 0
+    if not bf16_out:
+        nz = absd > 0
+        rel = err[nz] / absd[nz]
+        res["rms_rel"] = float(np.sqrt(np.mean(rel * rel))) if rel.size else 0.0
+        res["rms_bound"] = GEMM_RMS_FACTOR * np.sqrt(K) * 2.0 ** -24
+        ok = ok and res["rms_rel"] <= res["rms_bound"]
+    res["ok"] = ok
+    return res

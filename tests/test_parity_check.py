@@ -128,3 +128,24 @@ def test_unpooled_checks_leave_the_pool_alone():
     c, s, y, ab = data()
     pc.check_kq(c, s, c, s, y, ab, pool=False)
     assert pc.POOL == before
+
+
+def test_gemm_check_rms_statistic_catches_a_dropped_k_block():
+    # exact product rounded to fp32: passes both criteria
+    K = 1152
+    ca, sa = synth.mx_operand(64, K, 5)
+    cb, sb = synth.mx_operand(48, K, 6)
+    D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+    ok = pc.check_gemm(D.astype(np.float32), D, absd, K, False)
+    assert ok["ok"] and ok["rms_rel"] < ok["rms_bound"] / 10
+    # the last 64-element K step left out of every output: the statistic,
+    # taken over all outputs, is far above its bound
+    ca2 = ca.copy()
+    ca2[:, -32:] = 0
+    r = pc.check_gemm(oracle.mxf4_gemm(ca2, sa, cb, sb), D, absd, K, False)
+    assert not r["ok"] and r["rms_rel"] > 100 * r["rms_bound"]
+    # an error of a few hundred fp32 roundings per output, everywhere: within
+    # the worst-case K * 2^-23 bound but not the sqrt(K) statistic
+    noisy = D + 300 * 2.0 ** -24 * absd * np.where(np.arange(D.size).reshape(D.shape) % 2, 1, -1)
+    r2 = pc.check_gemm(noisy, D, absd, K, False)
+    assert r2["bad"] == 0 and not r2["ok"]
