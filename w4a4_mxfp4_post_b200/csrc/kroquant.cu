@@ -1598,9 +1598,10 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 // per warp a shuffle reduction of both rows' sums, per CTA the warps' partial
 // sums in a shared array double-buffered by step parity, so one barrier per
 // two rows suffices (a second one only on the two-pass branch).  Per element:
-// x / sigma - mu / sigma (one FMA), times 1 + gamma plus beta, the unit-
-// diagonal transform, MXFP4 -- the other two kernels' arithmetic except that
-// the normalisation is one FMA instead of a subtraction and a product.
+// x / sigma - mu / sigma (one FMA), times D (1 + gamma) plus D beta (one FMA:
+// the transform's diagonal folded into the modulation), the five unit stages
+// of K = U' D, MXFP4: seven FMA-pipe operations from x to y, where the
+// other two kernels take nine.
 template <bool SF>
 __device__ __forceinline__ void norm_store(uint4 c, uint32_t sb, int64_t r, int j, int nb, uint4 *__restrict__ codes,
                                            uint8_t *__restrict__ scales)
@@ -1636,6 +1637,7 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
     const int64_t r0 = smp * rows_per + rows_per * part / cps;
     const int64_t r1 = smp * rows_per + rows_per * (part + 1) / cps;
     const int d = nb * kBlk;
+    const float inv_d = 1.0f / float(d);
     const bool active = t < nb;
     const int j = active ? t : 0;
 
@@ -1655,19 +1657,57 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 #pragma unroll
     for (int k = 0; k < DEPTH; ++k) issue(r0 + k, k);
 
-    ring::Coef st;
+    // The transform in the form K = U' D: each factor G = [[1, g01 / g11], [g10 /
+    // g00, 1]] diag(g00, g11), so the diagonal D (the same as in K = D U) acts
+    // first and folds into the modulation: x'' = t (D (1 + gamma)) + D beta,
+    // then the five unit stages of U' -- no D multiply per element.  The table
+    // holds D (1 + gamma) and D beta + 0 (+0 for a zero product, so no
+    // intermediate is ever -0 and an exactly cancelling sum comes out +0).
+    // A column whose factors the split does not admit keeps 1 + gamma and beta
+    // in the table and runs the direct form.
+    float B[5], C[5];
     bool fast = true;
+    const float *gsm = gamma + smp * d + int64_t(j) * kBlk;
+    const float *bsm = beta + smp * d + int64_t(j) * kBlk;
     {
         float4 g[5];
         load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
-        fast = ring::coef_setup(g, st);
-        const float4 *gp = reinterpret_cast<const float4 *>(gamma + smp * d + int64_t(j) * kBlk);
-        const float4 *bp = reinterpret_cast<const float4 *>(beta + smp * d + int64_t(j) * kBlk);
+        float d0[5], d1[5];
+#pragma unroll
+        for (int k = 0; k < 5; ++k) {
+            d0[k] = g[k].x;
+            d1[k] = g[k].w;
+            const float bk = __fdividef(g[k].y, g[k].w), ck = __fdividef(g[k].z, g[k].x);
+            const float a0 = fabsf(d0[k]), a1 = fabsf(d1[k]);
+            fast &= a0 >= 0x1p-16f && a0 <= 0x1p16f && a1 >= 0x1p-16f && a1 <= 0x1p16f && fabsf(bk) <= 16.0f &&
+                    fabsf(ck) <= 16.0f;
+            B[4 - k] = bk;           // factor k (G_{k+1}) acts on in-block index bit 4 - k
+            C[4 - k] = ck;
+        }
+        float dd[32];
+        dd[0] = 1.0f;
+#pragma unroll
+        for (int bit = 0; bit < 5; ++bit) {
+            const int k = 4 - bit;
+#pragma unroll
+            for (int i = 0; i < (1 << bit); ++i) {
+                dd[i + (1 << bit)] = dd[i] * d1[k];
+                dd[i] = dd[i] * d0[k];
+            }
+        }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const float4 ga = active ? __ldg(gp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            gtab[q * nt + t] = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
-            btab[q * nt + t] = active ? __ldg(bp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 ga = active ? __ldg(reinterpret_cast<const float4 *>(gsm) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 ba = active ? __ldg(reinterpret_cast<const float4 *>(bsm) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 gg = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
+            float4 bb = ba;
+            if (fast) {
+                gg = make_float4(dd[4 * q] * gg.x, dd[4 * q + 1] * gg.y, dd[4 * q + 2] * gg.z, dd[4 * q + 3] * gg.w);
+                bb = make_float4(fmaf(dd[4 * q], bb.x, 0.0f), fmaf(dd[4 * q + 1], bb.y, 0.0f),
+                                 fmaf(dd[4 * q + 2], bb.z, 0.0f), fmaf(dd[4 * q + 3], bb.w, 0.0f));
+            }
+            gtab[q * nt + t] = gg;
+            btab[q * nt + t] = bb;
         }
     }
 
@@ -1725,8 +1765,8 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
             tot.z += v.z;
             tot.w += v.w;
         }
-        const float2 mu = make_float2(tot.x / float(d), tot.y / float(d));
-        const float2 ex2 = make_float2(tot.z / float(d), tot.w / float(d));
+        const float2 mu = make_float2(tot.x * inv_d, tot.y * inv_d);
+        const float2 ex2 = make_float2(tot.z * inv_d, tot.w * inv_d);
         const float2 nmu = make_float2(-mu.x, -mu.y);
         float2 m2;
         // uniform over the CTA: the same totals everywhere
@@ -1758,7 +1798,7 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
             m2.y = mu.y * mu.y <= ex2.y * (1.0f / 64.0f) ? fmaxf(ex2.y - mu.y * mu.y, 0.0f) * float(d) : two_pass.y;
         }
         if (!active) continue;
-        const float2 iv = make_float2(1.0f / sqrtf(m2.x / float(d) + eps), 1.0f / sqrtf(m2.y / float(d) + eps));
+        const float2 iv = make_float2(__frsqrt_rn(fmaf(m2.x, inv_d, eps)), __frsqrt_rn(fmaf(m2.y, inv_d, eps)));
         // ---- normalise, modulate (both rows): x / sigma - mu / sigma as one
         // FMA (the product x / sigma is exact inside it, so the result differs
         // from (x - mu) / sigma by one rounding of mu / sigma), then times
@@ -1776,7 +1816,11 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
             }
         }
         if (fast) {
-            ring::fast_apply(p, st);
+            ring::unit_stage<1>(p, B[0], C[0]);
+            ring::unit_stage<2>(p, B[1], C[1]);
+            ring::unit_stage<4>(p, B[2], C[2]);
+            ring::unit_stage<8>(p, B[3], C[3]);
+            ring::unit_stage<16>(p, B[4], C[4]);
         } else {   // rare: the raw factors, from L1
             float4 g[5];
             load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
