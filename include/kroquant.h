@@ -244,14 +244,19 @@ int mxf4_gemm(const uint8_t *a_codes, const uint8_t *a_sf,
 /* Test export: mxf4_gemm through a chosen tile configuration (128 x 256
  * output tiles unless stated, one CTA per SM; a k-chunk is CB bytes of codes
  * per row):
- *   0  the default (what mxf4_gemm runs: 4, or 6 where 256-column tiles
- *      fill the last wave of SMs badly),
+ *   0  the default (what mxf4_gemm runs): above 128 rows 7, or 8 where
+ *      256-column tiles fill the last wave of SM pairs badly; up to 128 rows
+ *      4, or 6 where 256-column tiles fill the last wave of SMs badly,
  *   1  CB = 128, 4 stages, epilogue stores from registers,
  *   2  CB = 64, 6 stages, bf16 epilogue through shared memory and TMA stores,
  *   3  CB = 64, 4 stages, TMA stores,
  *   4  CB = 128, 3 stages, TMA stores,
  *   5  CB = 64, 8 stages, stores from registers,
- *   6  as 4 with 192-column tiles.
+ *   6  as 4 with 192-column tiles,
+ *   7  SM pairs: clusters of two CTAs on two SMs, 256 x 256 tiles, one
+ *      M256 MMA (tcgen05 .cta_group::2) per K step for both SMs, CB = 128,
+ *      4 stages, TMA stores,
+ *   8  as 7 with 256 x 192 tiles and two accumulators.
  * Same results for every configuration (the K order of the MMAs is the same).
  * Other values return KQ_ERR_VARIANT. */
 int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf,

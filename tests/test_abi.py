@@ -194,6 +194,9 @@ def test_w4a4_argument_errors(L):
     assert L.mxf4_gemm(P(16), P(16), P(16), P(16), P(4), 1, 4, 8, 64, None) == -3
     assert L.mxf4_gemm(None, None, None, None, None, 0, 0, 8, 64, None) == 0
     assert L.mxf4_gemm(None, None, None, None, None, 0, 4, 0, 64, None) == 0
+    # tile configurations 0-8 exist; others are a variant error (checked before any launch)
+    assert L.mxf4_gemm_variant(9, P(16), P(16), P(16), P(16), P(16), 0, 4, 8, 64, None) == -5
+    assert L.mxf4_gemm_variant(-1, P(16), P(16), P(16), P(16), P(16), 0, 4, 8, 64, None) == -5
     # norm_kq_quantize_sf: h, gamma, beta, nsamples, eps, factors, shared, codes, sf, M, d, stream
     f = ctypes.c_float
     assert L.norm_kq_quantize_sf(P(16), P(16), P(16), 2, f(1e-6), P(16), 0, P(16), P(16), 5, 64, None) == -2

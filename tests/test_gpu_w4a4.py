@@ -124,6 +124,31 @@ def test_mxf4_gemm_random_operands(cuda_device, M, N, K, f32):
     assert kq.kq_wait_timeouts() == 0
 
 
+# The SM-pair forms (cta_group::2): 256 x 256 and 256 x 192 tiles.  Cases add
+# to the above: more tiles than SM pairs (every pair walks several tiles, both
+# accumulators cycle), a 256-row tile whose second CTA is past M, 192-column
+# tiles starting in the middle of a scale unit, K of one chunk and ragged K.
+PAIR_FORMS = (7, 8)
+PAIR_CASES = GEMM_CASES + [(2100, 3000, 192), (520, 1160, 640), (4096, 4608, 128)]
+
+
+@pytest.mark.parametrize("variant", PAIR_FORMS)
+@pytest.mark.parametrize("M,N,K", PAIR_CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}" for c in PAIR_CASES])
+@pytest.mark.parametrize("f32", [True, False], ids=["f32", "bf16"])
+def test_mxf4_gemm_sm_pair_forms(cuda_device, M, N, K, f32, variant):
+    import torch
+
+    ca, sa = synth.mx_operand(M, K, 23)
+    cb, sb = synth.mx_operand(N, K, 24)
+    D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+    kq.kq_wait_timeouts(reset=True)
+    out = kq.mxf4_gemm_variant(variant, dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device),
+                               dev(cb, cuda_device), dev(oracle.scales_to_sf(sb), cuda_device),
+                               out_dtype=torch.float32 if f32 else torch.bfloat16)
+    assert kq.kq_wait_timeouts() == 0
+    check_gemm(out.float().cpu().numpy(), D, absd, K, not f32)
+
+
 @pytest.mark.parametrize("M,N,K", [(300, 520, 1152), (77, 136, 5600), (256, 264, 96)])
 def test_mxf4_gemm_configurations_agree(cuda_device, M, N, K):
     """Every tile configuration gives the same bits (same K order), and the
@@ -138,7 +163,7 @@ def test_mxf4_gemm_configurations_agree(cuda_device, M, N, K):
     for dtype in (torch.float32, torch.bfloat16):
         ref = kq.mxf4_gemm_variant(1, *args, out_dtype=dtype)
         check_gemm(ref.float().cpu().numpy(), D, absd, K, dtype == torch.bfloat16)
-        for v in (0, 2, 3, 4, 5, 6):
+        for v in (0, 2, 3, 4, 5, 6) + PAIR_FORMS:
             got = kq.mxf4_gemm_variant(v, *args, out_dtype=dtype)
             assert torch.equal(got, ref), (v, dtype)
 
@@ -196,8 +221,9 @@ def test_w4a4_chain_on_oracle_operands(cuda_device):
     assert rel["unfolded"] > 0.9 and rel["hadamard"] < 0.5 * rel["unfolded"], rel
 
 
+@pytest.mark.parametrize("variant", (0,) + PAIR_FORMS)
 @pytest.mark.parametrize("N,K", synth.GEMM_LAYERS["pixart_mlp"]["layers"])
-def test_mxf4_gemm_full_size_sampled_rows(cuda_device, N, K):
+def test_mxf4_gemm_full_size_sampled_rows(cuda_device, N, K, variant):
     """The benchmark's launch (8192 tokens, PixArt-Sigma MLP layer), checked on
     sampled rows: head, tail and random rows of every row tile class."""
     import torch
@@ -205,8 +231,8 @@ def test_mxf4_gemm_full_size_sampled_rows(cuda_device, N, K):
     M = synth.GEMM_LAYERS["pixart_mlp"]["M"]
     ca, sa = synth.mx_operand(M, K, 41)
     cb, sb = synth.mx_operand(N, K, 42)
-    out = kq.mxf4_gemm(dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
-                       dev(oracle.scales_to_sf(sb), cuda_device))
+    out = kq.mxf4_gemm_variant(variant, dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device),
+                               dev(cb, cuda_device), dev(oracle.scales_to_sf(sb), cuda_device))
     rng = np.random.default_rng(N + K)
     rows = np.unique(np.concatenate([np.arange(8), np.arange(M - 8, M), rng.choice(M, 24, replace=False)]))
     D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, rows=rows, want_absbound=True)
@@ -214,7 +240,8 @@ def test_mxf4_gemm_full_size_sampled_rows(cuda_device, N, K):
     check_gemm(got, D, absd, K, True)
 
 
-def test_mxf4_gemm_extreme_scale_exponents(cuda_device):
+@pytest.mark.parametrize("variant", (0, 7))
+def test_mxf4_gemm_extreme_scale_exponents(cuda_device, variant):
     """Scale bytes at both ends of E8M0: A at 2^127 (0xFE) and 2^126, B at
     2^-127 (0x00) and 2^-126, so every product is of order one; the tensor
     core must apply both exponents exactly (oracle bound as above)."""
@@ -227,13 +254,14 @@ def test_mxf4_gemm_extreme_scale_exponents(cuda_device):
     sa = rng.choice(np.array([0xFE, 0xFD], np.uint8), size=(M, K // 32))
     sb = rng.choice(np.array([0x00, 0x01], np.uint8), size=(N, K // 32))
     D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
-    out = kq.mxf4_gemm(dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
-                       dev(oracle.scales_to_sf(sb), cuda_device), out_dtype=torch.float32)
+    out = kq.mxf4_gemm_variant(variant, dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device),
+                               dev(cb, cuda_device), dev(oracle.scales_to_sf(sb), cuda_device), out_dtype=torch.float32)
     assert np.all(np.isfinite(D))
     check_gemm(out.cpu().numpy(), D, absd, K, False)
 
 
-def test_mxf4_gemm_nan_scale_reaches_only_its_row(cuda_device):
+@pytest.mark.parametrize("variant", (0, 7))
+def test_mxf4_gemm_nan_scale_reaches_only_its_row(cuda_device, variant):
     """A scale byte 0xFF (E8M0 NaN) in one row of A makes exactly that output
     row NaN (the header's stated behaviour); every other row is unaffected."""
     import torch
@@ -244,8 +272,9 @@ def test_mxf4_gemm_nan_scale_reaches_only_its_row(cuda_device):
     sa = sa.copy()
     sa[5, 3] = 0xFF
     D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
-    out = kq.mxf4_gemm(dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device), dev(cb, cuda_device),
-                       dev(oracle.scales_to_sf(sb), cuda_device), out_dtype=torch.float32).cpu().numpy()
+    out = kq.mxf4_gemm_variant(variant, dev(ca, cuda_device), dev(oracle.scales_to_sf(sa), cuda_device),
+                               dev(cb, cuda_device), dev(oracle.scales_to_sf(sb), cuda_device),
+                               out_dtype=torch.float32).cpu().numpy()
     assert np.all(np.isnan(out[5])) and np.all(np.isnan(D[5]))
     keep = np.arange(M) != 5
     assert np.all(np.isfinite(out[keep]))

@@ -2142,6 +2142,28 @@ int encode_gemm_out_map(void *out, int64_t M, int64_t N, int box_cols, CUtensorM
     return KQ_OK;
 }
 
+// The scale units of an MXFP4 matrix in the scale-factor layout (row group
+// g's units contiguous, 512 bytes each) as a 3-D uint8 tensor {256 bytes,
+// 2 Ka half-units, row groups}; boxes of {256, 4, groups}: the two units of a
+// 256-element k-chunk for `groups` consecutive row groups.  Units past K and
+// row groups past the matrix read as zero.
+int encode_sf_map(const void *sf, int64_t rows, int64_t K, int groups, CUtensorMap *map)
+{
+    EncodeTiledFn enc;
+    int rc = encode_fn(&enc);
+    if (rc != KQ_OK) return rc;
+    const int64_t Ka = (K + 127) / 128;
+    const cuuint64_t dims[3] = {256, cuuint64_t(2 * Ka), cuuint64_t((rows + 127) / 128)};
+    const cuuint64_t strides[2] = {256, cuuint64_t(Ka) * 512};
+    const cuuint32_t box[3] = {256, 4, cuuint32_t(groups)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(sf), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", int(r));
+    return KQ_OK;
+}
+
 int64_t sf_bytes_of(int64_t rows, int64_t nb) { return ((rows + 127) / 128) * ((nb + 3) / 4) * 512; }
 
 // Default clock budget of a bounded wait: 2^31 cycles, about a second.
@@ -2308,11 +2330,21 @@ struct GemmArgs {
     cudaStream_t stream;
 };
 
-// Default tile configuration: 4 (256-column tiles) or 6 (192-column tiles),
-// whichever the cost model waves x (128 + BN) -- rounds of one tile per SM,
-// each moving A and B rows -- rates cheaper.
+// Default tile configuration.  Above 128 rows, the SM-pair form: 7 (256 x 256
+// tiles) or 8 (256 x 192 tiles), whichever the cost model waves x BN -- rounds
+// of one tile per SM pair, each as long as its MMAs -- rates cheaper.  Up to
+// 128 rows a pair tile would leave one SM of the pair idle: 4 (256-column
+// tiles) or 6 (192-column tiles), whichever waves x (128 + BN) -- rounds of
+// one tile per SM, each moving A and B rows -- rates cheaper.
 int default_gemm_variant(int64_t M, int64_t N, int sms)
 {
+    if (M > gemm::kBM) {
+        const int64_t pairs = sms / 2 > 0 ? sms / 2 : 1;
+        const int64_t mt2 = (M + 2 * gemm::kBM - 1) / (2 * gemm::kBM);
+        const int64_t p256 = (mt2 * ((N + 255) / 256) + pairs - 1) / pairs;
+        const int64_t p192 = (mt2 * ((N + 191) / 192) + pairs - 1) / pairs;
+        return p192 * 192 < p256 * 256 ? 8 : 7;
+    }
     const int64_t mt = (M + gemm::kBM - 1) / gemm::kBM;
     const int64_t w256 = (mt * ((N + 255) / 256) + sms - 1) / sms;
     const int64_t w192 = (mt * ((N + 191) / 192) + sms - 1) / sms;
@@ -2359,6 +2391,67 @@ int gemm_launch(const GemmArgs &g)
     if ((rc = sm_count(&sms)) != KQ_OK) return rc;
     const unsigned grid = unsigned(tiles < sms ? tiles : sms);
     return g.f32 ? gemm_launch_out<C, true>(g, amap, bmap, omap, grid) : gemm_launch_out<C, false>(g, amap, bmap, omap, grid);
+}
+
+// The SM-pair form: clusters of two CTAs, as many as fit at once (one CTA
+// per SM), each walking 256 x BN tiles.
+template <class C, bool F32>
+std::atomic<int> g_pair_clusters[kMaxDevices];
+
+template <class C, bool F32>
+int gemm_pair_launch_out(const GemmArgs &g, const CUtensorMap *maps, int64_t tiles)
+{
+    auto k = gemm::mxf4_gemm_pair_kernel<C, F32>;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    int clusters = (dev >= 0 && dev < kMaxDevices) ? g_pair_clusters<C, F32>[dev].load(std::memory_order_acquire) : 0;
+    if (clusters <= 0) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem));
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        int sms = 0;
+        int rc = sm_count(&sms);
+        if (rc != KQ_OK) return rc;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(unsigned(sms / 2 * 2), 1, 1);
+        cfg.blockDim = dim3(gemm::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = C::kSmem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&clusters, k, &cfg);
+        if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cluster occupancy query: %s", cudaGetErrorString(e));
+        if (clusters <= 0) return fail(KQ_ERR_CUDA, "mxf4_gemm: no SM pair can hold the kernel");
+        if (dev >= 0 && dev < kMaxDevices) g_pair_clusters<C, F32>[dev].store(clusters, std::memory_order_release);
+    }
+    const unsigned grid = 2u * unsigned(tiles < clusters ? tiles : clusters);
+    k<<<grid, gemm::kThreads, C::kSmem, g.stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], g.out, int(g.M),
+                                                     int(g.N), int(g.K), kWaitBudget);
+    return launch_check("mxf4_gemm");
+}
+
+template <class C>
+int gemm_pair_launch(const GemmArgs &g)
+{
+    const int64_t tiles = ((g.M + 2 * gemm::kBM - 1) / (2 * gemm::kBM)) * ((g.N + C::kBN - 1) / C::kBN);
+    if (tiles >= (int64_t(1) << 31)) return fail(KQ_ERR_SHAPE, "mxf4_gemm: too many output tiles");
+    CUtensorMap maps[5];   // A codes, B codes, A scales, B scales, D
+    int rc = encode_gemm_map(g.a_codes, g.M, g.K, C::kCB, gemm::kBM, &maps[0]);
+    if (rc != KQ_OK) return rc;
+    if ((rc = encode_gemm_map(g.b_codes, g.N, g.K, C::kCB, C::kBRows, &maps[1])) != KQ_OK) return rc;
+    if ((rc = encode_sf_map(g.a_sf, g.M, g.K, 1, &maps[2])) != KQ_OK) return rc;
+    if ((rc = encode_sf_map(g.b_sf, g.N, g.K, 2, &maps[3])) != KQ_OK) return rc;
+    // only the bf16 epilogue reads the output map ({32 x 32} boxes); fp32 gets a placeholder
+    if (!g.f32) {
+        if ((rc = encode_gemm_out_map(g.out, g.M, g.N, 32, &maps[4])) != KQ_OK) return rc;
+    } else {
+        maps[4] = maps[0];
+    }
+    return g.f32 ? gemm_pair_launch_out<C, true>(g, maps, tiles) : gemm_pair_launch_out<C, false>(g, maps, tiles);
 }
 
 // Shared memory of the long-row kernel: the (1 + gamma, beta) table, the
@@ -2811,7 +2904,7 @@ int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf, 
                     "(M=%lld, N=%lld, K=%lld)", fn, (long long)M, (long long)N, (long long)K);
     if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
         return fail(KQ_ERR_SHAPE, "%s: M, N and K must be below 2^31", fn);
-    if (variant < 0 || variant > 6) return fail(KQ_ERR_VARIANT, "%s: variant %d is not available", fn, variant);
+    if (variant < 0 || variant > 8) return fail(KQ_ERR_VARIANT, "%s: variant %d is not available", fn, variant);
     if (M == 0 || N == 0) return ok();
     if (!a_codes || !a_sf || !b_codes || !b_sf || !out) return fail(KQ_ERR_NULL, "%s: NULL pointer argument", fn);
     if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
@@ -2830,7 +2923,9 @@ int mxf4_gemm_variant(int variant, const uint8_t *a_codes, const uint8_t *a_sf, 
     case 3: return gemm_launch<gemm::Cfg3>(g);
     case 4: return gemm_launch<gemm::Cfg4>(g);
     case 5: return gemm_launch<gemm::Cfg5>(g);
-    default: return gemm_launch<gemm::Cfg6>(g);
+    case 6: return gemm_launch<gemm::Cfg6>(g);
+    case 7: return gemm_pair_launch<gemm::Pair7>(g);
+    default: return gemm_pair_launch<gemm::Pair8>(g);
     }
 }
 
