@@ -27,13 +27,13 @@
 //              past the matrix read as zero) and bulk copies of the chunk's
 //              scale units (A: its row group's, B: the tile's two row groups')
 //              into an ST-stage ring
-//   warp 1     allocates tensor memory; one thread issues the chunk's CB / 32
-//              MMAs (only the K=64 steps below K) once the copier has put the
+//   warp 1     allocates tensor memory; the warp (one elected lane) issues the
+//              chunk's CB / 32 MMAs (only the K=64 steps below K) once the copier has put the
 //              stage's scales in tensor memory, and commits the stage back to
 //              the producer; after a tile's last chunk it commits the
 //              accumulator.  Where two accumulators fit beside the scale
 //              columns (BN = 192) tiles alternate between them.
-//   warp 10    the scale copier: one thread copies each landed stage's scale
+//   warp 10    the scale copier: the warp (one elected lane) copies each landed stage's scale
 //              units to that stage's own tensor-memory columns (so a copy
 //              never waits on MMAs still reading an older stage) and commits
 //              them to the stage's `sf_ready` barrier.  A tcgen05 instruction
@@ -113,23 +113,46 @@ struct Cfg {
 // 128-element unit reads blocks 2j and 2j+1, i.e. bytes 2j, 2j+1 (sf_id 2j).
 __device__ __forceinline__ uint32_t idesc(uint32_t base, uint32_t sf_id) { return base | (sf_id << 4) | (sf_id << 29); }
 
+// The MMA and scale-copy warps run their loops with the whole warp, on
+// warp-uniform operands, and each tcgen05 instruction below is issued by the
+// one lane elect.sync picks: the operands then stay in uniform registers, and
+// the issuing thread is not held up moving them there one at a time.
 __device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t id,
                                           uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                 "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
                      tmem_d),
                  "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
                  : "memory");
 }
 
 // One 512-byte scale unit (shared memory, 32 rows x 16 bytes, no swizzle) to
-// 4 tensor-memory columns, replicated to the four 32-lane quarters.
+// 4 tensor-memory columns, replicated to the four 32-lane quarters (whole warp).
 __device__ __forceinline__ void tmem_copy_unit(uint32_t taddr, uint32_t saddr)
 {
     const uint64_t desc = mma::smem_desc(saddr, 128, 0);
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+    asm volatile("{\n\t.reg .pred e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// Arrive (once) on `bar` when the tcgen05 operations issued so far completed (whole warp).
+__device__ __forceinline__ void umma_commit_w(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .pred e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+// A bounded wait taken by the whole warp: true only if every lane saw the phase.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long budget)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, budget));
 }
 
 // Plain (untiled) bulk copy global -> shared, completing on `bar`.
@@ -361,8 +384,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- scale copies and MMAs (one thread)
+        // ---------------- MMAs (the whole warp; one elected lane issues)
+        {
             int k = 0, it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
@@ -370,16 +393,16 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 // scales off = 0 or 2 columns (32-row groups) into the first unit
                 const uint32_t off = uint32_t(((t % NT) * kBN % 128) / 32);
                 const int ab = it % NA;               // accumulator of this tile
-                if (it >= NA && !mbar_wait(&acc_empty[ab], ((it / NA) - 1) & 1, budget)) {
-                    atomicAdd(&g_wait_timeouts, 1);
+                if (it >= NA && !warp_wait(&acc_empty[ab], ((it / NA) - 1) & 1, budget)) {
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
                 mma::tc_fence_after();
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
                     // the stage landed and the copier has put its scale units in tensor memory
-                    if (!mbar_wait(&full[s], (k / ST) & 1, budget) || !mbar_wait(&sf_ready[s], (k / ST) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (!warp_wait(&full[s], (k / ST) & 1, budget) || !warp_wait(&sf_ready[s], (k / ST) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -398,18 +421,18 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                                   (tsf + 16 * u) | (sf_id << 30),
                                   (tsf + 16 * u + 8 + off) | (sf_id << 30), (c | j) != 0);
                     }
-                    mma::umma_commit(&empty[s]);
+                    umma_commit_w(&empty[s]);
                 }
                 if (!ok) break;
-                mma::umma_commit(&acc_full[ab]);
+                umma_commit_w(&acc_full[ab]);
             }
             // every MMA issued has completed before the tensor memory is freed
-            mma::umma_commit(done);
-            if (!mbar_wait(done, 0, budget)) atomicAdd(&g_wait_timeouts, 1);
+            umma_commit_w(done);
+            if (!warp_wait(done, 0, budget) && lane == 0) atomicAdd(&g_wait_timeouts, 1);
         }
     } else if (warp == kCopyWarp) {
-        if (lane == 0) {
-            // ---------------- scale copies (one thread): each stage's units to
+        {
+            // ---------------- scale copies (the whole warp): each stage's units to
             // that stage's own tensor-memory columns, so a copy never waits on
             // MMAs still reading an older stage, and the MMA thread only issues
             // MMAs.  Units past K or of a missing B row group are stale data:
@@ -419,8 +442,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
-                    if (!mbar_wait(&full[s], (k / ST) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (!warp_wait(&full[s], (k / ST) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -434,12 +457,12 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                         tmem_copy_unit(tsf + 16 * u + 8, sfb + u * kSfUnit);
                         tmem_copy_unit(tsf + 16 * u + 12, sfb + (C::kUnits + u) * kSfUnit);
                     }
-                    mma::umma_commit(&sf_ready[s]);
+                    umma_commit_w(&sf_ready[s]);
                     issued = k + 1;
                 }
             }
             // the copies issued have completed before the tensor memory is freed
-            if (issued > 0 && !mbar_wait(&sf_ready[(issued - 1) % ST], ((issued - 1) / ST) & 1, budget))
+            if (issued > 0 && !warp_wait(&sf_ready[(issued - 1) % ST], ((issued - 1) / ST) & 1, budget) && lane == 0)
                 atomicAdd(&g_wait_timeouts, 1);
         }
     } else {
@@ -492,7 +515,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
 //              row groups} (units past K or row groups past the matrix read
 //              as zero)
 //   warp 1     allocates the pair's tensor memory (.cta_group::2, both CTAs);
-//              in the leader one thread issues the MMAs and commits each stage
+//              in the leader the warp (one elected lane) issues the MMAs and commits each stage
 //              to the `empty` barrier of both CTAs and each finished tile to
 //              the `acc_full` barrier of both
 //   warp 10    in the leader, the scale copier: each stage's scale units into
@@ -606,9 +629,10 @@ __device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *m
 __device__ __forceinline__ void umma_mxf4_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t id,
                                                uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                 "@e tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
                      tmem_d),
                  "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
                  : "memory");
@@ -620,14 +644,19 @@ __device__ __forceinline__ void umma_mxf4_pair(uint32_t tmem_d, uint64_t adesc, 
 __device__ __forceinline__ void tmem_copy_unit_pair(uint32_t taddr, uint32_t saddr)
 {
     const uint64_t desc = mma::smem_desc(saddr, 128, 0);
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+    asm volatile("{\n\t.reg .pred e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 // Arrive on `bar` (shared::cluster, either CTA) when every tcgen05 operation
 // this thread issued so far has completed on both SMs.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar)
 {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+    asm volatile("{\n\t.reg .pred e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+                 : "memory");
 }
 
 template <class C, bool F32OUT>
@@ -735,8 +764,8 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                 }
         }
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
-            // ---------------- scale copies and MMAs (the leader's one thread)
+        if (rank == 0) {
+            // ---------------- MMAs (the leader's warp; one elected lane issues)
             const uint32_t empty0 = cluster_addr(smem_addr(empty), 0), empty1 = cluster_addr(smem_addr(empty), 1);
             const uint32_t accf0 = cluster_addr(smem_addr(acc_full), 0), accf1 = cluster_addr(smem_addr(acc_full), 1);
             int k = 0, it = 0;
@@ -746,15 +775,15 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                 // off = 0 or 2 columns (32-row groups) into the first unit
                 const uint32_t off = uint32_t(((t % NT) * kBN % 128) / 32);
                 const int ab = it % NA;
-                if (it >= NA && !mbar_wait(&acc_empty[ab], ((it / NA) - 1) & 1, budget)) {
-                    atomicAdd(&g_wait_timeouts, 1);
+                if (it >= NA && !warp_wait(&acc_empty[ab], ((it / NA) - 1) & 1, budget)) {
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
                 mma::tc_fence_after();
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
-                    if (!mbar_wait(&full[s], (k / ST) & 1, budget) || !mbar_wait(&sf_ready[s], (k / ST) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (!warp_wait(&full[s], (k / ST) & 1, budget) || !warp_wait(&sf_ready[s], (k / ST) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -783,22 +812,22 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
             // every MMA issued has completed before the tensor memory is freed
             umma_commit_pair(cluster_addr(smem_addr(done), 1));
             umma_commit_pair(cluster_addr(smem_addr(done), 0));
-            if (!mbar_wait(done, 0, budget)) atomicAdd(&g_wait_timeouts, 1);
-        } else if (lane == 0) {
+            if (!warp_wait(done, 0, budget) && lane == 0) atomicAdd(&g_wait_timeouts, 1);
+        } else {
             // the peer: the leader's final commit has arrived here too
-            if (!mbar_wait(done, 0, budget)) atomicAdd(&g_wait_timeouts, 1);
+            if (!warp_wait(done, 0, budget) && lane == 0) atomicAdd(&g_wait_timeouts, 1);
         }
     } else if (warp == kCopyWarp) {
-        if (lane == 0 && rank == 0) {
-            // ---------------- scale copies (the leader's one thread): each
+        if (rank == 0) {
+            // ---------------- scale copies (the leader's warp): each
             // CTA's units of the stage to its own tensor memory
             int k = 0, issued = 0;
             bool ok = true;
             for (int t = cid; t < tiles && ok; t += ncl) {
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
-                    if (!mbar_wait(&full[s], (k / ST) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (!warp_wait(&full[s], (k / ST) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -817,7 +846,7 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                     issued = k + 1;
                 }
             }
-            if (issued > 0 && !mbar_wait(&sf_ready[(issued - 1) % ST], ((issued - 1) / ST) & 1, budget))
+            if (issued > 0 && !warp_wait(&sf_ready[(issued - 1) % ST], ((issued - 1) / ST) & 1, budget) && lane == 0)
                 atomicAdd(&g_wait_timeouts, 1);
         }
     } else {
