@@ -22,7 +22,7 @@
 // t = blockIdx.x, + gridDim.x, ...; a k-chunk is CB bytes of codes per row
 // (2 CB elements, one CB-byte swizzle atom; CB / 64 scale units per row
 // group), CB, the ring depth ST and BN being compile-time choices (Cfg).
-//   warp 0     producer: per chunk, TMA loads of the A box {CB x 128 rows}
+//   warp 0     producer (one elected lane issues): per chunk, TMA loads of the A box {CB x 128 rows}
 //              and the B box {CB x BN rows} (CB-byte swizzle; rows and bytes
 //              past the matrix read as zero) and bulk copies of the chunk's
 //              scale units (A: its row group's, B: the tile's two row groups')
@@ -153,6 +153,14 @@ __device__ __forceinline__ void umma_commit_w(uint64_t *bar)
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long budget)
 {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, budget));
+}
+
+// True in the one lane of the (converged) warp that elect.sync picks.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t e;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+    return e != 0;
 }
 
 // Plain (untiled) bulk copy global -> shared, completing on `bar`.
@@ -344,8 +352,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- producer
+        {
+            // ---------------- producer (the whole warp; one elected lane issues)
             int k = 0, filled = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
@@ -354,8 +362,8 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                 const bool b_hi = g0 + 1 < NRa;               // its second row group exists
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
-                    if (k >= ST && !mbar_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (k >= ST && !warp_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -365,21 +373,24 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                     const int u0 = c * C::kUnits;
                     const int nu = Ka - u0 < C::kUnits ? Ka - u0 : C::kUnits;   // units of this chunk, >= 1
                     const uint32_t sfbytes = uint32_t(nu) * kSfUnit;
-                    mbar_expect_tx(&full[s], uint32_t(C::kABytes + C::kBBytes) + sfbytes * (b_hi ? 3u : 2u));
-                    mma::tma_load_2d(st, &a_map, c * C::kCB, mt * kBM, &full[s]);
-                    mma::tma_load_2d(st + C::kABytes, &b_map, c * C::kCB, nt * kBN, &full[s]);
-                    bulk_load(sfa, a_sf + (int64_t(mt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
-                    bulk_load(sfb, b_sf + (int64_t(g0) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
-                    if (b_hi)
-                        bulk_load(sfb + C::kUnits * kSfUnit, b_sf + (int64_t(g0 + 1) * Ka + u0) * kSfUnit, sfbytes,
-                                  &full[s]);
+                    if (elect_one()) {
+                        mbar_expect_tx(&full[s], uint32_t(C::kABytes + C::kBBytes) + sfbytes * (b_hi ? 3u : 2u));
+                        mma::tma_load_2d(st, &a_map, c * C::kCB, mt * kBM, &full[s]);
+                        mma::tma_load_2d(st + C::kABytes, &b_map, c * C::kCB, nt * kBN, &full[s]);
+                        bulk_load(sfa, a_sf + (int64_t(mt) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
+                        bulk_load(sfb, b_sf + (int64_t(g0) * Ka + u0) * kSfUnit, sfbytes, &full[s]);
+                        if (b_hi)
+                            bulk_load(sfb + C::kUnits * kSfUnit, b_sf + (int64_t(g0 + 1) * Ka + u0) * kSfUnit,
+                                      sfbytes, &full[s]);
+                    }
+                    __syncwarp();
                     filled = k + 1;
                 }
             }
             // drain: the copies issued have landed before the CTA may exit
             for (int kk = (filled > ST ? filled - ST : 0); kk < filled; ++kk)
-                if (!mbar_wait(&full[kk % ST], (kk / ST) & 1, budget)) {
-                    atomicAdd(&g_wait_timeouts, 1);
+                if (!warp_wait(&full[kk % ST], (kk / ST) & 1, budget)) {
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
         }
@@ -716,8 +727,8 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- producer (both CTAs)
+        {
+            // ---------------- producer (both CTAs; the whole warp, one elected lane issues)
             const uint32_t lead_full = cluster_addr(smem_addr(full), 0);
             int k = 0, filled = 0;
             bool ok = true;
@@ -729,8 +740,8 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                 const int gb = nt * kBN / 128;               // the tile's first B row group
                 for (int c = 0; c < KC; ++c, ++k) {
                     const int s = k % ST;
-                    if (k >= ST && !mbar_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (k >= ST && !warp_wait(&empty[s], ((k / ST) - 1) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         ok = false;
                         break;
                     }
@@ -738,12 +749,15 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                     uint8_t *sfa = st + C::kABytes + C::kBBytes;
                     uint8_t *sfb = sfa + C::kSfaBytes;
                     const uint32_t bar = lead_full + uint32_t(s) * 8;
-                    if (rank == 0) mbar_expect_tx(&full[s], C::kPairTx);
-                    tma_load_2d_pair(st, &a_map, c * C::kCB, row_a, bar);
-                    tma_load_2d_pair(st + C::kABytes, &b_map, c * C::kCB, row_b, bar);
-                    // scale units 2c, 2c + 1 = 256-byte rows 4c .. 4c + 3 of the row group
-                    tma_load_3d_pair(sfa, &asf_map, 0, 4 * c, ga, bar);
-                    tma_load_3d_pair(sfb, &bsf_map, 0, 4 * c, gb, bar);
+                    if (elect_one()) {
+                        if (rank == 0) mbar_expect_tx(&full[s], C::kPairTx);
+                        tma_load_2d_pair(st, &a_map, c * C::kCB, row_a, bar);
+                        tma_load_2d_pair(st + C::kABytes, &b_map, c * C::kCB, row_b, bar);
+                        // scale units 2c, 2c + 1 = 256-byte rows 4c .. 4c + 3 of the row group
+                        tma_load_3d_pair(sfa, &asf_map, 0, 4 * c, ga, bar);
+                        tma_load_3d_pair(sfb, &bsf_map, 0, 4 * c, gb, bar);
+                    }
+                    __syncwarp();
                     filled = k + 1;
                 }
             }
@@ -753,13 +767,13 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
             const int k0 = filled > ST ? filled - ST : 0;
             if (rank == 0)
                 for (int kk = k0; kk < filled; ++kk)
-                    if (!mbar_wait(&full[kk % ST], (kk / ST) & 1, budget)) {
-                        atomicAdd(&g_wait_timeouts, 1);
+                    if (!warp_wait(&full[kk % ST], (kk / ST) & 1, budget)) {
+                        if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                         break;
                     }
             for (int kk = k0; kk < filled; ++kk)
-                if (!mbar_wait(&empty[kk % ST], (kk / ST) & 1, budget)) {
-                    atomicAdd(&g_wait_timeouts, 1);
+                if (!warp_wait(&empty[kk % ST], (kk / ST) & 1, budget)) {
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1);
                     break;
                 }
         }
