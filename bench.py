@@ -85,7 +85,7 @@ TRAFFIC = {"source_sha": "2f5b27cf4f68040f", "bytes_per_launch": 127422976.0,
 # helper it uses) and the host functions that size and launch it.
 KERNEL_START = "kq_packed_kernel(const uint4 *__restrict__ act"
 LAUNCH_FUNCS = ("int sm_count(", "Geometry pinned_geometry(", "int resident_threads(",
-                "int launch_pinned(const char *fn, KernelId id", "int kq_launch(")
+                "int launch_pinned(const char *fn, KernelId id", "void launch(void (*kernel)", "int kq_launch(")
 
 
 def _function_text(src: str, head: str) -> str:

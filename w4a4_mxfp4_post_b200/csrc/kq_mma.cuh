@@ -246,6 +246,7 @@ kq_mma_kernel(const __grid_constant__ CUtensorMap act_map, const __grid_constant
               const float4 *__restrict__ factors, int shared, uint8_t *__restrict__ scales,
               float4 *__restrict__ y_out, int64_t M, int nb, long long budget)
 {
+    pdl_wait();
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;

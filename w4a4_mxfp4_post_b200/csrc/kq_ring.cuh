@@ -194,6 +194,7 @@ kq_ring_kernel(const __grid_constant__ CUtensorMap act_map, const uint4 *__restr
                const float *__restrict__ factors, int shared, uint4 *__restrict__ codes,
                uint8_t *__restrict__ scales, int64_t nblocks, int nb, long long budget)
 {
+    pdl_wait();
     using C = Cfg<P>;
     extern __shared__ uint8_t smem_dyn[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));

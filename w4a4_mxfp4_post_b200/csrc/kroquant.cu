@@ -27,6 +27,7 @@
 #include <cstdio>
 #include <cmath>
 #include <cstring>
+#include <utility>
 
 #include "kroquant.h"
 
@@ -212,12 +213,20 @@ __device__ __forceinline__ void load_block(const uint4 *__restrict__ act, int64_
 // ---------------------------------------------------------------------------
 enum class KqOut { kCodes, kF32 };
 
+// Every kernel of the library begins with griddepcontrol.wait, and every
+// launch allows programmatic stream serialization (launch() below): a kernel
+// may then be scheduled while its predecessor on the stream finishes, but it
+// touches no memory before that predecessor has completed and its writes are
+// visible.  Launched without the attribute, the wait returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <KqOut OUT>
 __global__ void __launch_bounds__(kThreads)
 kq_butterfly_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ factors, int shared,
                     uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
                     int64_t nblocks, int nb, int64_t T)
 {
+    pdl_wait();
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
     const int j = int(t % nb);
@@ -261,6 +270,7 @@ __global__ void __launch_bounds__(kThreads)
 fold_kernel(const float4 *__restrict__ W, const float4 *__restrict__ factors, int shared,
             float4 *__restrict__ W_out, int64_t nblocks, int nb, int64_t T)
 {
+    pdl_wait();
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
     const int j = int(t % nb);
@@ -642,6 +652,7 @@ kq_packed_kernel(const uint4 *__restrict__ act, const float *__restrict__ params
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, float4 *__restrict__ y_out,
                  int64_t nblocks, int nb, int64_t T)
 {
+    pdl_wait();
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
     SfPos sp{};
@@ -725,6 +736,7 @@ __global__ void __launch_bounds__(kThreads)
 fwht_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks,
             int64_t T, int xstages, float inv_sqrt_h)
 {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t t0 = int64_t(blockIdx.x) * kThreads + (threadIdx.x & ~31);   // the warp's first thread
     for (int64_t g0 = t0; g0 < nblocks; g0 += T) {                            // warp-uniform walk
@@ -772,6 +784,7 @@ __global__ void __launch_bounds__(kThreads)
 sq_packed_kernel(const uint4 *__restrict__ act, const float4 *__restrict__ mult, uint4 *__restrict__ codes,
                  uint8_t *__restrict__ scales, int64_t nblocks, int nb, int64_t T)
 {
+    pdl_wait();
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= T || t >= nblocks) return;
     const int j = int(t % nb);
@@ -815,6 +828,7 @@ __global__ void __launch_bounds__(kThreads)
 mx_packed_kernel(const uint4 *__restrict__ act, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
                  int64_t nblocks, int64_t T)
 {
+    pdl_wait();
     const int64_t t = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (t >= nblocks) return;
     int64_t gi = t;
@@ -1017,6 +1031,7 @@ kq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const uint4 *__res
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb,
                  long long budget, int issue_copies)
 {
+    pdl_wait();
     const StagedRing r = staged_setup();
     const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
     if (threadIdx.x >= kConsumers) {
@@ -1057,6 +1072,7 @@ sq_staged_kernel(const __grid_constant__ CUtensorMap act_map, const float4 *__re
                  uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int64_t nblocks, int nb, long long budget,
                  int issue_copies)
 {
+    pdl_wait();
     const StagedRing r = staged_setup();
     const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
     if (threadIdx.x >= kConsumers) {
@@ -1094,6 +1110,7 @@ __global__ void __launch_bounds__(kStagedThreads, 2)
 mx_staged_kernel(const __grid_constant__ CUtensorMap act_map, uint4 *__restrict__ codes,
                  uint8_t *__restrict__ scales, int64_t nblocks, long long budget, int issue_copies)
 {
+    pdl_wait();
     const StagedRing r = staged_setup();
     const int64_t nchunks = (nblocks + kStageRows - 1) / kStageRows;
     if (threadIdx.x >= kConsumers) {
@@ -1134,6 +1151,7 @@ __global__ void __launch_bounds__(kThreads)
 mx_dequantize_kernel(const uint4 *__restrict__ codes, const uint8_t *__restrict__ scales, float4 *__restrict__ out,
                      int64_t nblocks)
 {
+    pdl_wait();
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < nblocks; g += stride) {
         const uint4 c = __ldg(codes + g);
@@ -1163,6 +1181,7 @@ __global__ void __launch_bounds__(kThreads)
 mx_f32_kernel(const float4 *__restrict__ x, uint4 *__restrict__ codes, uint8_t *__restrict__ scales,
               int64_t nblocks, int nb)
 {
+    pdl_wait();
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < nblocks; g += stride) {
         float v[32];
@@ -1195,6 +1214,7 @@ mx_f32_kernel(const float4 *__restrict__ x, uint4 *__restrict__ codes, uint8_t *
 __global__ void __launch_bounds__(kThreads)
 sf_relayout_kernel(const uint8_t *__restrict__ scales, uint8_t *__restrict__ sf, int64_t n, int nb)
 {
+    pdl_wait();
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t g = int64_t(blockIdx.x) * kThreads + threadIdx.x; g < n; g += stride) {
         SfPos sp = sf_pos(g, g + 1, nb);
@@ -1274,6 +1294,7 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
                int64_t rows_per, float eps, const float *__restrict__ factors, int shared, uint4 *__restrict__ codes,
                uint8_t *__restrict__ scales, int64_t M, int nb)
 {
+    pdl_wait();
     extern __shared__ __align__(16) float tab[];   // [nb][kNormSlot]
     // coefficient table (every column of the row, computed once per CTA)
     for (int j = threadIdx.x; j < nb; j += blockDim.x) {
@@ -1406,6 +1427,7 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
                     int64_t rows_per, float eps, const float *__restrict__ factors, int shared,
                     uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int nb, int cps, int nbuf)
 {
+    pdl_wait();
     extern __shared__ float4 smf[];
     float4 *tab = smf;                                                        // [nb][kNormRowSlot]
     uint4 *rowbuf = reinterpret_cast<uint4 *>(smf + size_t(nb) * kNormRowSlot);   // [warps][nbuf][nb * 4]
@@ -1623,6 +1645,7 @@ norm_kq_cols_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
                     int64_t rows_per, float eps, const float *__restrict__ factors, int shared,
                     uint4 *__restrict__ codes, uint8_t *__restrict__ scales, int nb, int cps)
 {
+    pdl_wait();
     static_assert(DEPTH % 2 == 0 && DEPTH >= 2, "the ring holds whole pairs of rows");
     extern __shared__ float4 smc[];
     const int nt = int(blockDim.x);                                        // threads = nb rounded up to 32
@@ -1918,6 +1941,24 @@ int resident_threads(KernelId id, const void *fn, int64_t *out)
     }
     *out = int64_t(sms) * c * kThreads;
     return KQ_OK;
+}
+
+// Launch with programmatic stream serialization (see pdl_wait); a launch
+// error is left for launch_check, as with the <<< >>> form.
+template <typename... P, typename... A>
+void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, A &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
 int launch_check(const char *what)
@@ -2217,7 +2258,7 @@ int ring_launch(const char *fn, KernelId id, const void *act, const float *facto
     if ((rc = smem_prepare(id, reinterpret_cast<const void *>(k), C::kSmem)) != KQ_OK) return rc;
     CUtensorMap map;
     if ((rc = encode_act_map(act, nblocks, &map, C::kBoxRows)) != KQ_OK) return rc;
-    k<<<grid, C::kThreads, C::kSmem, stream>>>(map, static_cast<const uint4 *>(act), factors, shared,
+    launch(k, grid, C::kThreads, C::kSmem, stream, map, static_cast<const uint4 *>(act), factors, shared,
                                                reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb),
                                                kWaitBudget);
     *launched = true;
@@ -2263,14 +2304,14 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
             auto k = mma::kq_mma_kernel<KqOut::kF32>;
             if ((rc = mma_prepare(kKqMmaF32, reinterpret_cast<const void *>(k))) != KQ_OK) return rc;
             // the codes map is unused by the fp32 export; any valid map will do
-            k<<<grid, mma::kThreads, mma::kSmem, stream>>>(map, map, f4, shared, nullptr,
+            launch(k, grid, mma::kThreads, mma::kSmem, stream, map, map, f4, shared, nullptr,
                                                            reinterpret_cast<float4 *>(y), M, int(nb4), kWaitBudget);
         } else {
             CUtensorMap cmap;
             if ((rc = encode_codes_map(codes, M, d, &cmap)) != KQ_OK) return rc;
             auto k = mma::kq_mma_kernel<KqOut::kCodes>;
             if ((rc = mma_prepare(kKqMma, reinterpret_cast<const void *>(k))) != KQ_OK) return rc;
-            k<<<grid, mma::kThreads, mma::kSmem, stream>>>(map, cmap, f4, shared, scales, nullptr, M, int(nb4),
+            launch(k, grid, mma::kThreads, mma::kSmem, stream, map, cmap, f4, shared, scales, nullptr, M, int(nb4),
                                                            kWaitBudget);
         }
         return launch_check(fn);
@@ -2289,30 +2330,30 @@ int kq_launch(const char *fn, int variant, const void *act, const float *factors
         int64_t resident = 0;
         if ((rc = staged_prepare(kKqStaged, reinterpret_cast<const void *>(kq_staged_kernel), &resident)) != KQ_OK)
             return rc;
-        kq_staged_kernel<<<staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream>>>(
+        launch(kq_staged_kernel, staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream,
             map, a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nblocks, int(nb), kWaitBudget, 1);
     } else if (variant == 1) {
         if (f32) {
             auto k = kq_butterfly_kernel<KqOut::kF32>;
             if ((rc = launch_pinned(fn, kKqDirectF32, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
+            launch(k, geo.grid, kThreads, 0, stream, a, f, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
                                                  nblocks, int(nb), geo.T);
         } else {
             auto k = kq_butterfly_kernel<KqOut::kCodes>;
             if ((rc = launch_pinned(fn, kKqDirect, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
+            launch(k, geo.grid, kThreads, 0, stream, a, f, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
                                                  nblocks, int(nb), geo.T);
         }
     } else {
         if (f32) {
             auto k = kq_packed_kernel<KqOut::kF32>;
             if ((rc = launch_pinned(fn, kKqPackedF32, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, factors, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
+            launch(k, geo.grid, kThreads, 0, stream, a, factors, shared, nullptr, nullptr, reinterpret_cast<float4 *>(y),
                                                  nblocks, int(nb), geo.T);
         } else {
             auto k = kq_packed_kernel<KqOut::kCodes>;
             if ((rc = launch_pinned(fn, kKqPacked, k, M, nb, &geo)) != KQ_OK) return rc;
-            k<<<geo.grid, kThreads, 0, stream>>>(a, factors, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
+            launch(k, geo.grid, kThreads, 0, stream, a, factors, shared, reinterpret_cast<uint4 *>(codes), scales, nullptr,
                                                  nblocks, int(nb), geo.T);
         }
     }
@@ -2367,7 +2408,7 @@ int gemm_launch_out(const GemmArgs &g, const CUtensorMap &amap, const CUtensorMa
         if (e != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         if (dev >= 0 && dev < kMaxDevices) g_gemm_smem_set<C, F32>[dev].store(1, std::memory_order_release);
     }
-    k<<<grid, gemm::kThreads, C::kSmem, g.stream>>>(amap, bmap, omap, g.a_sf, g.b_sf, g.out, int(g.M), int(g.N),
+    launch(k, grid, gemm::kThreads, C::kSmem, g.stream, amap, bmap, omap, g.a_sf, g.b_sf, g.out, int(g.M), int(g.N),
                                                      int(g.K), kWaitBudget);
     return launch_check("mxf4_gemm");
 }
@@ -2429,7 +2470,7 @@ int gemm_pair_launch_out(const GemmArgs &g, const CUtensorMap *maps, int64_t til
         if (dev >= 0 && dev < kMaxDevices) g_pair_clusters<C, F32>[dev].store(clusters, std::memory_order_release);
     }
     const unsigned grid = 2u * unsigned(tiles < clusters ? tiles : clusters);
-    k<<<grid, gemm::kThreads, C::kSmem, g.stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], g.out, int(g.M),
+    launch(k, grid, gemm::kThreads, C::kSmem, g.stream, maps[0], maps[1], maps[2], maps[3], maps[4], g.out, int(g.M),
                                                      int(g.N), int(g.K), kWaitBudget);
     return launch_check("mxf4_gemm");
 }
@@ -2477,7 +2518,7 @@ int cols_launch(const char *fn, const void *h_bf16, const float *gamma, const fl
     if (cps > rows_per) cps = rows_per;
     if (cps < 1) cps = 1;
     if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
-    k<<<unsigned(cps * nsamples), nt, smem, stream>>>(static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps,
+    launch(k, unsigned(cps * nsamples), nt, smem, stream, static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps,
                                                       factors, shared ? 1 : 0, reinterpret_cast<uint4 *>(out_codes),
                                                       out_scales, nb, int(cps));
     return launch_check(fn);
@@ -2562,7 +2603,7 @@ int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const fl
             if (cps < 1) cps = 1;
             if (cps * nsamples >= (int64_t(1) << 31)) cps = ((int64_t(1) << 31) - 1) / nsamples;
             const size_t smem_r = tab + size_t(warps) * nbuf * row;
-            norm_kq_rows_kernel<SF><<<unsigned(cps * nsamples), 32 * warps, smem_r, stream>>>(
+            launch(norm_kq_rows_kernel<SF>, unsigned(cps * nsamples), 32 * warps, smem_r, stream,
                 static_cast<const uint4 *>(h_bf16), gamma, beta, rows_per, eps, factors, shared ? 1 : 0,
                 reinterpret_cast<uint4 *>(out_codes), out_scales, nb, int(cps), nbuf);
             return launch_check(fn);
@@ -2586,7 +2627,7 @@ int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const fl
     int64_t grid = int64_t(sms) * per_sm;
     const int64_t need = (warps_needed + (kThreads / 32) - 1) / (kThreads / 32);
     if (grid > need) grid = need;
-    norm_kq_kernel<SF><<<unsigned(grid), kThreads, smem, stream>>>(
+    launch(norm_kq_kernel<SF>, unsigned(grid), kThreads, smem, stream,
         static_cast<const uint4 *>(h_bf16), gamma, beta, M / nsamples, eps, factors, shared ? 1 : 0,
         reinterpret_cast<uint4 *>(out_codes), out_scales, M, nb);
     return launch_check(fn);
@@ -2667,14 +2708,14 @@ int sq_quantize_variant(int variant, const void *act_bf16, const float *mult, ui
         int64_t resident = 0;
         if ((rc = staged_prepare(kSqStaged, reinterpret_cast<const void *>(sq_staged_kernel), &resident)) != KQ_OK)
             return rc;
-        sq_staged_kernel<<<staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream>>>(
+        launch(sq_staged_kernel, staged_grid(nblocks, nb, resident), kStagedThreads, kStagedSmem, stream,
             map, reinterpret_cast<const float4 *>(mult), reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
             int(nb), kWaitBudget, 1);
         return launch_check(fn);
     }
     Geometry geo;
     if ((rc = launch_pinned(fn, kSqPacked, sq_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
-    sq_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+    launch(sq_packed_kernel, geo.grid, kThreads, 0, stream, static_cast<const uint4 *>(act_bf16),
                                                         reinterpret_cast<const float4 *>(mult),
                                                         reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
                                                         int(nb), geo.T);
@@ -2700,13 +2741,13 @@ int mx_quantize_variant(int variant, const void *act_bf16, uint8_t *out_codes, u
         if ((rc = staged_prepare(kMxStaged, reinterpret_cast<const void *>(mx_staged_kernel), &resident)) != KQ_OK)
             return rc;
         // any grid works for MX (no per-column state); keep the same sizing
-        mx_staged_kernel<<<staged_grid(nblocks, 1, resident), kStagedThreads, kStagedSmem, stream>>>(
+        launch(mx_staged_kernel, staged_grid(nblocks, 1, resident), kStagedThreads, kStagedSmem, stream,
             map, reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks, kWaitBudget, 1);
         return launch_check(fn);
     }
     Geometry geo;
     if ((rc = launch_pinned(fn, kMxPacked, mx_packed_kernel, M, nb, &geo)) != KQ_OK) return rc;
-    mx_packed_kernel<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+    launch(mx_packed_kernel, geo.grid, kThreads, 0, stream, static_cast<const uint4 *>(act_bf16),
                                                         reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
                                                         geo.T);
     return launch_check(fn);
@@ -2730,7 +2771,7 @@ int kq_quantize_lu(const void *act_bf16, const float *lu_params, int shared, uin
     auto k = kq_packed_kernel<KqOut::kCodes, true>;
     int rc = launch_pinned(fn, kKqLu, k, M, nb, &geo);
     if (rc != KQ_OK) return rc;
-    k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16), lu_params, shared ? 1 : 0,
+    launch(k, geo.grid, kThreads, 0, stream, static_cast<const uint4 *>(act_bf16), lu_params, shared ? 1 : 0,
                                          reinterpret_cast<uint4 *>(out_codes), out_scales, nullptr, M * nb, int(nb),
                                          geo.T);
     return launch_check(fn);
@@ -2764,7 +2805,7 @@ int fwht_quantize(const void *act_bf16, int64_t H, uint8_t *out_codes, uint8_t *
     const unsigned grid = unsigned((T + kThreads - 1) / kThreads);
     // 1/sqrt(H) rounded to fp32: H = 2^(5 + s); sqrt(2^n) = 2^(n/2) * (sqrt 2 if n odd)
     const double inv = 1.0 / std::sqrt(double(H));
-    fwht_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16),
+    launch(fwht_kernel, grid, kThreads, 0, stream, static_cast<const uint4 *>(act_bf16),
                                                reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks,
                                                int64_t(grid) * kThreads, xstages, float(inv));
     return launch_check(fn);
@@ -2784,7 +2825,7 @@ int kq_inverse_f32(const float *y, const float *factors, int shared, float *x_ou
     Geometry geo;
     int rc = launch_pinned(fn, kInverse, fold_kernel<true>, M, nb, &geo);
     if (rc != KQ_OK) return rc;
-    fold_kernel<true><<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(y),
+    launch(fold_kernel<true>, geo.grid, kThreads, 0, stream, reinterpret_cast<const float4 *>(y),
                                                          reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
                                                          reinterpret_cast<float4 *>(x_out), M * nb, int(nb), geo.T);
     return launch_check(fn);
@@ -2803,7 +2844,7 @@ int mx_dequantize(const uint8_t *codes, const uint8_t *scales, float *out, int64
     int rc = resident_threads(kDequant, reinterpret_cast<const void *>(mx_dequantize_kernel), &target);
     if (rc != KQ_OK) return rc;
     int64_t T = target < nblocks ? target : nblocks;
-    mx_dequantize_kernel<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(
+    launch(mx_dequantize_kernel, unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream,
         reinterpret_cast<const uint4 *>(codes), scales, reinterpret_cast<float4 *>(out), nblocks);
     return launch_check(fn);
 }
@@ -2849,7 +2890,7 @@ int kq_quantize_sf(const void *act_bf16, const float *factors, int shared, uint8
     Geometry geo;
     auto k = kq_packed_kernel<KqOut::kCodes, false, true>;
     if ((rc = launch_pinned(fn, kKqPackedSf, k, M, nb, &geo)) != KQ_OK) return rc;
-    k<<<geo.grid, kThreads, 0, stream>>>(static_cast<const uint4 *>(act_bf16), factors, shared ? 1 : 0,
+    launch(k, geo.grid, kThreads, 0, stream, static_cast<const uint4 *>(act_bf16), factors, shared ? 1 : 0,
                                          reinterpret_cast<uint4 *>(out_codes), out_sf, nullptr, M * nb, int(nb),
                                          geo.T);
     return launch_check(fn);
@@ -2872,7 +2913,7 @@ int mx_quantize_f32(const float *x, uint8_t *out_codes, uint8_t *out_scales, int
     if ((rc = resident_threads(sf ? kMxF32Sf : kMxF32, reinterpret_cast<const void *>(k), &target)) != KQ_OK)
         return rc;
     const int64_t T = target < nblocks ? target : nblocks;
-    k<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(
+    launch(k, unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream,
         reinterpret_cast<const float4 *>(x), reinterpret_cast<uint4 *>(out_codes), out_scales, nblocks, int(nb));
     return launch_check(fn);
 }
@@ -2890,7 +2931,7 @@ int mx_scales_to_sf(const uint8_t *scales, uint8_t *out_sf, int64_t M, int64_t d
     int rc = resident_threads(kSfRelayout, reinterpret_cast<const void *>(sf_relayout_kernel), &target);
     if (rc != KQ_OK) return rc;
     const int64_t T = target < n ? target : n;
-    sf_relayout_kernel<<<unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream>>>(scales, out_sf, n,
+    launch(sf_relayout_kernel, unsigned((T + kThreads - 1) / kThreads), kThreads, 0, stream, scales, out_sf, n,
                                                                                           int(d / kBlk));
     return launch_check(fn);
 }
@@ -2966,7 +3007,7 @@ int kq_selftest_bounded_wait(cudaStream_t stream)
     int64_t resident = 0;
     if ((rc = staged_prepare(kMxStaged, reinterpret_cast<const void *>(mx_staged_kernel), &resident)) != KQ_OK)
         return rc;
-    mx_staged_kernel<<<1, kStagedThreads, kStagedSmem, stream>>>(map, static_cast<uint4 *>(dummy),
+    launch(mx_staged_kernel, 1, kStagedThreads, kStagedSmem, stream, map, static_cast<uint4 *>(dummy),
                                                                  static_cast<uint8_t *>(dummy), nblocks, 1LL << 21, 0);
     return launch_check("kq_selftest_bounded_wait");
 }
@@ -2986,7 +3027,7 @@ int kq_fold_weights(const float *W, const float *factors, int shared, float *W_o
     Geometry geo;
     int rc = launch_pinned("kq_fold_weights", kFold, fold_kernel<false>, N, nb, &geo);
     if (rc != KQ_OK) return rc;
-    fold_kernel<false><<<geo.grid, kThreads, 0, stream>>>(reinterpret_cast<const float4 *>(W),
+    launch(fold_kernel<false>, geo.grid, kThreads, 0, stream, reinterpret_cast<const float4 *>(W),
                                                    reinterpret_cast<const float4 *>(factors), shared ? 1 : 0,
                                                    reinterpret_cast<float4 *>(W_out), N * nb, int(nb), geo.T);
     return launch_check("kq_fold_weights");

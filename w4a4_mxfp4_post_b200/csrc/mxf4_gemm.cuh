@@ -302,6 +302,7 @@ mxf4_gemm_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_constan
                  const __grid_constant__ CUtensorMap out_map, const uint8_t *__restrict__ a_sf,
                  const uint8_t *__restrict__ b_sf, void *__restrict__ out, int M, int N, int K, long long budget)
 {
+    pdl_wait();
     constexpr int ST = C::kST;
     constexpr int kBN = C::kBN;
     constexpr bool kStaged = C::kTmaOut && !F32OUT;
@@ -677,6 +678,7 @@ mxf4_gemm_pair_kernel(const __grid_constant__ CUtensorMap a_map, const __grid_co
                       const __grid_constant__ CUtensorMap out_map, void *__restrict__ out, int M, int N, int K,
                       long long budget)
 {
+    pdl_wait();
     constexpr int ST = C::kST;
     constexpr int kBN = C::kBN;
     constexpr int NA = C::kAccBufs;
