@@ -76,7 +76,7 @@ KERNEL_SOURCES = [os.path.join(ROOT, "w4a4_mxfp4_post_b200", "csrc", "kroquant.c
 # largest layer, FLUX 4608 x 12288), from one ncu capture, valid only for the kernel source it was taken
 # on (sha256 prefix of kernel_source_text: the kernel, its helpers and its
 # launch path).  Updated after each capture.
-TRAFFIC = {"source_sha": "2f5b27cf4f68040f", "bytes_per_launch": 127422976.0,
+TRAFFIC = {"source_sha": "8cd74afaa15c5b7a", "bytes_per_launch": 127987968.0,
            "capture": "ncu --set full, kq_packed_kernel, 4608x12288, dram__bytes_read.sum + dram__bytes_write.sum"}
 
 
