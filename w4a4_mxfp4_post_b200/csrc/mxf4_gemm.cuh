@@ -18,27 +18,33 @@
 // x 4 blocks per copy, 32 lanes x 128 bits replicated to the four lane
 // quarters).
 //
-// A CTA owns one SM (persistent) and walks the 128 x BN output tiles
-// t = blockIdx.x, + gridDim.x, ...; a k-chunk is CB bytes of codes per row
-// (2 CB elements, one CB-byte swizzle atom; CB / 64 scale units per row
+// Two kernels: the one-SM form below (configurations 1-6, the default up to
+// 128 rows) and the SM-pair form (configurations 7 and 8, the default above
+// 128 rows), described before mxf4_gemm_pair_kernel.
+//
+// One-SM form.  A CTA owns one SM (persistent) and walks the 128 x BN output
+// tiles t = blockIdx.x, + gridDim.x, ...; a k-chunk is CB bytes of codes per
+// row (2 CB elements, one CB-byte swizzle atom; CB / 64 scale units per row
 // group), CB, the ring depth ST and BN being compile-time choices (Cfg).
-//   warp 0     producer (one elected lane issues): per chunk, TMA loads of the A box {CB x 128 rows}
+// Every issuing role runs its loop on the whole warp with warp-uniform
+// operands, and one elected lane issues.
+//   warp 0     producer: per chunk, TMA loads of the A box {CB x 128 rows}
 //              and the B box {CB x BN rows} (CB-byte swizzle; rows and bytes
 //              past the matrix read as zero) and bulk copies of the chunk's
 //              scale units (A: its row group's, B: the tile's two row groups')
 //              into an ST-stage ring
-//   warp 1     allocates tensor memory; the warp (one elected lane) issues the
-//              chunk's CB / 32 MMAs (only the K=64 steps below K) once the copier has put the
-//              stage's scales in tensor memory, and commits the stage back to
-//              the producer; after a tile's last chunk it commits the
+//   warp 1     allocates tensor memory; issues the chunk's CB / 32 MMAs (only
+//              the K=64 steps below K) once the copier has put the stage's
+//              scales in tensor memory, and commits the stage back to the
+//              producer; after a tile's last chunk it commits the
 //              accumulator.  Where two accumulators fit beside the scale
 //              columns (BN = 192) tiles alternate between them.
-//   warp 10    the scale copier: the warp (one elected lane) copies each landed stage's scale
-//              units to that stage's own tensor-memory columns (so a copy
-//              never waits on MMAs still reading an older stage) and commits
-//              them to the stage's `sf_ready` barrier.  A tcgen05 instruction
-//              holds its issuing thread for tens of cycles, so the copies of
-//              stage s + 1 go out while the MMA thread issues stage s.
+//   warp 10    the scale copier: copies each landed stage's scale units to
+//              that stage's own tensor-memory columns (so a copy never waits
+//              on MMAs still reading an older stage) and commits them to the
+//              stage's `sf_ready` barrier.  A tcgen05 instruction holds its
+//              issuing warp for tens of cycles, so the copies of stage s + 1
+//              go out while the MMA warp issues stage s.
 //   warps 2-9  epilogue: warp w reads accumulator lanes 32 (w % 4) .. +31 (tile
 //              rows) and columns BN/2 ((w - 2) / 4) .. + BN/2 - 1 into
 //              registers and hands the accumulator back at once; then, while
