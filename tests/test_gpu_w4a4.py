@@ -279,3 +279,44 @@ def test_mxf4_gemm_nan_scale_reaches_only_its_row(cuda_device, variant):
     keep = np.arange(M) != 5
     assert np.all(np.isfinite(out[keep]))
     check_gemm(out[keep], D[keep], absd[keep], K, False)
+
+
+def test_back_to_back_launches_see_their_producers_writes(cuda_device):
+    """Every launch allows programmatic dependent launch, and every kernel waits
+    for its predecessor's writes before it touches memory.  Fold -> quantize the
+    weights -> quantize the activation -> product, on one stream with no
+    synchronisation, three times into the same code and scale buffers (which
+    start out holding other bytes): each product must be the oracle's product of
+    the codes its own quantizer wrote, so a kernel that read early, or a
+    quantizer that overwrote codes the previous product still needed, fails."""
+    import torch
+
+    M, N, d = 520, 392, 1152
+    F = synth.factors(d // 32, 8)
+    Fd = dev(F, cuda_device)
+    codes = torch.full((M, d // 2), 0x77, dtype=torch.uint8, device=cuda_device)
+    sf = torch.full((kq.kq_sf_bytes(M, d),), 0x7F, dtype=torch.uint8, device=cuda_device)
+    wcodes = torch.full((N, d // 2), 0x77, dtype=torch.uint8, device=cuda_device)
+    wsf = torch.full((kq.kq_sf_bytes(N, d),), 0x7F, dtype=torch.uint8, device=cuda_device)
+    xs = [synth.activation("pixart", M, d, seed) for seed in range(3)]
+    Ws = [synth.weights(N, d, 10 + seed) for seed in range(3)]
+    xds = [dev_bf16(x, cuda_device) for x in xs]
+    Wds = [dev(W, cuda_device) for W in Ws]
+    torch.cuda.synchronize()
+    outs = []
+    for xd, Wd in zip(xds, Wds):
+        kq.mx_quantize_f32(kq.kq_fold_weights(Wd, Fd), sf_layout=True, out_codes=wcodes, out_scales=wsf)
+        kq.kq_quantize_sf(xd, Fd, out_codes=codes, out_sf=sf)
+        outs.append(kq.mxf4_gemm(codes, sf, wcodes, wsf, out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    for xd, Wd, out in zip(xds, Wds, outs):
+        # the same (deterministic) kernels once more, one at a time
+        wc, ws = kq.mx_quantize_f32(kq.kq_fold_weights(Wd, Fd), sf_layout=True)
+        c, s = kq.kq_quantize_sf(xd, Fd)
+        torch.cuda.synchronize()
+        ca, cb = c.cpu().numpy(), wc.cpu().numpy()
+        sa = gather_rowmajor(s.cpu().numpy(), M, d // 32)
+        sb = gather_rowmajor(ws.cpu().numpy(), N, d // 32)
+        D, absd = oracle.mxf4_gemm(ca, sa, cb, sb, want_absbound=True)
+        check_gemm(out.cpu().numpy(), D, absd, d, False)
+    assert kq.kq_wait_timeouts() == 0
