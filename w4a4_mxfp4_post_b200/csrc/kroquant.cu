@@ -1407,9 +1407,11 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
 // Single-pass form of the fused normalisation + quantizer, used wherever its
 // shared memory fits (the kernel above is the general fallback).  Each CTA
 // owns a contiguous range of rows of one sample; its shared-memory table holds,
-// per column, the transform coefficients (as above) and that sample's 1 + gamma
-// and beta (kNormRowSlot float4, an odd number of 16-byte units; a column in
-// the direct form, which is rare, reloads its raw factors).  Each warp
+// per column, the unit-stage coefficients of K = U' D and that sample's
+// D (1 + gamma) and D beta, the transform's diagonal folded into the
+// modulation (kNormRowSlot float4, an odd number of 16-byte units; a column in
+// the direct form, which is rare, keeps 1 + gamma and beta and reloads its raw
+// factors).  Each warp
 // streams whole rows into a ring of nbuf row buffers with cp.async (every
 // instruction of a warp copies 512 contiguous bytes; the 16-byte piece p of
 // block b lands at b * 64 + 16 (p ^ ((b >> 1) & 3)), so the per-lane block
@@ -1419,7 +1421,7 @@ norm_kq_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma, con
 // second sweep over (x - mu)^2 only where the mean is large against the root
 // mean square), then normalises, modulates, transforms and quantizes every
 // block.
-constexpr int kNormRowSlot = 27;   // 8 D + 2 B/C + 1 (b4, c4, flag) + 8 (1 + gamma) + 8 beta
+constexpr int kNormRowSlot = 19;   // 2 B/C + 1 (b4, c4, flag) + 8 D (1 + gamma) + 8 D beta
 
 template <bool SF>
 __global__ void __launch_bounds__(512, 1)
@@ -1437,25 +1439,61 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
     const int64_t r0 = smp * rows_per + rows_per * part / cps;
     const int64_t r1 = smp * rows_per + rows_per * (part + 1) / cps;
     const int d = nb * kBlk;
+    // The transform in the form K = U' D (as the long-row kernel): each factor
+    // G = [[1, g01 / g11], [g10 / g00, 1]] diag(g00, g11), so D acts first and
+    // folds into the modulation, whose table entry holds D (1 + gamma) and
+    // D beta + 0 (+0 for a zero product: no intermediate is ever -0, and an
+    // exactly cancelling sum comes out +0); the five unit stages of U' follow,
+    // with no D multiply per element.  A column the split does not admit keeps
+    // 1 + gamma and beta and runs the direct form.  Entry layout: [0], [1] the
+    // (b, c) of the stages on bits 0-3, [2] (b, c) of bit 4 and the flag,
+    // [3 + q] D (1 + gamma) and [11 + q] D beta for elements 4q .. 4q + 3.
     for (int j = threadIdx.x; j < nb; j += blockDim.x) {
         float4 g[5];
         load_factors(reinterpret_cast<const float4 *>(factors), shared, j, g);
-        KqFast st;
-        const bool fast = kq_fast_setup(g, st);
-        float4 *e = tab + size_t(j) * kNormRowSlot;
+        float d0[5], d1[5], bk[5], ck[5];
+        bool fast = true;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            e[q] = make_float4(st.DP[2 * q].x, st.DP[2 * q].y, st.DP[2 * q + 1].x, st.DP[2 * q + 1].y);
-        e[8] = make_float4(st.B[0], st.C[0], st.B[1], st.C[1]);
-        e[9] = make_float4(st.B[2], st.C[2], st.B[3], st.C[3]);
-        e[10] = make_float4(st.b4, st.c4, fast ? 1.0f : 0.0f, 0.0f);
+        for (int k = 0; k < 5; ++k) {
+            d0[k] = g[k].x;
+            d1[k] = g[k].w;
+            bk[k] = __fdividef(g[k].y, g[k].w);
+            ck[k] = __fdividef(g[k].z, g[k].x);
+            const float a0 = fabsf(d0[k]), a1 = fabsf(d1[k]);
+            fast &= a0 >= 0x1p-16f && a0 <= 0x1p16f && a1 >= 0x1p-16f && a1 <= 0x1p16f && fabsf(bk[k]) <= 16.0f &&
+                    fabsf(ck[k]) <= 16.0f;
+        }
+        float dd[32];
+        dd[0] = 1.0f;
+#pragma unroll
+        for (int bit = 0; bit < 5; ++bit) {
+            const int k = 4 - bit;
+#pragma unroll
+            for (int i = 0; i < (1 << bit); ++i) {
+                dd[i + (1 << bit)] = dd[i] * d1[k];
+                dd[i] = dd[i] * d0[k];
+            }
+        }
+        float4 *e = tab + size_t(j) * kNormRowSlot;
+        // factor k (G_{k+1}) acts on in-block index bit 4 - k
+        e[0] = make_float4(bk[4], ck[4], bk[3], ck[3]);
+        e[1] = make_float4(bk[2], ck[2], bk[1], ck[1]);
+        e[2] = make_float4(bk[0], ck[0], fast ? 1.0f : 0.0f, 0.0f);
         const float4 *gp = reinterpret_cast<const float4 *>(gamma + smp * d + int64_t(j) * kBlk);
         const float4 *bp = reinterpret_cast<const float4 *>(beta + smp * d + int64_t(j) * kBlk);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const float4 ga = __ldg(gp + q);
-            e[11 + q] = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
-            e[19 + q] = __ldg(bp + q);
+            const float4 ba = __ldg(bp + q);
+            float4 gg = make_float4(1.0f + ga.x, 1.0f + ga.y, 1.0f + ga.z, 1.0f + ga.w);
+            float4 bb = ba;
+            if (fast) {
+                gg = make_float4(dd[4 * q] * gg.x, dd[4 * q + 1] * gg.y, dd[4 * q + 2] * gg.z, dd[4 * q + 3] * gg.w);
+                bb = make_float4(fmaf(dd[4 * q], bb.x, 0.0f), fmaf(dd[4 * q + 1], bb.y, 0.0f),
+                                 fmaf(dd[4 * q + 2], bb.z, 0.0f), fmaf(dd[4 * q + 3], bb.w, 0.0f));
+            }
+            e[3 + q] = gg;
+            e[11 + q] = bb;
         }
     }
     __syncthreads();
@@ -1557,7 +1595,7 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
             const float4 *eq = tab + size_t(jb) * kNormRowSlot;
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-                const float4 ga = eq[11 + q4], gb = eq[15 + q4], ba = eq[19 + q4], bb = eq[23 + q4];
+                const float4 ga = eq[3 + q4], gb = eq[7 + q4], ba = eq[11 + q4], bb = eq[15 + q4];
                 const float g_lo[4] = {ga.x, ga.y, ga.z, ga.w}, g_hi[4] = {gb.x, gb.y, gb.z, gb.w};
                 const float b_lo[4] = {ba.x, ba.y, ba.z, ba.w}, b_hi[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
@@ -1567,23 +1605,17 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
                     p[i2] = __ffma2_rn(t, make_float2(g_lo[e], g_hi[e]), make_float2(b_lo[e], b_hi[e]));
                 }
             }
-            const float4 c4q = eq[10];
+            const float4 c4q = eq[2];
             if (c4q.z != 0.0f) {
-                const float4 c01 = eq[8], c23 = eq[9];
+                const float4 c01 = eq[0], c23 = eq[1];
                 unit_stage2<1>(p, bcast(c01.x), bcast(c01.y));
                 unit_stage2<2>(p, bcast(c01.z), bcast(c01.w));
                 unit_stage2<4>(p, bcast(c23.x), bcast(c23.y));
                 unit_stage2<8>(p, bcast(c23.z), bcast(c23.w));
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 dd = eq[q];   // (D_2q, D_2q+16, D_2q+1, D_2q+17)
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int i2 = 2 * q + h2;
-                        const float lo = p[i2].x, hi = p[i2].y;
-                        const float2 dp = h2 ? make_float2(dd.z, dd.w) : make_float2(dd.x, dd.y);
-                        p[i2] = __ffma2_rn(make_float2(fmaf(c4q.x, hi, lo), fmaf(c4q.y, lo, hi)), dp, plus_zero2());
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    const float lo = p[i].x, hi = p[i].y;
+                    p[i] = make_float2(fmaf(c4q.x, hi, lo), fmaf(c4q.y, lo, hi));
                 }
             } else {   // rare: the raw factors, from L1
                 float4 g[5];
@@ -2581,7 +2613,7 @@ int norm_launch(const char *fn, const void *h_bf16, const float *gamma, const fl
             if (e2 != cudaSuccess) return fail(KQ_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e2));
             // fewer than 4 row buffers per CTA would leave the SM nearly idle: the
             // fallback kernel is then faster
-            const int cfg[7][2] = {{16, 1}, {8, 2}, {12, 1}, {4, 2}, {8, 1}, {2, 2}, {4, 1}};
+            const int cfg[8][2] = {{16, 2}, {16, 1}, {8, 2}, {12, 1}, {4, 2}, {8, 1}, {2, 2}, {4, 1}};
             for (const auto &c : cfg) {
                 const size_t smem_r = tab + size_t(c[0]) * c[1] * row;
                 if (smem_r > kNormRowsSmemMax) continue;
