@@ -1583,8 +1583,12 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m2 += __shfl_xor_sync(0xffffffffu, m2, off);
         }
-        const float inv = 1.0f / sqrtf(m2 / float(d) + eps);
+        // x / sigma - mu / sigma as one FMA (the product x / sigma is exact inside
+        // it, so the result differs from (x - mu) / sigma by one rounding of
+        // mu / sigma), as in the long-row kernel
+        const float inv = __frsqrt_rn(fmaf(m2, 1.0f / float(d), eps));
         const float2 iv = make_float2(inv, inv);
+        const float2 off = make_float2(-mu * inv, -mu * inv);
         // ---- normalise, modulate, transform, quantize
         for (int jb = lane; jb < nb; jb += 32) {
             uint4 raw[4];
@@ -1601,7 +1605,7 @@ norm_kq_rows_kernel(const uint4 *__restrict__ h, const float *__restrict__ gamma
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int i2 = 4 * q4 + e;
-                    const float2 t = __fmul2_rn(__fadd2_rn(p[i2], nmu), iv);
+                    const float2 t = __ffma2_rn(p[i2], iv, off);
                     p[i2] = __ffma2_rn(t, make_float2(g_lo[e], g_hi[e]), make_float2(b_lo[e], b_hi[e]));
                 }
             }
