@@ -39,3 +39,25 @@ def test_every_mode_is_offered_on_the_command_line():
         assert mode in out
     for flag in ("--shapes", "--reps", "--kernels", "--launches"):
         assert flag in out
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the CPU oracle on a bounded sample of the
+    same workload and prints one JSON line with the contract's keys (no GPU)."""
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, check=True, timeout=600)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
